@@ -1,0 +1,214 @@
+/*
+ * sigattn -- sigmoid attention over padded variable-length batches, sm_100a (B200).
+ *
+ * C ABI of libsigattn.so.  Plain pointers and sizes only; no framework types.
+ *
+ * What it computes (per batch b, head h, query row i with key set J(i)):
+ *     s_ij = scale * (q_i . k_j) + bias_i
+ *     SIGMOID   o_i = sum_{j in J(i)} sigma(s_ij) v_j
+ *     SOFTMAX   o_i = sum_j exp(s_ij) v_j / sum_j exp(s_ij)
+ *     SOFTMAX1  o_i = sum_j exp(s_ij) v_j / (1 + sum_j exp(s_ij))
+ * Sigmoid attention with b = -log(n): "Better Models, Faster Training: Sigmoid
+ * Attention for single-cell Foundation Models", section 2A; its backward with
+ * sigma' = sigma (1 - sigma) and no row-sum term: same page, section 2B, split into a
+ * dQ kernel and a dK/dV kernel with sigma recomputed tile by tile: section 2C.
+ * softmax_1: the QuietAttention page, section "Proposition : softmax_1 et
+ * QuietAttention".  Rows with no key, and pad rows, give exactly 0 in every output.
+ *
+ * Tiles.  The attention matrix of each batch entry is cut into 128 x 128 tiles.  A
+ * plan lists the tiles that hold at least one unmasked (query, key) pair ("Binary
+ * Block Masking for FlashAttention", section "Comment ça marche ?"; "Better Models,
+ * Faster Training", section 2C, blocks that are padding on either side are skipped).
+ * Only listed tiles are computed.  A tile is FULL (every pair unmasked, no masking
+ * work) or PARTIAL (it carries a 128 x 128 bitmask).
+ *
+ * Conventions for every call:
+ *   - Tensors Q, K, V, O, dO, dQ, dK, dV are bf16 with layout [B, N, H, d]: d is
+ *     contiguous; the three element strides (batch, token, head) are passed in
+ *     that order.  Every device pointer must be 16-byte aligned and every stride
+ *     a multiple of 8 elements (16 bytes).  Q/O/dO/dQ have N = Nq rows, K/V/dK/dV
+ *     have N = Nk rows.  Supported head dims: d = 64 and d = 128.
+ *   - bias is fp32 [B, Nq] (per query row; row stride 1, batch stride given); NULL
+ *     means 0.  For sigmoid attention the caller fills -log(n), e.g. with
+ *     sigattn_bias_from_counts.
+ *   - Ownership: the caller owns every tensor; a plan owns its own device buffers.
+ *   - Asynchrony: every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) unless its comment says it synchronises.
+ *   - Errors: 0 on success, a negative SIGATTN_ERR_* code otherwise; nothing is
+ *     launched when an argument check fails.  Kernels never trap: a device-side wait
+ *     that runs past its time limit records SIGATTN_ERR_TIMEOUT in a device status
+ *     word, read (and cleared) by sigattn_get_status.
+ */
+#ifndef SIGATTN_H_
+#define SIGATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SIGATTN_TILE 128
+
+#if defined(__GNUC__)
+#define SIGATTN_API __attribute__((visibility("default")))
+#else
+#define SIGATTN_API
+#endif
+
+typedef struct sigattn_plan sigattn_plan;
+typedef void* sigattn_stream; /* cudaStream_t */
+
+enum sigattn_epilogue {
+  SIGATTN_SIGMOID = 0,  /* sigma(s), no normalisation */
+  SIGATTN_SOFTMAX = 1,  /* online softmax (comparison mode) */
+  SIGATTN_SOFTMAX1 = 2  /* online softmax_1: 1 + sum exp in the denominator */
+};
+
+enum sigattn_status {
+  SIGATTN_OK = 0,
+  SIGATTN_ERR_INVALID = -1,     /* null pointer, negative size, bad enum */
+  SIGATTN_ERR_UNSUPPORTED = -2, /* head dim other than 64 / 128, sizes past limits */
+  SIGATTN_ERR_ALIGNMENT = -3,   /* pointer not 16-byte aligned or stride not a multiple of 8 */
+  SIGATTN_ERR_SHAPE = -4,       /* tensor shapes disagree with the plan */
+  SIGATTN_ERR_CUDA = -5,        /* a CUDA runtime / driver call failed */
+  SIGATTN_ERR_TIMEOUT = -6,     /* a device-side bounded wait expired (see sigattn_get_status) */
+  SIGATTN_ERR_NO_DEVICE = -7,   /* no sm_100 device is current */
+  SIGATTN_ERR_NOMEM = -8        /* device allocation failed */
+};
+
+/* Sizes of a plan.  QT = ceil(Nq / 128), KT = ceil(Nk / 128). */
+typedef struct sigattn_plan_sizes {
+  int32_t B, Nq, Nk, QT, KT;
+  int64_t nonempty;     /* listed tiles (FULL + PARTIAL) */
+  int64_t full;         /* FULL tiles */
+  int64_t partial;      /* PARTIAL tiles (each owns 512 uint32 of bitmask) */
+  int64_t grid_total;   /* B * QT * KT: tiles of the padded grid */
+  int32_t rows_nonempty;  /* (b, q-tile) rows with at least one tile */
+  int32_t cols_nonempty;  /* (b, k-tile) columns with at least one tile */
+} sigattn_plan_sizes;
+
+/*
+ * Plan for a padded batch: query i of batch entry b sees key j iff i < n_b and
+ * j < n_b (Nq = Nk = Npad).  d_lengths: device int32 [B], each in [0, Npad].
+ * Builds the tile list on the device; synchronises `stream` once to size the
+ * plan's buffers.  On success *out owns device memory until sigattn_plan_destroy.
+ * Errors: INVALID (null, B < 1, Npad < 1), UNSUPPORTED (B * QT * KT > 2^28),
+ * CUDA, NOMEM.  Lengths outside [0, Npad] are clamped into it.
+ */
+SIGATTN_API int sigattn_plan_from_lengths(const int32_t* d_lengths, int B, int Npad, sigattn_stream stream,
+                              sigattn_plan** out);
+
+/*
+ * Plan for an element mask: d_mask is device uint8 [B, Nq, Nk], nonzero = attend;
+ * element (b, i, j) at d_mask[b * stride_b + i * stride_q + j].  The mask is shared by
+ * all heads.  Reads the mask once to classify blocks and once more for the PARTIAL
+ * blocks' bitmasks.  Synchronises `stream` once.  Errors as for the lengths plan.
+ */
+SIGATTN_API int sigattn_plan_from_mask(const uint8_t* d_mask, int B, int Nq, int Nk, int64_t stride_b,
+                           int64_t stride_q, sigattn_stream stream, sigattn_plan** out);
+
+/* Fills *sizes (host struct).  No device work. */
+SIGATTN_API int sigattn_plan_get_sizes(const sigattn_plan* plan, sigattn_plan_sizes* sizes);
+
+/*
+ * Copies the tile list to HOST buffers (any may be NULL to skip it); synchronises.
+ *   row_ptr  int32 [B*QT + 1]  CSR offsets by q-tile row r = b*QT + qt
+ *   col_idx  int32 [nonempty]  k-tile of each entry, ascending within a row
+ *   kind     uint8 [nonempty]  1 = FULL, 2 = PARTIAL
+ *   pidx     int32 [nonempty]  bitmask number of a PARTIAL entry (CSR order), -1 if FULL
+ *   colT_ptr int32 [B*KT + 1]  CSC offsets by k-tile column c = b*KT + kt
+ *   rowT_idx int32 [nonempty]  q-tile of each CSC entry, ascending within a column
+ *   csc_map  int32 [nonempty]  CSR index of each CSC entry
+ *   bits     uint32 [partial * 512]  bit (k % 32) of word (q*4 + k/32) = mask(qt*128+q, kt*128+k)
+ */
+SIGATTN_API int sigattn_plan_export(const sigattn_plan* plan, int32_t* row_ptr, int32_t* col_idx,
+                        uint8_t* kind, int32_t* pidx, int32_t* colT_ptr, int32_t* rowT_idx,
+                        int32_t* csc_map, uint32_t* bits);
+
+/*
+ * Copies the two work lists to HOST buffers (either may be NULL); synchronises.
+ *   row_work int32 [B*QT]  every q-tile row r, ordered by tile count descending, ties by r
+ *   col_work int32 [B*KT]  every k-tile column c, ordered the same way
+ * Rows / columns with no tile come last.  Counts past 4094 are ordered as equal.
+ */
+SIGATTN_API int sigattn_plan_export_work(const sigattn_plan* plan, int32_t* row_work, int32_t* col_work);
+
+/* Releases the plan's device memory.  Safe on NULL.  The caller must ensure no
+ * kernel that uses the plan is still running. */
+SIGATTN_API void sigattn_plan_destroy(sigattn_plan* plan);
+
+/*
+ * bias[i] = -log(counts[i]) for counts[i] > 0, else 0 (b = -log(n) of "Better Models,
+ * Faster Training", section 2A; counts[i] is the n of query row i: its sequence's
+ * valid length, or its document's length).  Device int32 in, device fp32 out, n items.
+ */
+SIGATTN_API int sigattn_bias_from_counts(const int32_t* d_counts, int64_t n, float* d_bias,
+                             sigattn_stream stream);
+
+/*
+ * Forward.  O[b, i, h, :] for every b < B, i < Nq, h < H (pad rows and rows with no key
+ * are written as 0).  lse: fp32 [B, H, Nq] natural-log normaliser of each row
+ * (log sum exp, or log(1 + sum exp) for SOFTMAX1; -inf for a SOFTMAX row with no key);
+ * required for SOFTMAX / SOFTMAX1 (the backward reads it), ignored for SIGMOID (may be
+ * NULL).  scale is usually 1/sqrt(d).
+ * Errors: INVALID, UNSUPPORTED (d), ALIGNMENT, CUDA.
+ */
+SIGATTN_API int sigattn_fwd(const sigattn_plan* plan, int epilogue, int H, int d, float scale,
+                const void* q, const int64_t q_strides[3],
+                const void* k, const int64_t k_strides[3],
+                const void* v, const int64_t v_strides[3],
+                const float* bias, int64_t bias_stride_b,
+                void* o, const int64_t o_strides[3],
+                float* lse, sigattn_stream stream);
+
+/*
+ * Backward of L = sum(dO * O): writes dQ, dK, dV (bf16, fp32 accumulation; pad rows 0).
+ * Two kernels, no atomics: a dK/dV kernel walks each k-tile column of the plan, a dQ
+ * kernel walks each q-tile row; both recompute the attention weights tile by tile.
+ * SOFTMAX / SOFTMAX1 also need o, lse (from sigattn_fwd) and workspace: fp32
+ * [B * H * Nq] for D_i = dO_i . O_i; SIGMOID ignores o, lse and workspace (may be NULL).
+ * Errors: as sigattn_fwd.
+ */
+SIGATTN_API int sigattn_bwd(const sigattn_plan* plan, int epilogue, int H, int d, float scale,
+                const void* q, const int64_t q_strides[3],
+                const void* k, const int64_t k_strides[3],
+                const void* v, const int64_t v_strides[3],
+                const void* o, const int64_t o_strides[3],
+                const void* dout, const int64_t do_strides[3],
+                const float* bias, int64_t bias_stride_b,
+                const float* lse, float* workspace,
+                void* dq, const int64_t dq_strides[3],
+                void* dk, const int64_t dk_strides[3],
+                void* dv, const int64_t dv_strides[3],
+                sigattn_stream stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of the current
+ * device: SIGATTN_OK, or SIGATTN_ERR_TIMEOUT if a kernel's bounded wait expired since the
+ * last call (that kernel's outputs are then undefined), or SIGATTN_ERR_CUDA.
+ */
+SIGATTN_API int sigattn_get_status(sigattn_stream stream);
+
+/* Device-side wait limit in nanoseconds for all kernels of this library on the current
+ * device (default 2e9).  A wait that exceeds it records SIGATTN_ERR_TIMEOUT and the
+ * kernel returns early. */
+SIGATTN_API int sigattn_set_wait_limit_ns(uint64_t ns);
+
+/* Self-test of the bounded wait: launches one CTA that waits on a barrier nothing
+ * arrives at, with a limit of `ns`; the kernel gives up, records SIGATTN_ERR_TIMEOUT and
+ * returns.  Used by the tests of the failure path; never faults or hangs. */
+SIGATTN_API int sigattn_selftest_wait_timeout(uint64_t ns, sigattn_stream stream);
+
+/* Static description of an error code. */
+SIGATTN_API const char* sigattn_error_string(int code);
+
+/* Library version, e.g. 100 for 0.1.0. */
+SIGATTN_API int sigattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SIGATTN_H_ */

@@ -1,0 +1,236 @@
+"""Thin ctypes binding of libsigattn.so (declared in include/sigattn.h).
+
+Argument marshalling only: every step of the attention path runs in the library's
+CUDA kernels.  PyTorch provides device memory and streams.  There is no fallback: if
+the library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsigattn.so")
+
+SIGMOID, SOFTMAX, SOFTMAX1 = 0, 1, 2
+OK = 0
+ERR = {-1: "INVALID", -2: "UNSUPPORTED", -3: "ALIGNMENT", -4: "SHAPE", -5: "CUDA",
+       -6: "TIMEOUT", -7: "NO_DEVICE", -8: "NOMEM"}
+
+
+class SigattnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: sigattn error {code} ({ERR.get(code, '?')}): "
+                         f"{_lib.sigattn_error_string(code).decode()}")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m padded_variable_length_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_p = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_i64 = ctypes.c_int64
+_u64 = ctypes.c_uint64
+_I64x3 = ctypes.c_int64 * 3
+
+
+class PlanSizes(ctypes.Structure):
+    _fields_ = [("B", _i32), ("Nq", _i32), ("Nk", _i32), ("QT", _i32), ("KT", _i32),
+                ("nonempty", _i64), ("full", _i64), ("partial", _i64), ("grid_total", _i64),
+                ("rows_nonempty", _i32), ("cols_nonempty", _i32)]
+
+
+def _sig(name, res, *args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = list(args)
+    return f
+
+
+_sig("sigattn_plan_from_lengths", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, _p, ctypes.POINTER(_p))
+_sig("sigattn_plan_from_mask", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _i64, _i64,
+     _p, ctypes.POINTER(_p))
+_sig("sigattn_plan_get_sizes", ctypes.c_int, _p, ctypes.POINTER(PlanSizes))
+_sig("sigattn_plan_export", ctypes.c_int, _p, _p, _p, _p, _p, _p, _p, _p, _p)
+_sig("sigattn_plan_export_work", ctypes.c_int, _p, _p, _p)
+_sig("sigattn_plan_destroy", None, _p)
+_sig("sigattn_bias_from_counts", ctypes.c_int, _p, _i64, _p, _p)
+_sig("sigattn_fwd", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+     _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _i64, _p, _I64x3, _p, _p)
+_sig("sigattn_bwd", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+     _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _i64, _p, _p,
+     _p, _I64x3, _p, _I64x3, _p, _I64x3, _p)
+_sig("sigattn_get_status", ctypes.c_int, _p)
+_sig("sigattn_set_wait_limit_ns", ctypes.c_int, _u64)
+_sig("sigattn_selftest_wait_timeout", ctypes.c_int, _u64, _p)
+_sig("sigattn_error_string", ctypes.c_char_p, ctypes.c_int)
+_sig("sigattn_version", ctypes.c_int)
+
+lib = _lib
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise SigattnError(rc, what)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _strides(t: torch.Tensor) -> ctypes.Array:
+    if t.dim() != 4 or t.dtype != torch.bfloat16 or t.stride(3) != 1:
+        raise ValueError("expected a bf16 [B, N, H, d] tensor with d contiguous")
+    return _I64x3(t.stride(0), t.stride(1), t.stride(2))
+
+
+class Plan:
+    """A tile plan (owns device buffers; destroyed with the object)."""
+
+    def __init__(self, handle: int):
+        self._h = ctypes.c_void_p(handle)
+
+    @classmethod
+    def from_lengths(cls, lengths: torch.Tensor, npad: int, stream=None) -> "Plan":
+        if lengths.dtype != torch.int32 or not lengths.is_cuda or not lengths.is_contiguous():
+            raise ValueError("lengths must be a contiguous int32 CUDA tensor")
+        h = ctypes.c_void_p()
+        _check(_lib.sigattn_plan_from_lengths(lengths.data_ptr(), lengths.numel(), int(npad),
+                                              _stream(stream), ctypes.byref(h)), "plan_from_lengths")
+        return cls(h.value)
+
+    @classmethod
+    def from_mask(cls, mask: torch.Tensor, stream=None) -> "Plan":
+        if mask.dtype != torch.uint8 or not mask.is_cuda or mask.dim() != 3 or mask.stride(2) != 1:
+            raise ValueError("mask must be a uint8 CUDA tensor [B, Nq, Nk] with Nk contiguous")
+        h = ctypes.c_void_p()
+        B, Nq, Nk = mask.shape
+        _check(_lib.sigattn_plan_from_mask(mask.data_ptr(), B, Nq, Nk, mask.stride(0), mask.stride(1),
+                                           _stream(stream), ctypes.byref(h)), "plan_from_mask")
+        return cls(h.value)
+
+    @property
+    def handle(self):
+        return self._h
+
+    def sizes(self) -> dict:
+        s = PlanSizes()
+        _check(_lib.sigattn_plan_get_sizes(self._h, ctypes.byref(s)), "plan_get_sizes")
+        return {f: getattr(s, f) for f, _ in PlanSizes._fields_}
+
+    def export(self) -> dict:
+        z = self.sizes()
+        rows, cols, nz, npart = z["B"] * z["QT"], z["B"] * z["KT"], z["nonempty"], z["partial"]
+        out = {
+            "row_ptr": np.zeros(rows + 1, np.int32), "col_idx": np.zeros(nz, np.int32),
+            "kind": np.zeros(nz, np.uint8), "pidx": np.zeros(nz, np.int32),
+            "colT_ptr": np.zeros(cols + 1, np.int32), "rowT_idx": np.zeros(nz, np.int32),
+            "csc_map": np.zeros(nz, np.int32), "bits": np.zeros((npart, 512), np.uint32),
+        }
+        ptr = lambda a: a.ctypes.data if a.size else None
+        _check(_lib.sigattn_plan_export(self._h, *(ptr(out[k]) for k in
+                                                   ("row_ptr", "col_idx", "kind", "pidx", "colT_ptr",
+                                                    "rowT_idx", "csc_map", "bits"))), "plan_export")
+        return out
+
+    def export_work(self):
+        z = self.sizes()
+        rw = np.zeros(z["B"] * z["QT"], np.int32)
+        cw = np.zeros(z["B"] * z["KT"], np.int32)
+        _check(_lib.sigattn_plan_export_work(self._h, rw.ctypes.data, cw.ctypes.data), "plan_export_work")
+        return rw, cw
+
+    def close(self):
+        if self._h is not None and self._h.value:
+            _lib.sigattn_plan_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def bias_from_counts(counts: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """b = -log(n) per query row from the int32 counts n (0 where n = 0)."""
+    if counts.dtype != torch.int32 or not counts.is_cuda or not counts.is_contiguous():
+        raise ValueError("counts must be a contiguous int32 CUDA tensor")
+    if out is None:
+        out = torch.empty(counts.shape, dtype=torch.float32, device=counts.device)
+    _check(_lib.sigattn_bias_from_counts(counts.data_ptr(), counts.numel(), out.data_ptr(),
+                                         _stream(stream)), "bias_from_counts")
+    return out
+
+
+def _bias_args(bias):
+    if bias is None:
+        return None, 0
+    if bias.dtype != torch.float32 or bias.dim() != 2 or bias.stride(1) != 1:
+        raise ValueError("bias must be fp32 [B, Nq] with unit row stride")
+    return bias.data_ptr(), bias.stride(0)
+
+
+def fwd(plan: Plan, q, k, v, bias=None, epilogue: int = SIGMOID, scale: Optional[float] = None,
+        out=None, lse=None, stream=None):
+    """O (and the row log-normaliser for the softmax modes) of the planned attention."""
+    B, Nq, H, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if epilogue != SIGMOID and lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    bp, bs = _bias_args(bias)
+    _check(_lib.sigattn_fwd(plan.handle, epilogue, H, d, float(scale),
+                            q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
+                            v.data_ptr(), _strides(v), bp, bs, out.data_ptr(), _strides(out),
+                            lse.data_ptr() if lse is not None else None, _stream(stream)), "fwd")
+    return out, lse
+
+
+def bwd(plan: Plan, q, k, v, o, do, bias=None, epilogue: int = SIGMOID, lse=None,
+        scale: Optional[float] = None, workspace=None, dq=None, dk=None, dv=None, stream=None):
+    """dQ, dK, dV of L = sum(dO * O)."""
+    B, Nq, H, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if epilogue != SIGMOID and workspace is None:
+        workspace = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    bp, bs = _bias_args(bias)
+    o_ptr = o.data_ptr() if o is not None else None
+    o_str = _strides(o) if o is not None else _I64x3(0, 0, 0)
+    _check(_lib.sigattn_bwd(plan.handle, epilogue, H, d, float(scale),
+                            q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
+                            v.data_ptr(), _strides(v), o_ptr, o_str, do.data_ptr(), _strides(do),
+                            bp, bs, lse.data_ptr() if lse is not None else None,
+                            workspace.data_ptr() if workspace is not None else None,
+                            dq.data_ptr(), _strides(dq), dk.data_ptr(), _strides(dk),
+                            dv.data_ptr(), _strides(dv), _stream(stream)), "bwd")
+    return dq, dk, dv
+
+
+def get_status(stream=None) -> int:
+    """Synchronises the stream; returns and clears the device status word (0 or TIMEOUT)."""
+    return _lib.sigattn_get_status(_stream(stream))
+
+
+def set_wait_limit_ns(ns: int):
+    _check(_lib.sigattn_set_wait_limit_ns(int(ns)), "set_wait_limit_ns")
+
+
+def selftest_wait_timeout(ns: int, stream=None):
+    _check(_lib.sigattn_selftest_wait_timeout(int(ns), _stream(stream)), "selftest_wait_timeout")

@@ -1,0 +1,100 @@
+"""GPU tile planner vs the brute-force oracle tile list: bit-exact (CSR, CSC, kinds,
+PARTIAL bitmasks), plus validity of the longest-first work lists."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import tiles as OT
+from padded_variable_length_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+KEYS = ("row_ptr", "col_idx", "kind", "pidx", "colT_ptr", "rowT_idx", "csc_map", "bits")
+
+
+def _compare(plan, ref):
+    got = plan.export()
+    for k in KEYS:
+        assert got[k].shape == ref[k].shape, (k, got[k].shape, ref[k].shape)
+        assert np.array_equal(got[k], ref[k]), f"{k} differs"
+    z = plan.sizes()
+    assert z["nonempty"] == len(ref["col_idx"])
+    assert z["full"] == int((ref["kind"] == 1).sum())
+    assert z["partial"] == ref["bits"].shape[0]
+    rows_cnt = np.diff(ref["row_ptr"])
+    cols_cnt = np.diff(ref["colT_ptr"])
+    assert z["rows_nonempty"] == int((rows_cnt > 0).sum())
+    assert z["cols_nonempty"] == int((cols_cnt > 0).sum())
+    rw, cw = plan.export_work()
+    for work, cnt in ((rw, rows_cnt), (cw, cols_cnt)):
+        assert sorted(work.tolist()) == list(range(len(cnt)))
+        c = np.minimum(cnt[work], 4095)
+        assert np.all(np.diff(c) <= 0), "work list not longest-first"
+        for v in np.unique(c):  # ties keep ascending index (stable)
+            idx = work[c == v]
+            assert np.all(np.diff(idx) > 0)
+
+
+LENGTH_CASES = [
+    ([37, 64, 100, 128], 128),
+    ([0, 1, 128, 129, 256], 300),
+    ([640], 640),
+    ([383, 129], 384),
+    ([0, 0, 0], 5),
+    ([1], 1),
+]
+
+
+@pytest.mark.parametrize("lengths,npad", LENGTH_CASES)
+def test_plan_from_lengths(lengths, npad):
+    from padded_variable_length_b200 import binding as Bd
+    plan = Bd.Plan.from_lengths(torch.tensor(lengths, dtype=torch.int32, device="cuda"), npad)
+    _compare(plan, OT.tile_list_from_lengths(lengths, npad))
+
+
+def test_plan_from_lengths_random():
+    from padded_variable_length_b200 import binding as Bd
+    rng = np.random.default_rng(12)
+    for _ in range(6):
+        npad = int(rng.integers(1, 1500))
+        lengths = rng.integers(0, npad + 1, int(rng.integers(1, 9))).astype(np.int32)
+        plan = Bd.Plan.from_lengths(torch.from_numpy(lengths).cuda(), npad)
+        _compare(plan, OT.tile_list_from_lengths(lengths, npad))
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_plan_workload_lengths(cfg):
+    from padded_variable_length_b200 import binding as Bd
+    w = W.config(cfg)
+    plan = Bd.Plan.from_lengths(torch.from_numpy(w.lengths.astype(np.int32)).cuda(), w.Nq)
+    _compare(plan, OT.tile_list_from_lengths(w.lengths, w.Nq))
+
+
+@pytest.mark.parametrize("shape", [(2, 300, 300), (1, 128, 256), (3, 257, 129), (1, 1, 1)])
+def test_plan_from_random_mask(shape):
+    from padded_variable_length_b200 import binding as Bd
+    rng = np.random.default_rng(sum(shape))
+    m = W.random_mask(rng, *shape, density=0.3, empty_rows=2)
+    plan = Bd.Plan.from_mask(torch.from_numpy(m).cuda())
+    _compare(plan, OT.tile_list(m))
+
+
+def test_plan_from_strided_mask():
+    """A mask that is a view with a padded row stride (not 16-byte aligned rows)."""
+    from padded_variable_length_b200 import binding as Bd
+    rng = np.random.default_rng(77)
+    big = W.random_mask(rng, 2, 260, 301, density=0.5, empty_rows=1)
+    view = torch.from_numpy(big).cuda()[:, :, :290]
+    plan = Bd.Plan.from_mask(view)
+    _compare(plan, OT.tile_list(big[:, :, :290]))
+
+
+def test_plan_packed_documents():
+    from padded_variable_length_b200 import binding as Bd
+    w = W.config(4)
+    plan = Bd.Plan.from_mask(torch.from_numpy(w.mask).cuda())
+    ref = OT.tile_list(w.mask)
+    _compare(plan, ref)
+    z = plan.sizes()
+    pop = int(np.unpackbits(ref["bits"].view(np.uint8)).sum())
+    assert pop + 16384 * z["full"] == w.pairs()
