@@ -184,6 +184,33 @@ SIGATTN_API int sigattn_bwd(const sigattn_plan* plan, int epilogue, int H, int d
                 void* dv, const int64_t dv_strides[3],
                 sigattn_stream stream);
 
+/* Parts of the backward for sigattn_bwd_ex (bit mask). */
+enum sigattn_bwd_parts {
+  SIGATTN_BWD_PREP = 1, /* D_i = dO_i . O_i into workspace (softmax modes only; no-op for SIGMOID) */
+  SIGATTN_BWD_DKDV = 2, /* the dK / dV kernel */
+  SIGATTN_BWD_DQ = 4,   /* the dQ kernel */
+  SIGATTN_BWD_ALL = 7
+};
+
+/*
+ * sigattn_bwd restricted to the parts in `parts` (launched in the order PREP, DKDV, DQ),
+ * so that a caller can time or overlap the two kernels.  DKDV and DQ of the softmax modes
+ * read the workspace that PREP wrote.  Arguments and errors as sigattn_bwd; parts outside
+ * SIGATTN_BWD_ALL give INVALID.
+ */
+SIGATTN_API int sigattn_bwd_ex(const sigattn_plan* plan, int epilogue, int H, int d, float scale,
+                               const void* q, const int64_t q_strides[3],
+                               const void* k, const int64_t k_strides[3],
+                               const void* v, const int64_t v_strides[3],
+                               const void* o, const int64_t o_strides[3],
+                               const void* dout, const int64_t do_strides[3],
+                               const float* bias, int64_t bias_stride_b,
+                               const float* lse, float* workspace,
+                               void* dq, const int64_t dq_strides[3],
+                               void* dk, const int64_t dk_strides[3],
+                               void* dv, const int64_t dv_strides[3],
+                               int parts, sigattn_stream stream);
+
 /*
  * Synchronises `stream`, then returns and clears the device status word of the current
  * device: SIGATTN_OK, or SIGATTN_ERR_TIMEOUT if a kernel's bounded wait expired since the

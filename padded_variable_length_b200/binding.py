@@ -68,6 +68,9 @@ _sig("sigattn_fwd", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, 
 _sig("sigattn_bwd", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
      _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _i64, _p, _p,
      _p, _I64x3, _p, _I64x3, _p, _I64x3, _p)
+_sig("sigattn_bwd_ex", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+     _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _i64, _p, _p,
+     _p, _I64x3, _p, _I64x3, _p, _I64x3, ctypes.c_int, _p)
 _sig("sigattn_get_status", ctypes.c_int, _p)
 _sig("sigattn_set_wait_limit_ns", ctypes.c_int, _u64)
 _sig("sigattn_selftest_wait_timeout", ctypes.c_int, _u64, _p)
@@ -199,9 +202,13 @@ def fwd(plan: Plan, q, k, v, bias=None, epilogue: int = SIGMOID, scale: Optional
     return out, lse
 
 
+BWD_PREP, BWD_DKDV, BWD_DQ, BWD_ALL = 1, 2, 4, 7
+
+
 def bwd(plan: Plan, q, k, v, o, do, bias=None, epilogue: int = SIGMOID, lse=None,
-        scale: Optional[float] = None, workspace=None, dq=None, dk=None, dv=None, stream=None):
-    """dQ, dK, dV of L = sum(dO * O)."""
+        scale: Optional[float] = None, workspace=None, dq=None, dk=None, dv=None, stream=None,
+        parts: int = BWD_ALL):
+    """dQ, dK, dV of L = sum(dO * O) (``parts`` selects PREP / DKDV / DQ)."""
     B, Nq, H, d = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
@@ -213,13 +220,13 @@ def bwd(plan: Plan, q, k, v, o, do, bias=None, epilogue: int = SIGMOID, lse=None
     bp, bs = _bias_args(bias)
     o_ptr = o.data_ptr() if o is not None else None
     o_str = _strides(o) if o is not None else _I64x3(0, 0, 0)
-    _check(_lib.sigattn_bwd(plan.handle, epilogue, H, d, float(scale),
-                            q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
-                            v.data_ptr(), _strides(v), o_ptr, o_str, do.data_ptr(), _strides(do),
-                            bp, bs, lse.data_ptr() if lse is not None else None,
-                            workspace.data_ptr() if workspace is not None else None,
-                            dq.data_ptr(), _strides(dq), dk.data_ptr(), _strides(dk),
-                            dv.data_ptr(), _strides(dv), _stream(stream)), "bwd")
+    _check(_lib.sigattn_bwd_ex(plan.handle, epilogue, H, d, float(scale),
+                               q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
+                               v.data_ptr(), _strides(v), o_ptr, o_str, do.data_ptr(), _strides(do),
+                               bp, bs, lse.data_ptr() if lse is not None else None,
+                               workspace.data_ptr() if workspace is not None else None,
+                               dq.data_ptr(), _strides(dq), dk.data_ptr(), _strides(dk),
+                               dv.data_ptr(), _strides(dv), int(parts), _stream(stream)), "bwd")
     return dq, dk, dv
 
 

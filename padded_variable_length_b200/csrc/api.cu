@@ -26,7 +26,7 @@ int launch_bwd_impl(const sigattn_plan* plan, int epilogue, int H, int d, float 
                     const CUtensorMap& tdo, const TensorDesc& o, const TensorDesc& dout,
                     const float* bias, int64_t bias_sb, const float* lse, float* workspace,
                     const TensorDesc& dq, const TensorDesc& dk, const TensorDesc& dv,
-                    int* status, unsigned long long wait_ns, cudaStream_t stream);
+                    int parts, int* status, unsigned long long wait_ns, cudaStream_t stream);
 
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return SIGATTN_OK;
@@ -181,15 +181,18 @@ extern "C" int sigattn_fwd(const sigattn_plan* plan, int epilogue, int H, int d,
                          status, g_wait_limit_ns.load(), static_cast<cudaStream_t>(s));
 }
 
-extern "C" int sigattn_bwd(const sigattn_plan* plan, int epilogue, int H, int d, float scale,
-                           const void* q, const int64_t q_strides[3], const void* k,
-                           const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
-                           const void* o, const int64_t o_strides[3], const void* dout,
-                           const int64_t do_strides[3], const float* bias, int64_t bias_stride_b,
-                           const float* lse, float* workspace, void* dq,
-                           const int64_t dq_strides[3], void* dk, const int64_t dk_strides[3],
-                           void* dv, const int64_t dv_strides[3], sigattn_stream s) {
+extern "C" int sigattn_bwd_ex(const sigattn_plan* plan, int epilogue, int H, int d, float scale,
+                              const void* q, const int64_t q_strides[3], const void* k,
+                              const int64_t k_strides[3], const void* v,
+                              const int64_t v_strides[3], const void* o,
+                              const int64_t o_strides[3], const void* dout,
+                              const int64_t do_strides[3], const float* bias,
+                              int64_t bias_stride_b, const float* lse, float* workspace, void* dq,
+                              const int64_t dq_strides[3], void* dk, const int64_t dk_strides[3],
+                              void* dv, const int64_t dv_strides[3], int parts,
+                              sigattn_stream s) {
   if (!plan || H < 1 || !std::isfinite(scale)) return SIGATTN_ERR_INVALID;
+  if (parts <= 0 || (parts & ~SIGATTN_BWD_ALL) != 0) return SIGATTN_ERR_INVALID;
   if (epilogue < 0 || epilogue > 2) return SIGATTN_ERR_INVALID;
   if (d != 64 && d != 128) return SIGATTN_ERR_UNSUPPORTED;
   if (epilogue != SIGATTN_SIGMOID && (!lse || !workspace || !o)) return SIGATTN_ERR_INVALID;
@@ -218,8 +221,21 @@ extern "C" int sigattn_bwd(const sigattn_plan* plan, int epilogue, int H, int d,
   if ((rc = make_tmap_bf16(&mv, tv, plan->B, H, d)) != SIGATTN_OK) return rc;
   if ((rc = make_tmap_bf16(&mdo, tdo, plan->B, H, d)) != SIGATTN_OK) return rc;
   return launch_bwd_impl(plan, epilogue, H, d, scale, mq, mk, mv, mdo, to, tdo, bias,
-                         bias_stride_b, lse, workspace, tdq, tdk, tdv, status,
+                         bias_stride_b, lse, workspace, tdq, tdk, tdv, parts, status,
                          g_wait_limit_ns.load(), static_cast<cudaStream_t>(s));
+}
+
+extern "C" int sigattn_bwd(const sigattn_plan* plan, int epilogue, int H, int d, float scale,
+                           const void* q, const int64_t q_strides[3], const void* k,
+                           const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
+                           const void* o, const int64_t o_strides[3], const void* dout,
+                           const int64_t do_strides[3], const float* bias, int64_t bias_stride_b,
+                           const float* lse, float* workspace, void* dq,
+                           const int64_t dq_strides[3], void* dk, const int64_t dk_strides[3],
+                           void* dv, const int64_t dv_strides[3], sigattn_stream s) {
+  return sigattn_bwd_ex(plan, epilogue, H, d, scale, q, q_strides, k, k_strides, v, v_strides, o,
+                        o_strides, dout, do_strides, bias, bias_stride_b, lse, workspace, dq,
+                        dq_strides, dk, dk_strides, dv, dv_strides, SIGATTN_BWD_ALL, s);
 }
 
 extern "C" int sigattn_bias_from_counts(const int32_t* d_counts, int64_t n, float* d_bias,

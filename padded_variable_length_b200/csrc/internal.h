@@ -8,7 +8,8 @@
 #include "../../include/sigattn.h"
 
 // Device buffers of a tile plan.  Layouts are those of sigattn_plan_export; in addition
-// the plan keeps two work lists ordered longest-first (count descending, then index):
+// the plan keeps the transposed PARTIAL bitmasks (for kernels that own a key per thread)
+// and two work lists ordered longest-first (count descending, then index):
 //   row_work[B*QT]  every (b, q-tile) row, rows with no tile last
 //   col_work[B*KT]  every (b, k-tile) column, columns with no tile last
 struct sigattn_plan {
@@ -24,6 +25,7 @@ struct sigattn_plan {
   int32_t* rowT_idx;
   int32_t* csc_map;
   uint32_t* bits;
+  uint32_t* bitsT;  // [partial * 512] the same bitmasks transposed: bit (q % 32) of word (k*4 + q/32)
   int32_t* row_work;
   int32_t* col_work;
 };

@@ -346,6 +346,20 @@ __global__ void __launch_bounds__(128) k_bits_from_lengths(const int32_t* __rest
   reinterpret_cast<uint4*>(bits + static_cast<int64_t>(blockIdx.x) * 512)[q] = w;
 }
 
+// One CTA of 128 threads per PARTIAL block: thread k gathers column k of the bitmask.
+__global__ void __launch_bounds__(128) k_transpose_bits(const uint32_t* __restrict__ bits,
+                                                        uint32_t* __restrict__ bitsT) {
+  __shared__ uint32_t w[512];
+  const uint32_t* src = bits + static_cast<int64_t>(blockIdx.x) * 512;
+  for (int i = threadIdx.x; i < 512; i += 128) w[i] = src[i];
+  __syncthreads();
+  const int k = threadIdx.x;
+  uint32_t out[4] = {0u, 0u, 0u, 0u};
+  for (int q = 0; q < 128; ++q) out[q >> 5] |= ((w[q * 4 + (k >> 5)] >> (k & 31)) & 1u) << (q & 31);
+  reinterpret_cast<uint4*>(bitsT + static_cast<int64_t>(blockIdx.x) * 512)[k] =
+      make_uint4(out[0], out[1], out[2], out[3]);
+}
+
 template <class T>
 int dev_alloc(T** p, size_t count) {
   *p = nullptr;
@@ -389,8 +403,8 @@ struct Scratch {
 };
 
 void plan_free_buffers(sigattn_plan* p) {
-  void* ps[] = {p->row_ptr, p->col_idx, p->kind,     p->pidx,     p->colT_ptr,
-                p->rowT_idx, p->csc_map, p->bits,    p->row_work, p->col_work};
+  void* ps[] = {p->row_ptr,  p->col_idx, p->kind, p->pidx,     p->colT_ptr, p->rowT_idx,
+                p->csc_map,  p->bits,    p->bitsT, p->row_work, p->col_work};
   for (void* q : ps)
     if (q) cudaFree(q);
 }
@@ -453,6 +467,7 @@ int finish_plan(sigattn_plan* plan, Scratch& sc, cudaStream_t stream, BitsFn bit
   SIGATTN_TRY(dev_alloc(&plan->rowT_idx, plan->nonempty));
   SIGATTN_TRY(dev_alloc(&plan->csc_map, plan->nonempty));
   SIGATTN_TRY(dev_alloc(&plan->bits, static_cast<size_t>(plan->partial) * 512));
+  SIGATTN_TRY(dev_alloc(&plan->bitsT, static_cast<size_t>(plan->partial) * 512));
   SIGATTN_TRY(scratch_alloc(&sc.eidx, static_cast<size_t>(rows) * KT, stream));
   SIGATTN_TRY(scratch_alloc(&sc.ptile, static_cast<size_t>(plan->partial), stream));
   if (plan->nonempty > 0) {
@@ -462,7 +477,11 @@ int finish_plan(sigattn_plan* plan, Scratch& sc, cudaStream_t stream, BitsFn bit
     k_fill_csc<<<grid_for(static_cast<int64_t>(cols) * 32, 256), 256, 0, stream>>>(
         sc.kinds, sc.eidx, B, QT, KT, plan->colT_ptr, plan->rowT_idx, plan->csc_map);
   }
-  if (plan->partial > 0) bits_kernel(sc.ptile, plan->bits, static_cast<int>(plan->partial));
+  if (plan->partial > 0) {
+    bits_kernel(sc.ptile, plan->bits, static_cast<int>(plan->partial));
+    k_transpose_bits<<<static_cast<unsigned>(plan->partial), 128, 0, stream>>>(plan->bits,
+                                                                               plan->bitsT);
+  }
   SIGATTN_TRY_CUDA(cudaGetLastError());
   sc.release(stream);
   *out = plan;
