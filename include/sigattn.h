@@ -212,6 +212,37 @@ SIGATTN_API int sigattn_bwd_ex(const sigattn_plan* plan, int epilogue, int H, in
                                int parts, sigattn_stream stream);
 
 /*
+ * Backward that allocates nothing, for callers that cannot call cudaMalloc: code running
+ * under a memory manager that owns all device memory (a framework's caching allocator, or a
+ * fixed budget set by a host application that loads this library as a plug-in), and step
+ * loops that cannot afford cudaMalloc's implicit device-wide synchronisation and
+ * unpredictable latency.  The paper has no counterpart to this entry point.
+ *
+ * Same arguments, results and errors as sigattn_bwd, without `workspace`: the fp32 D_i =
+ * dO_i . O_i values of the softmax modes go into a scratch array that the library keeps in
+ * device memory (a file-scope __device__ array of SIGATTN_NOALLOC_MAX_ROWS floats, 8 MiB, held
+ * by every GPU that loads the library until the process exits).  B * H * Nq above
+ * SIGATTN_NOALLOC_MAX_ROWS gives SIGATTN_ERR_UNSUPPORTED for SOFTMAX / SOFTMAX1 (SIGMOID uses
+ * no scratch and has no limit).  The first call on a device looks up the array's device
+ * address (once per device, with that device current); make that first call before any
+ * stream capture.  All calls share the one array and it keeps the last call's contents;
+ * every value a call reads is written by that same call first, so nothing has to be cleared,
+ * but calls whose kernels overlap on the GPU (other streams, other threads) race on it.
+ */
+#define SIGATTN_NOALLOC_MAX_ROWS (1 << 21)
+SIGATTN_API int sigattn_bwd_noalloc(const sigattn_plan* plan, int epilogue, int H, int d,
+                                    float scale, const void* q, const int64_t q_strides[3],
+                                    const void* k, const int64_t k_strides[3],
+                                    const void* v, const int64_t v_strides[3],
+                                    const void* o, const int64_t o_strides[3],
+                                    const void* dout, const int64_t do_strides[3],
+                                    const float* bias, int64_t bias_stride_b, const float* lse,
+                                    void* dq, const int64_t dq_strides[3],
+                                    void* dk, const int64_t dk_strides[3],
+                                    void* dv, const int64_t dv_strides[3],
+                                    sigattn_stream stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of the current
  * device: SIGATTN_OK, or SIGATTN_ERR_TIMEOUT if a kernel's bounded wait expired since the
  * last call (that kernel's outputs are then undefined), or SIGATTN_ERR_CUDA.

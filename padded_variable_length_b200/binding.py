@@ -71,6 +71,9 @@ _sig("sigattn_bwd", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, 
 _sig("sigattn_bwd_ex", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
      _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _i64, _p, _p,
      _p, _I64x3, _p, _I64x3, _p, _I64x3, ctypes.c_int, _p)
+_sig("sigattn_bwd_noalloc", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+     _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _i64, _p,
+     _p, _I64x3, _p, _I64x3, _p, _I64x3, _p)
 _sig("sigattn_get_status", ctypes.c_int, _p)
 _sig("sigattn_set_wait_limit_ns", ctypes.c_int, _u64)
 _sig("sigattn_selftest_wait_timeout", ctypes.c_int, _u64, _p)

@@ -19,6 +19,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -728,3 +730,64 @@ int launch_bwd_impl(const sigattn_plan* plan, int epilogue, int H, int d, float 
 }
 
 }  // namespace sigattn
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free backward.  Callers that cannot call cudaMalloc (see sigattn.h) get the
+// softmax modes' D workspace from this array instead of passing one in.  It is part of the
+// library's device image, so every GPU that loads the library holds it until exit.
+// ---------------------------------------------------------------------------------------
+static __device__ __align__(256) float g_noalloc_scratch[SIGATTN_NOALLOC_MAX_ROWS];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device.  In host code the array's
+// name is only a host-side stand-in, so the address is looked up once per device, with that
+// device current, and reused.
+int noalloc_scratch(float** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SIGATTN_ERR_NO_DEVICE;
+  }
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return SIGATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    float* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_noalloc_scratch);
+    if (e != cudaSuccess) return sigattn::cuda_status(e);
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SIGATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int sigattn_bwd_noalloc(const sigattn_plan* plan, int epilogue, int H, int d,
+                                   float scale, const void* q, const int64_t q_strides[3],
+                                   const void* k, const int64_t k_strides[3], const void* v,
+                                   const int64_t v_strides[3], const void* o,
+                                   const int64_t o_strides[3], const void* dout,
+                                   const int64_t do_strides[3], const float* bias,
+                                   int64_t bias_stride_b, const float* lse, void* dq,
+                                   const int64_t dq_strides[3], void* dk,
+                                   const int64_t dk_strides[3], void* dv,
+                                   const int64_t dv_strides[3], sigattn_stream stream) {
+  if (!plan || H < 1) return SIGATTN_ERR_INVALID;
+  float* workspace = nullptr;
+  if (epilogue == SIGATTN_SOFTMAX || epilogue == SIGATTN_SOFTMAX1) {
+    // The D preprocess writes every one of the B * H * Nq values before the two gradient
+    // kernels read them, so the array needs no clearing between calls.
+    if (static_cast<int64_t>(plan->B) * H * plan->Nq > SIGATTN_NOALLOC_MAX_ROWS)
+      return SIGATTN_ERR_UNSUPPORTED;
+    const int rc = noalloc_scratch(&workspace);
+    if (rc != SIGATTN_OK) return rc;
+  }
+  return sigattn_bwd_ex(plan, epilogue, H, d, scale, q, q_strides, k, k_strides, v, v_strides, o,
+                        o_strides, dout, do_strides, bias, bias_stride_b, lse, workspace, dq,
+                        dq_strides, dk, dk_strides, dv, dv_strides, SIGATTN_BWD_ALL, stream);
+}
