@@ -59,17 +59,14 @@ struct BwdParams {
   unsigned long long wait_ns;
 };
 
-__device__ __forceinline__ float sigmoid_from_u(float u) {
-  return rcp_approx(1.0f + ex2_approx(u));
-}
-
-// Exponent offset of one query row: p = 2^(c1 s + off).  SIGMOID: off = -bias log2 e with
-// c1 = -scale log2 e, and p = 1 / (1 + 2^(...)).  Softmax modes: off = (bias - lse) log2 e.
+// Offset of one query row in the weight's argument, with c1 the matching slope:
+// SIGMOID  p = 0.5 + 0.5 tanh(c1 s + off),  c1 = scale / 2,  off = bias / 2;
+// softmax  p = 2^(c1 s + off),               c1 = scale log2 e,  off = (bias - lse) log2 e.
 template <int EPI>
 __device__ __forceinline__ float row_offset(const BwdParams& p, int b, int h, int qg) {
   if (qg >= p.Nq) return 0.0f;
   const float bias = p.bias ? p.bias[b * p.bias_sb + qg] : 0.0f;
-  if (EPI == 0) return -bias * kLog2e;
+  if (EPI == 0) return 0.5f * bias;
   return (bias - p.lse[(static_cast<int64_t>(b) * p.H + h) * p.Nq + qg]) * kLog2e;
 }
 
@@ -84,7 +81,7 @@ template <int EPI>
 __device__ __forceinline__ void weight_grad(float s, float dp, float c1, float off, float Drow,
                                             bool keep, float& pw, float& ds) {
   if (EPI == 0) {
-    const float sg = sigmoid_from_u(fmaf(s, c1, off));
+    const float sg = sigmoid_tanh(s, c1, off);
     pw = keep ? sg : 0.0f;
     ds = dp * pw * (1.0f - pw);
   } else {
@@ -335,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = wq * 32 + lane;  // key row of the tile
     const int kg = kt * kTile + row;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const float c1 = (EPI == 0 ? -1.0f : 1.0f) * p.scale * kLog2e;
+    const float c1 = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
       const int s = i % S;
@@ -568,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = wq * 32 + lane;
     const int qg = qt * kTile + row;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const float c1 = (EPI == 0 ? -1.0f : 1.0f) * p.scale * kLog2e;
+    const float c1 = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
     const float off = row_offset<EPI>(p, b, h, qg);
     const float Drow = row_D<EPI>(p, b, h, qg);
     bool ok = true;

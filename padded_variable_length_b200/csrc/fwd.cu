@@ -71,12 +71,6 @@ struct FwdLayout {
   static constexpr int kAlloc = kBytes + 1024;               // slack for 1024-byte alignment
 };
 
-__device__ __forceinline__ float sigmoid_from_u(float u) {
-  // u = -x log2(e): sigma(x) = 1 / (1 + 2^u).  2^u overflows to +inf for very negative x,
-  // giving 1/inf = 0; it underflows to 0 for large x, giving 1.
-  return rcp_approx(1.0f + ex2_approx(u));
-}
-
 template <int D, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -234,9 +228,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rg = qt * kTile + row;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float bias_r = (p.bias != nullptr && rg < p.Nq) ? p.bias[b * p.bias_sb + rg] : 0.0f;
-    // sigmoid: u = -(scale s + bias) log2 e ; softmax: t = (scale s + bias) log2 e
-    const float c1 = (EPI == 0 ? -1.0f : 1.0f) * p.scale * kLog2e;
-    const float c0 = (EPI == 0 ? -1.0f : 1.0f) * bias_r * kLog2e;
+    // sigmoid: sigma(x) = 0.5 + 0.5 tanh(x/2), x = scale s + bias -> (c1, c0) = halves;
+    // softmax: t = (scale s + bias) log2 e
+    const float c1 = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
+    const float c0 = EPI == 0 ? 0.5f * bias_r : bias_r * kLog2e;
     float m_run = EPI == 2 ? 0.0f : kNegBig;  // base-2 running max (softmax modes)
     float l_run = (EPI == 2 && g == 0) ? 1.0f : 0.0f;
     // `ok` stays warp-uniform (tcgen05.ld/st are warp-collective).  After an abort the
@@ -270,8 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (EPI == 0) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float u = fmaf(__uint_as_float(sr[c]), c1, c0);
-          const float sg = sigmoid_from_u(u);
+          const float sg = sigmoid_tanh(__uint_as_float(sr[c]), c1, c0);
           const uint32_t bit = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
           pv[c] = bit ? sg : 0.0f;
         }

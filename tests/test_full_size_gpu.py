@@ -1,0 +1,68 @@
+"""Parity at the full sizes of the long-ragged batch (B=8, lengths up to 16384, H=16,
+d=128) and the packed-document mask (B=4, N=8192, H=16, d=128), in the launch configuration
+bench.py times: the whole batch goes through the CUDA path, and the oracle recomputes
+sampled rows of O and dQ and sampled key rows of dK and dV one by one (tile edges, sequence
+ends and random rows) for a few (batch entry, head) pairs.  Pad rows are checked exactly
+zero over the whole tensors."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as A
+from padded_variable_length_b200 import workloads as W
+from tests import harness as Hn
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+def _sample_rows(rng, n, count=24):
+    base = [0, 1, 126, 127, 128, 129, n // 2, n - 2, n - 1]
+    base = [r for r in base if 0 <= r < n]
+    extra = rng.choice(n, size=min(count, n), replace=False).tolist()
+    return np.array(sorted(set(base + extra)))
+
+
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_full_size_sampled(cfg):
+    from padded_variable_length_b200 import binding as Bd
+    w = W.config(cfg)
+    t = W.tensors(w)
+    d, plan, bias = Hn.device_setup(w, t)
+    o, _ = Bd.fwd(plan, d["q"], d["k"], d["v"], bias)
+    dq, dk, dv = Bd.bwd(plan, d["q"], d["k"], d["v"], o, d["do"], bias)
+    assert Bd.get_status() == 0
+    # pad rows exactly zero, everywhere
+    if w.lengths is not None:
+        for b, n in enumerate(w.lengths):
+            for x in (o, dq, dk, dv):
+                assert torch.all(x[b, int(n):] == 0)
+    for x in (o, dq, dk, dv):
+        assert torch.isfinite(x).all()
+    rng = np.random.default_rng(cfg)
+    scale = 1.0 / math.sqrt(w.d)
+    bias_ref = A.bias_from_counts(w.counts)
+    mp = A.mask_provider(w.lengths, w.mask, w.Nq, w.Nk)
+    got = {"o": [], "dq": [], "dk": [], "dv": []}
+    ref = {"o": [], "dq": [], "dk": [], "dv": []}
+    pairs = [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2)]
+    for (b, h) in pairs:
+        n = int(w.lengths[b]) if w.lengths is not None else w.Nq
+        rows = _sample_rows(rng, n)
+        q, k, v, do = (Hn.to_f64(t[x][b, :, h]) for x in ("q", "k", "v", "do"))
+        mr = mp(b)
+        o_ref, _ = A.head_forward(q, k, v, mr, bias_ref[b], scale, A.SIGMOID, rows=rows)
+        dq_ref = A.query_rows_backward(q, k, v, do, mr, bias_ref[b], scale, A.SIGMOID, rows)
+        dk_ref, dv_ref = A.key_columns_backward(q, k, v, do, mr, bias_ref[b], scale, A.SIGMOID, rows)
+        got["o"].append(Hn.to_f64(o[b, rows, h]))
+        got["dq"].append(Hn.to_f64(dq[b, rows, h]))
+        got["dk"].append(Hn.to_f64(dk[b, rows, h]))
+        got["dv"].append(Hn.to_f64(dv[b, rows, h]))
+        ref["o"].append(o_ref)
+        ref["dq"].append(dq_ref)
+        ref["dk"].append(dk_ref)
+        ref["dv"].append(dv_ref)
+    for name in got:
+        Hn.check_close(np.concatenate(got[name]), np.concatenate(ref[name]),
+                       f"{w.name} {name} (sampled)")
