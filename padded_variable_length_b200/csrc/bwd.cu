@@ -11,14 +11,15 @@
 //   dV += P^T dO      dK += scale dS^T Q      dQ += scale dS K
 //
 // Thread layout as in the forward: warp 0 TMA producer, warp 1 TMEM allocator and MMA
-// issuer, warps 4-11 two epilogue warpgroups (thread = TMEM lane; warpgroup g owns tile
-// columns [64g, 64g+64) and accumulator columns [g d/2, (g+1) d/2)).
+// issuer, warps 4-11 two epilogue warpgroups (thread = TMEM lane; warpgroup h owns column
+// half h of every tile and accumulator columns [h d/2, (h+1) d/2)).
 // TMEM: [0,128) S (or S^T), [128,256) dP (or dP^T), then the fp32 accumulators.  The bf16
 // P / dS values overwrite the columns of S / dP that the same warpgroup already read, and
 // are the TMEM A operand of the accumulating MMAs.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "internal.h"
@@ -43,7 +44,7 @@ struct BwdParams {
   const int32_t* csc_map;
   const int32_t* row_work;
   const int32_t* col_work;
-  int QT, KT, Nq, Nk, H;
+  int B, QT, KT, Nq, Nk, H;
   float scale;
   const float* bias;
   int64_t bias_sb;
@@ -76,29 +77,26 @@ __device__ __forceinline__ float row_D(const BwdParams& p, int b, int h, int qg)
   return p.Dws[(static_cast<int64_t>(b) * p.H + h) * p.Nq + qg];
 }
 
-// p and ds of one element; `keep` is the mask bit.
+// p and ds of two neighbouring elements (packed fp32 pairs); k0 / k1 are the mask bits.
+// SIGMOID: th = tanh(c1 s + off), p = (1 + th) / 2, p (1 - p) = (1 - th^2) / 4, so
+//   ds = dp (1/4 - th^2 / 4); a masked element takes th = -1, which gives p = ds = 0.
+// softmax: p = 2^(c1 s + off), ds = p (dp - D); a masked element takes p = 0.
 template <int EPI>
-__device__ __forceinline__ void weight_grad(float s, float dp, float c1, float off, float Drow,
-                                            bool keep, float& pw, float& ds) {
+__device__ __forceinline__ void weight_grad2(float2 s, float2 dp, float2 c1, float2 off, float2 Dv,
+                                             bool k0, bool k1, float2& pw, float2& ds) {
+  const float2 x = fma2(s, c1, off);
   if (EPI == 0) {
-    const float sg = sigmoid_tanh(s, c1, off);
-    pw = keep ? sg : 0.0f;
-    ds = dp * pw * (1.0f - pw);
+    float2 th = make_float2(tanh_approx(x.x), tanh_approx(x.y));
+    th.x = k0 ? th.x : -1.0f;
+    th.y = k1 ? th.y : -1.0f;
+    pw = fma2(th, make_float2(0.5f, 0.5f), make_float2(0.5f, 0.5f));
+    const float2 m = mul2(th, make_float2(-0.25f, -0.25f));
+    const float2 w = fma2(m, th, make_float2(0.25f, 0.25f));
+    ds = mul2(w, dp);
   } else {
-    pw = keep ? ex2_approx(fmaf(s, c1, off)) : 0.0f;
-    ds = pw * (dp - Drow);
+    pw = make_float2(k0 ? ex2_approx(x.x) : 0.0f, k1 ? ex2_approx(x.y) : 0.0f);
+    ds = mul2(pw, fma2(Dv, make_float2(-1.0f, -1.0f), dp));
   }
-}
-
-__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_t (&acc)[32],
-                                               float mul) {
-  uint32_t pk[16];
-#pragma unroll
-  for (int c = 0; c < 16; ++c)
-    pk[c] = pack_bf16x2(__uint_as_float(acc[2 * c]) * mul, __uint_as_float(acc[2 * c + 1]) * mul);
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
 }
 
 template <int D>
@@ -149,22 +147,64 @@ __global__ void d_preprocess_kernel(const __nv_bfloat16* __restrict__ o, int64_t
 }
 
 // ---------------------------------------------------------------------------------------
-// dK / dV
+// Shared pieces of the two gradient kernels.
+//
+// Both are persistent (one CTA per SM, static stride over the plan's longest-first work
+// list) and split every 128 x 128 tile into two column halves: epilogue warpgroup h owns
+// half h, with its own "S ready" and "P ready" barriers.  The MMA thread interleaves the
+// halves: the accumulating MMAs of half h of the previous tile, then S / dP of half h of
+// the current tile.  While one warpgroup recomputes the weights of its half, the tensor
+// pipe works on the other half, and the two warpgroups' latencies interleave instead of
+// coinciding.
+// ---------------------------------------------------------------------------------------
+struct WorkRef {
+  int b, t, h, e0, n;  // batch, tile index on the item's own axis, head, list range
+};
+
+// dK/dV: item w -> (k-tile column, head); dQ: item w -> (q-tile row, head).
+__device__ __forceinline__ WorkRef decode_col(const BwdParams& p, int w) {
+  WorkRef r;
+  const int c = p.col_work[w / p.H];
+  r.h = w % p.H;
+  r.b = c / p.KT;
+  r.t = c % p.KT;
+  r.e0 = p.colT_ptr[c];
+  r.n = p.colT_ptr[c + 1] - r.e0;
+  return r;
+}
+
+__device__ __forceinline__ WorkRef decode_row(const BwdParams& p, int w) {
+  WorkRef r;
+  const int q = p.row_work[w / p.H];
+  r.h = w % p.H;
+  r.b = q / p.QT;
+  r.t = q % p.QT;
+  r.e0 = p.row_ptr[q];
+  r.n = p.row_ptr[q + 1] - r.e0;
+  return r;
+}
+
+// ---------------------------------------------------------------------------------------
+// dK / dV: one item = one k-tile column of the plan for one head; thread = key row.
+// TMEM: S^T half h [64h, 64h+64), dP^T half h [128+64h, ...), then per accumulator buffer a:
+// dV [256 + 2Da, +D), dK [256 + 2Da + D, +D).
 // ---------------------------------------------------------------------------------------
 template <int D>
 struct DkvLayout {
-  static constexpr int kStages = D == 64 ? 4 : 2;
+  static constexpr int kStages = D == 64 ? 3 : 2;   // Q / dO ring
+  static constexpr int kKVBufs = D == 64 ? 2 : 1;   // K / V of consecutive items
+  static constexpr int kAccBufs = D == 64 ? 2 : 1;  // dV / dK accumulators in TMEM
   static constexpr int kBoxes = D / 64;
   static constexpr int kBoxBytes = 128 * 128;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
   static constexpr int kK = 0;
-  static constexpr int kV = kTileBytes;
-  static constexpr int kQ = 2 * kTileBytes;
+  static constexpr int kV = kK + kKVBufs * kTileBytes;
+  static constexpr int kQ = kV + kKVBufs * kTileBytes;
   static constexpr int kDO = kQ + kStages * kTileBytes;
-  static constexpr int kVec = kDO + kStages * kTileBytes;      // float [S][2][128]
+  static constexpr int kVec = kDO + kStages * kTileBytes;  // float [S][2][128]
   static constexpr int kBar = kVec + kStages * 2 * 128 * 4;
-  // kv_full, acc_full, s_full, p_full, q_full[S], q_empty[S]
-  static constexpr int kNumBars = 4 + 2 * kStages;
+  // kv_full[KV] kv_empty[KV] q_full[S] q_empty[S] s_full[2] p_full[2] acc_full[A] acc_empty[A]
+  static constexpr int kNumBars = 2 * kKVBufs + 2 * kStages + 4 + 2 * kAccBufs;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -176,34 +216,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                 const BwdParams p) {
   using L = DkvLayout<D>;
-  constexpr int S = L::kStages;
+  constexpr int S = L::kStages, KVB = L::kKVBufs, ACB = L::kAccBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
-  const int wi = blockIdx.x / p.H, h = blockIdx.x % p.H;
-  const int c = p.col_work[wi];
-  const int b = c / p.KT, kt = c % p.KT;
-  const int e0 = p.colT_ptr[c];
-  const int n = p.colT_ptr[c + 1] - e0;
-
-  if (n == 0) {
-    // No query attends to this k-tile: dK = dV = 0 on its rows.
-    const int rows = min(kTile, p.Nk - kt * kTile);
-    zero_rows<D>(p.dk + b * p.dk_sb + static_cast<int64_t>(kt * kTile) * p.dk_sn + h * p.dk_sh,
-                 p.dk_sn, rows, threadIdx.x, kThreads);
-    zero_rows<D>(p.dv + b * p.dv_sb + static_cast<int64_t>(kt * kTile) * p.dv_sn + h * p.dv_sh,
-                 p.dv_sn, rows, threadIdx.x, kThreads);
-    return;
-  }
+  const int nitems = p.B * p.KT * p.H;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* kv_full = bars + 0;
-  uint64_t* acc_full = bars + 1;
-  uint64_t* s_full = bars + 2;
-  uint64_t* p_full = bars + 3;
-  uint64_t* q_full = bars + 4;
-  uint64_t* q_empty = bars + 4 + S;
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = kv_full + KVB;
+  uint64_t* q_full = kv_empty + KVB;
+  uint64_t* q_empty = q_full + S;
+  uint64_t* s_full = q_empty + S;   // [2] per half
+  uint64_t* p_full = s_full + 2;    // [2] per half
+  uint64_t* acc_full = p_full + 2;  // [ACB]
+  uint64_t* acc_empty = acc_full + ACB;
   float* vec = reinterpret_cast<float*>(smem + L::kVec);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
@@ -211,13 +239,380 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wctx{p.status, p.wait_ns, abort_flag};
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
-    mbar_init(acc_full, 1);
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 8);
+    for (int i = 0; i < KVB; ++i) {
+      mbar_init(kv_full + i, 1);
+      mbar_init(kv_empty + i, 1);
+    }
     for (int i = 0; i < S; ++i) {
       mbar_init(q_full + i, 2);  // TMA bytes + the producer warp's column vectors
       mbar_init(q_empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(p_full + i, 4);  // the four warps of one epilogue warpgroup
+    }
+    for (int i = 0; i < ACB; ++i) {
+      mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, 8);
+    }
+    *abort_flag = 0;
+    *drain_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    int qc = 0, ii = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
+      const WorkRef it = decode_col(p, w);
+      if (it.n == 0) continue;
+      const int kb = ii % KVB;
+      if (lane == 0 && ii >= KVB) ok = mbar_wait(kv_empty + kb, ((ii / KVB) - 1) & 1, wctx);
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(kv_full + kb, 2 * L::kTileBytes);
+        for (int x = 0; x < L::kBoxes; ++x) {
+          tma_load_4d(smem + L::kK + kb * L::kTileBytes + x * L::kBoxBytes, &tk, kv_full + kb,
+                      x * 64, it.t * kTile, it.h, it.b);
+          tma_load_4d(smem + L::kV + kb * L::kTileBytes + x * L::kBoxBytes, &tv, kv_full + kb,
+                      x * 64, it.t * kTile, it.h, it.b);
+        }
+      }
+      ++ii;
+      for (int i = 0; i < it.n; ++i, ++qc) {
+        const int s = qc % S;
+        if (lane == 0 && qc >= S) ok = mbar_wait(q_empty + s, ((qc / S) - 1) & 1, wctx);
+        ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        const int qt = p.rowT_idx[it.e0 + i];
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full + s, 2 * L::kTileBytes);
+          for (int x = 0; x < L::kBoxes; ++x) {
+            tma_load_4d(smem + L::kQ + s * L::kTileBytes + x * L::kBoxBytes, &tq, q_full + s,
+                        x * 64, qt * kTile, it.h, it.b);
+            tma_load_4d(smem + L::kDO + s * L::kTileBytes + x * L::kBoxBytes, &tdo, q_full + s,
+                        x * 64, qt * kTile, it.h, it.b);
+          }
+        }
+        float* vs = vec + s * 256;
+        for (int cc = lane; cc < 128; cc += 32) {
+          const int qg = qt * kTile + cc;
+          vs[cc] = row_offset<EPI>(p, it.b, it.h, qg);
+          vs[128 + cc] = row_D<EPI>(p, it.b, it.h, qg);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_full + s);
+      }
+    }
+    if (lane == 0 && *abort_flag) {
+      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      for (int u = max(0, ii - KVB); u < ii; ++u) mbar_wait(kv_full + u % KVB, (u / KVB) & 1, drain);
+      for (int u = max(0, qc - S); u < qc; ++u) mbar_wait(q_full + u % S, (u / S) & 1, drain);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_half = idesc_bf16_f32(128, 64, false);  // S^T / dP^T halves
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);     // dV / dK
+      // d = 64 (three Q / dO stages): the dV / dK MMAs of half h of a tile are issued just
+      // before the S^T / dP^T of half h of the next tile, so the tensor pipe moves on to the
+      // next tile while the other warpgroup still works.  d = 128 (two stages, MMA-bound):
+      // a tile's accumulating MMAs follow its own S^T / dP^T, which frees its Q / dO stage
+      // one tile earlier and keeps the next loads ahead of the MMAs.
+      constexpr bool kDeferAcc = D == 64;
+      bool ok = true;
+      // accumulating MMAs of half h of the q-tile with global index qt_, stage s, buffer ab
+      auto acc_half = [&](int h, int qt_, int s, int ab, bool first, int item) -> bool {
+        if (!mbar_wait(p_full + h, qt_ & 1, wctx)) return false;
+        if (h == 0 && first && item >= ACB &&
+            !mbar_wait(acc_empty + ab, ((item / ACB) - 1) & 1, wctx))
+          return false;
+        tc_fence_after();
+        const uint32_t q_s = smem_u32(smem + L::kQ + s * L::kTileBytes);
+        const uint32_t do_s = smem_u32(smem + L::kDO + s * L::kTileBytes);
+        const uint32_t t_dv = tmem + 256 + ab * 2 * D, t_dk = t_dv + D;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t acc = (first && h == 0 && kk == 0) ? 0u : 1u;
+          const uint32_t boff = (4 * h + kk) * 2048;  // query rows 64h + 16kk
+          mma_ts(t_dv, tmem + 64 * h + kk * 8,
+                 smem_desc_sw128(do_s + boff, L::kBoxBytes, 1024), idesc_acc, acc);
+          mma_ts(t_dk, tmem + 128 + 64 * h + kk * 8,
+                 smem_desc_sw128(q_s + boff, L::kBoxBytes, 1024), idesc_acc, acc);
+        }
+        return true;
+      };
+      auto sdp_half = [&](int h, uint32_t k_base, uint32_t v_base, uint32_t q_s, uint32_t do_s) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
+          mma_ss(tmem + 64 * h, smem_desc_sw128(k_base + off, 16, 1024),
+                 smem_desc_sw128(q_s + off + h * 8192, 16, 1024), idesc_half, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
+          mma_ss(tmem + 128 + 64 * h, smem_desc_sw128(v_base + off, 16, 1024),
+                 smem_desc_sw128(do_s + off + h * 8192, 16, 1024), idesc_half, kk > 0);
+        }
+        mma_commit(s_full + h);
+      };
+      // the q-tile whose accumulating MMAs are deferred (kDeferAcc)
+      int pend_qt = -1, pend_s = 0, pend_ab = 0, pend_item = 0;
+      bool pend_first = false, pend_last = false;
+      auto finish_pending = [&]() {
+        mma_commit(q_empty + pend_s);
+        if (pend_last) mma_commit(acc_full + pend_ab);
+      };
+      int qc = 0, ii = 0;
+      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
+        const WorkRef it = decode_col(p, w);
+        if (it.n == 0) continue;
+        const int kb = ii % KVB, ab = ii % ACB;
+        if (kDeferAcc && pend_qt >= 0) {  // previous item's last tile, before new K / V
+          if (!(ok = acc_half(0, pend_qt, pend_s, pend_ab, pend_first, pend_item) &&
+                     acc_half(1, pend_qt, pend_s, pend_ab, pend_first, pend_item)))
+            break;
+          finish_pending();
+          pend_qt = -1;
+        }
+        if (!(ok = mbar_wait(kv_full + kb, (ii / KVB) & 1, wctx))) break;
+        tc_fence_after();
+        const uint32_t k_base = smem_u32(smem + L::kK + kb * L::kTileBytes);
+        const uint32_t v_base = smem_u32(smem + L::kV + kb * L::kTileBytes);
+        for (int i = 0; i < it.n; ++i, ++qc) {
+          const int s = qc % S;
+          if (!(ok = mbar_wait(q_full + s, (qc / S) & 1, wctx))) break;
+          tc_fence_after();
+          const uint32_t q_s = smem_u32(smem + L::kQ + s * L::kTileBytes);
+          const uint32_t do_s = smem_u32(smem + L::kDO + s * L::kTileBytes);
+          if (kDeferAcc) {
+            for (int h = 0; h < 2 && ok; ++h) {
+              if (pend_qt >= 0 &&
+                  !(ok = acc_half(h, pend_qt, pend_s, pend_ab, pend_first, pend_item)))
+                break;
+              sdp_half(h, k_base, v_base, q_s, do_s);
+            }
+            if (!ok) break;
+            if (pend_qt >= 0) finish_pending();
+            if (i == it.n - 1) mma_commit(kv_empty + kb);
+            pend_qt = qc;
+            pend_s = s;
+            pend_ab = ab;
+            pend_item = ii;
+            pend_first = i == 0;
+            pend_last = i == it.n - 1;
+          } else {
+            sdp_half(0, k_base, v_base, q_s, do_s);
+            sdp_half(1, k_base, v_base, q_s, do_s);
+            if (!(ok = acc_half(0, qc, s, ab, i == 0, ii) && acc_half(1, qc, s, ab, i == 0, ii)))
+              break;
+            mma_commit(q_empty + s);
+            if (i == it.n - 1) {
+              mma_commit(acc_full + ab);
+              mma_commit(kv_empty + kb);
+            }
+          }
+        }
+        ++ii;
+      }
+      if (kDeferAcc && ok && pend_qt >= 0 &&
+          acc_half(0, pend_qt, pend_s, pend_ab, pend_first, pend_item) &&
+          acc_half(1, pend_qt, pend_s, pend_ab, pend_first, pend_item))
+        finish_pending();
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ---------------------------------------------------------------- epilogue
+    const int h = (warp - kEpiWarp0) >> 2;  // query half of every tile
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;  // key row of the tile
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float c1s = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
+    const float2 c1 = make_float2(c1s, c1s);
+    bool ok = true;
+    int qc = 0, ii = 0;
+    for (int w = blockIdx.x; w < nitems; w += gridDim.x) {
+      const WorkRef it = decode_col(p, w);
+      if (it.n == 0) {
+        // No query attends to this k-tile: dK = dV = 0 on its rows.
+        const int rows = min(kTile, p.Nk - it.t * kTile);
+        const int tid = threadIdx.x - kEpiWarp0 * 32;
+        zero_rows<D>(p.dk + it.b * p.dk_sb + static_cast<int64_t>(it.t * kTile) * p.dk_sn +
+                         it.h * p.dk_sh, p.dk_sn, rows, tid, 256);
+        zero_rows<D>(p.dv + it.b * p.dv_sb + static_cast<int64_t>(it.t * kTile) * p.dv_sn +
+                         it.h * p.dv_sh, p.dv_sn, rows, tid, 256);
+        continue;
+      }
+      if (!ok) break;
+      const int ab = ii % ACB;
+      for (int i = 0; i < it.n; ++i, ++qc) {
+        const int s = qc % S;
+        const int e = p.csc_map[it.e0 + i];
+        const int kd = p.kind[e];
+        uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+        if (kd == 2)
+          mb = *reinterpret_cast<const uint2*>(p.bitsT + static_cast<int64_t>(p.pidx[e]) * 512 +
+                                               row * 4 + 2 * h);
+        if (ok) ok = mbar_wait(q_full + s, (qc / S) & 1, wctx);
+        if (ok) ok = mbar_wait(s_full + h, qc & 1, wctx);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float* vs = vec + s * 256 + 64 * h;
+        uint32_t sr[2][32], dpr[2][32];
+        tmem_ld32(t_lane + 64 * h, sr[0]);
+        tmem_ld32(t_lane + 128 + 64 * h, dpr[0]);
+        tmem_wait_ld();
+        tmem_ld32(t_lane + 64 * h + 32, sr[1]);
+        tmem_ld32(t_lane + 128 + 64 * h + 32, dpr[1]);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (c == 1) tmem_wait_ld();
+          const uint32_t mw = c ? mb.y : mb.x;
+          uint32_t pk[16], dk[16];
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            float2 pw, ds;
+            const float2 off2 = *reinterpret_cast<const float2*>(vs + 32 * c + cc);
+            const float2 D2 = EPI == 0 ? make_float2(0.0f, 0.0f)
+                                       : *reinterpret_cast<const float2*>(vs + 128 + 32 * c + cc);
+            weight_grad2<EPI>(make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
+                              make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])),
+                              c1, off2, D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
+            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
+            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+          }
+          tmem_st16(t_lane + 64 * h + 16 * c, pk);
+          tmem_st16(t_lane + 128 + 64 * h + 16 * c, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + h);
+      }
+      if (!ok) break;
+      // ---- output of this item: dV, dK (this warpgroup's half of the columns)
+      ok = mbar_wait(acc_full + ab, (ii / ACB) & 1, wctx);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      constexpr int kOc = D / 2;
+      uint32_t pv[kOc / 2], pkk[kOc / 2];
+#pragma unroll
+      for (int c0 = 0; c0 < kOc; c0 += 32) {
+        uint32_t acc[32];
+        tmem_ld32(t_lane + 256 + ab * 2 * D + h * kOc + c0, acc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pv[c0 / 2 + c] = pack_bf16x2(__uint_as_float(acc[2 * c]), __uint_as_float(acc[2 * c + 1]));
+        tmem_ld32(t_lane + 256 + ab * 2 * D + D + h * kOc + c0, acc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pkk[c0 / 2 + c] = pack_bf16x2(__uint_as_float(acc[2 * c]) * p.scale,
+                                        __uint_as_float(acc[2 * c + 1]) * p.scale);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + ab);
+      const int kg = it.t * kTile + row;
+      if (kg < p.Nk) {
+        uint4* dvp = reinterpret_cast<uint4*>(p.dv + it.b * p.dv_sb + static_cast<int64_t>(kg) * p.dv_sn +
+                                              it.h * p.dv_sh + h * kOc);
+        uint4* dkp = reinterpret_cast<uint4*>(p.dk + it.b * p.dk_sb + static_cast<int64_t>(kg) * p.dk_sn +
+                                              it.h * p.dk_sh + h * kOc);
+#pragma unroll
+        for (int c = 0; c < kOc / 8; ++c) {
+          dvp[c] = make_uint4(pv[4 * c], pv[4 * c + 1], pv[4 * c + 2], pv[4 * c + 3]);
+          dkp[c] = make_uint4(pkk[4 * c], pkk[4 * c + 1], pkk[4 * c + 2], pkk[4 * c + 3]);
+        }
+      }
+      ++ii;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// dQ: one item = one q-tile row of the plan for one head; thread = query row.
+// TMEM: S half h [64h, 64h+64), dP half h [128+64h, ...), dQ buffer a [256 + Da, +D).
+// ---------------------------------------------------------------------------------------
+template <int D>
+struct DqLayout {
+  static constexpr int kStages = D == 64 ? 3 : 2;   // K / V ring
+  static constexpr int kQBufs = D == 64 ? 2 : 1;    // Q / dO of consecutive items
+  static constexpr int kAccBufs = D == 64 ? 2 : 1;  // dQ accumulators in TMEM
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kBoxBytes = 128 * 128;
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;
+  static constexpr int kQ = 0;
+  static constexpr int kDO = kQ + kQBufs * kTileBytes;
+  static constexpr int kK = kDO + kQBufs * kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kBar = kV + kStages * kTileBytes;
+  // qd_full[QB] qd_empty[QB] kv_full[S] kv_empty[S] s_full[2] ds_full[2] acc_full[A] acc_empty[A]
+  static constexpr int kNumBars = 2 * kQBufs + 2 * kStages + 4 + 2 * kAccBufs;
+  static constexpr int kMisc = kBar + 8 * kNumBars;
+  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+template <int D, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+              const BwdParams p) {
+  using L = DqLayout<D>;
+  constexpr int S = L::kStages, QB = L::kQBufs, ACB = L::kAccBufs;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int warp = warp_id(), lane = lane_id();
+  const int nitems = p.B * p.QT * p.H;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* qd_full = bars;
+  uint64_t* qd_empty = qd_full + QB;
+  uint64_t* kv_full = qd_empty + QB;
+  uint64_t* kv_empty = kv_full + S;
+  uint64_t* s_full = kv_empty + S;   // [2] per half
+  uint64_t* ds_full = s_full + 2;    // [2] per half
+  uint64_t* acc_full = ds_full + 2;  // [ACB]
+  uint64_t* acc_empty = acc_full + ACB;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* drain_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
+  const WaitCtx wctx{p.status, p.wait_ns, abort_flag};
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < QB; ++i) {
+      mbar_init(qd_full + i, 1);
+      mbar_init(qd_empty + i, 1);
+    }
+    for (int i = 0; i < S; ++i) {
+      mbar_init(kv_full + i, 1);
+      mbar_init(kv_empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(ds_full + i, 4);
+    }
+    for (int i = 0; i < ACB; ++i) {
+      mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, 8);
     }
     *abort_flag = 0;
     *drain_flag = 0;
@@ -232,170 +627,228 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      tma_prefetch_desc(&tq);
-      tma_prefetch_desc(&tk);
-      tma_prefetch_desc(&tv);
-      tma_prefetch_desc(&tdo);
-      mbar_arrive_expect_tx(kv_full, 2 * L::kTileBytes);
-      for (int x = 0; x < L::kBoxes; ++x) {
-        tma_load_4d(smem + L::kK + x * L::kBoxBytes, &tk, kv_full, x * 64, kt * kTile, h, b);
-        tma_load_4d(smem + L::kV + x * L::kBoxBytes, &tv, kv_full, x * 64, kt * kTile, h, b);
-      }
-    }
-    int issued = 0;
-    for (int i = 0; i < n; ++i) {
-      const int s = i % S;
+      int tk_ = 0, ii = 0;
       bool ok = true;
-      if (lane == 0 && i >= S) ok = mbar_wait(q_empty + s, ((i / S) - 1) & 1, wctx);
-      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      const int qt = p.rowT_idx[e0 + i];
-      if (lane == 0) {
-        mbar_arrive_expect_tx(q_full + s, 2 * L::kTileBytes);
+      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
+        const WorkRef it = decode_row(p, w);
+        if (it.n == 0) continue;
+        const int qb = ii % QB;
+        if (ii >= QB && !(ok = mbar_wait(qd_empty + qb, ((ii / QB) - 1) & 1, wctx))) break;
+        mbar_arrive_expect_tx(qd_full + qb, 2 * L::kTileBytes);
         for (int x = 0; x < L::kBoxes; ++x) {
-          tma_load_4d(smem + L::kQ + s * L::kTileBytes + x * L::kBoxBytes, &tq, q_full + s, x * 64,
-                      qt * kTile, h, b);
-          tma_load_4d(smem + L::kDO + s * L::kTileBytes + x * L::kBoxBytes, &tdo, q_full + s,
-                      x * 64, qt * kTile, h, b);
+          tma_load_4d(smem + L::kQ + qb * L::kTileBytes + x * L::kBoxBytes, &tq, qd_full + qb,
+                      x * 64, it.t * kTile, it.h, it.b);
+          tma_load_4d(smem + L::kDO + qb * L::kTileBytes + x * L::kBoxBytes, &tdo, qd_full + qb,
+                      x * 64, it.t * kTile, it.h, it.b);
+        }
+        ++ii;
+        for (int j = 0; j < it.n; ++j, ++tk_) {
+          const int s = tk_ % S;
+          if (tk_ >= S && !(ok = mbar_wait(kv_empty + s, ((tk_ / S) - 1) & 1, wctx))) break;
+          const int kt = p.col_idx[it.e0 + j];
+          mbar_arrive_expect_tx(kv_full + s, 2 * L::kTileBytes);
+          for (int x = 0; x < L::kBoxes; ++x) {
+            tma_load_4d(smem + L::kK + s * L::kTileBytes + x * L::kBoxBytes, &tk, kv_full + s,
+                        x * 64, kt * kTile, it.h, it.b);
+            tma_load_4d(smem + L::kV + s * L::kTileBytes + x * L::kBoxBytes, &tv, kv_full + s,
+                        x * 64, kt * kTile, it.h, it.b);
+          }
         }
       }
-      float* vs = vec + s * 256;
-      for (int cc = lane; cc < 128; cc += 32) {
-        const int qg = qt * kTile + cc;
-        vs[cc] = row_offset<EPI>(p, b, h, qg);
-        vs[128 + cc] = row_D<EPI>(p, b, h, qg);
+      if (*abort_flag) {
+        const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+        for (int u = max(0, ii - QB); u < ii; ++u) mbar_wait(qd_full + u % QB, (u / QB) & 1, drain);
+        for (int u = max(0, tk_ - S); u < tk_; ++u) mbar_wait(kv_full + u % S, (u / S) & 1, drain);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_full + s);
-      issued = i + 1;
-    }
-    if (lane == 0 && *abort_flag) {
-      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
-      mbar_wait(kv_full, 0, drain);
-      for (int i = max(0, issued - S); i < issued; ++i) mbar_wait(q_full + i % S, (i / S) & 1, drain);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_ss = idesc_bf16_f32(128, 128, false);
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
-      const uint32_t k_base = smem_u32(smem + L::kK);
-      const uint32_t v_base = smem_u32(smem + L::kV);
-      const uint32_t t_dv = tmem + 256, t_dk = tmem + 256 + D;
-      bool ok = mbar_wait(kv_full, 0, wctx);
-      tc_fence_after();
-      for (int i = 0; ok && i <= n; ++i) {
-        if (i >= 1) {
-          const int ii = i - 1, s2 = ii % S;
-          if (!(ok = mbar_wait(p_full, ii & 1, wctx))) break;
-          tc_fence_after();
-          const uint32_t q_s = smem_u32(smem + L::kQ + s2 * L::kTileBytes);
-          const uint32_t do_s = smem_u32(smem + L::kDO + s2 * L::kTileBytes);
+      constexpr uint32_t idesc_half = idesc_bf16_f32(128, 64, false);  // S / dP halves
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);     // dQ
+      constexpr bool kDeferAcc = D == 64;  // as in the dK / dV kernel
+      bool ok = true;
+      auto acc_half = [&](int h, int t_, int s, int ab, bool first, int item) -> bool {
+        if (!mbar_wait(ds_full + h, t_ & 1, wctx)) return false;
+        if (h == 0 && first && item >= ACB &&
+            !mbar_wait(acc_empty + ab, ((item / ACB) - 1) & 1, wctx))
+          return false;
+        tc_fence_after();
+        const uint32_t k_s = smem_u32(smem + L::kK + s * L::kTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t a_col = (kk >> 2) * 64 + (kk & 3) * 8;
-            const uint32_t acc = (ii > 0 || kk > 0) ? 1u : 0u;
-            mma_ts(t_dv, tmem + a_col, smem_desc_sw128(do_s + kk * 2048, L::kBoxBytes, 1024),
-                   idesc_acc, acc);
-            mma_ts(t_dk, tmem + 128 + a_col, smem_desc_sw128(q_s + kk * 2048, L::kBoxBytes, 1024),
-                   idesc_acc, acc);
-          }
-          mma_commit(q_empty + s2);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + 256 + ab * D, tmem + 128 + 64 * h + kk * 8,
+                 smem_desc_sw128(k_s + (4 * h + kk) * 2048, L::kBoxBytes, 1024), idesc_acc,
+                 (first && h == 0 && kk == 0) ? 0u : 1u);
+        return true;
+      };
+      auto sdp_half = [&](int h, uint32_t q_base, uint32_t do_base, uint32_t k_s, uint32_t v_s) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
+          mma_ss(tmem + 64 * h, smem_desc_sw128(q_base + off, 16, 1024),
+                 smem_desc_sw128(k_s + off + h * 8192, 16, 1024), idesc_half, kk > 0);
         }
-        if (i < n) {
-          const int s = i % S;
-          if (!(ok = mbar_wait(q_full + s, (i / S) & 1, wctx))) break;
-          tc_fence_after();
-          const uint32_t q_s = smem_u32(smem + L::kQ + s * L::kTileBytes);
-          const uint32_t do_s = smem_u32(smem + L::kDO + s * L::kTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-            mma_ss(tmem, smem_desc_sw128(k_base + off, 16, 1024),
-                   smem_desc_sw128(q_s + off, 16, 1024), idesc_ss, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-            mma_ss(tmem + 128, smem_desc_sw128(v_base + off, 16, 1024),
-                   smem_desc_sw128(do_s + off, 16, 1024), idesc_ss, kk > 0);
-          }
-          mma_commit(s_full);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
+          mma_ss(tmem + 128 + 64 * h, smem_desc_sw128(do_base + off, 16, 1024),
+                 smem_desc_sw128(v_s + off + h * 8192, 16, 1024), idesc_half, kk > 0);
         }
+        mma_commit(s_full + h);
+      };
+      int pend_t = -1, pend_s = 0, pend_ab = 0, pend_item = 0;
+      bool pend_first = false, pend_last = false;
+      auto finish_pending = [&]() {
+        mma_commit(kv_empty + pend_s);
+        if (pend_last) mma_commit(acc_full + pend_ab);
+      };
+      int tk_ = 0, ii = 0;
+      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
+        const WorkRef it = decode_row(p, w);
+        if (it.n == 0) continue;
+        const int qb = ii % QB, ab = ii % ACB;
+        if (kDeferAcc && pend_t >= 0) {
+          if (!(ok = acc_half(0, pend_t, pend_s, pend_ab, pend_first, pend_item) &&
+                     acc_half(1, pend_t, pend_s, pend_ab, pend_first, pend_item)))
+            break;
+          finish_pending();
+          pend_t = -1;
+        }
+        if (!(ok = mbar_wait(qd_full + qb, (ii / QB) & 1, wctx))) break;
+        tc_fence_after();
+        const uint32_t q_base = smem_u32(smem + L::kQ + qb * L::kTileBytes);
+        const uint32_t do_base = smem_u32(smem + L::kDO + qb * L::kTileBytes);
+        for (int j = 0; j < it.n; ++j, ++tk_) {
+          const int s = tk_ % S;
+          if (!(ok = mbar_wait(kv_full + s, (tk_ / S) & 1, wctx))) break;
+          tc_fence_after();
+          const uint32_t k_s = smem_u32(smem + L::kK + s * L::kTileBytes);
+          const uint32_t v_s = smem_u32(smem + L::kV + s * L::kTileBytes);
+          if (kDeferAcc) {
+            for (int h = 0; h < 2 && ok; ++h) {
+              if (pend_t >= 0 &&
+                  !(ok = acc_half(h, pend_t, pend_s, pend_ab, pend_first, pend_item)))
+                break;
+              sdp_half(h, q_base, do_base, k_s, v_s);
+            }
+            if (!ok) break;
+            if (pend_t >= 0) finish_pending();
+            if (j == it.n - 1) mma_commit(qd_empty + qb);
+            pend_t = tk_;
+            pend_s = s;
+            pend_ab = ab;
+            pend_item = ii;
+            pend_first = j == 0;
+            pend_last = j == it.n - 1;
+          } else {
+            sdp_half(0, q_base, do_base, k_s, v_s);
+            sdp_half(1, q_base, do_base, k_s, v_s);
+            if (!(ok = acc_half(0, tk_, s, ab, j == 0, ii) && acc_half(1, tk_, s, ab, j == 0, ii)))
+              break;
+            mma_commit(kv_empty + s);
+            if (j == it.n - 1) {
+              mma_commit(acc_full + ab);
+              mma_commit(qd_empty + qb);
+            }
+          }
+        }
+        ++ii;
       }
-      mma_commit(acc_full);
+      if (kDeferAcc && ok && pend_t >= 0 &&
+          acc_half(0, pend_t, pend_s, pend_ab, pend_first, pend_item) &&
+          acc_half(1, pend_t, pend_s, pend_ab, pend_first, pend_item))
+        finish_pending();
     }
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- epilogue
-    const int g = (warp - kEpiWarp0) >> 2;
+    const int h = (warp - kEpiWarp0) >> 2;  // key half of every tile
     const int wq = warp & 3;
-    const int row = wq * 32 + lane;  // key row of the tile
-    const int kg = kt * kTile + row;
+    const int row = wq * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const float c1 = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
+    const float c1s = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
+    const float2 c1 = make_float2(c1s, c1s);
     bool ok = true;
-    for (int i = 0; i < n; ++i) {
-      const int s = i % S;
-      if (ok) ok = mbar_wait(q_full + s, (i / S) & 1, wctx);
-      if (ok) ok = mbar_wait(s_full, i & 1, wctx);
+    int tk_ = 0, ii = 0;
+    for (int w = blockIdx.x; w < nitems; w += gridDim.x) {
+      const WorkRef it = decode_row(p, w);
+      if (it.n == 0) {
+        const int rows = min(kTile, p.Nq - it.t * kTile);
+        zero_rows<D>(p.dq + it.b * p.dq_sb + static_cast<int64_t>(it.t * kTile) * p.dq_sn +
+                         it.h * p.dq_sh, p.dq_sn, rows, threadIdx.x - kEpiWarp0 * 32, 256);
+        continue;
+      }
+      if (!ok) break;
+      const int ab = ii % ACB;
+      const int qg = it.t * kTile + row;
+      const float off = row_offset<EPI>(p, it.b, it.h, qg);
+      const float Drow = row_D<EPI>(p, it.b, it.h, qg);
+      const float2 off2 = make_float2(off, off), D2 = make_float2(Drow, Drow);
+      for (int j = 0; j < it.n; ++j, ++tk_) {
+        const int e = it.e0 + j;
+        const int kd = p.kind[e];
+        uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+        if (kd == 2)
+          mb = *reinterpret_cast<const uint2*>(p.bits + static_cast<int64_t>(p.pidx[e]) * 512 +
+                                               row * 4 + 2 * h);
+        if (ok) ok = mbar_wait(s_full + h, tk_ & 1, wctx);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[2][32], dpr[2][32];
+        tmem_ld32(t_lane + 64 * h, sr[0]);
+        tmem_ld32(t_lane + 128 + 64 * h, dpr[0]);
+        tmem_wait_ld();
+        tmem_ld32(t_lane + 64 * h + 32, sr[1]);
+        tmem_ld32(t_lane + 128 + 64 * h + 32, dpr[1]);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (c == 1) tmem_wait_ld();
+          const uint32_t mw = c ? mb.y : mb.x;
+          uint32_t dk[16];
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            float2 pw, ds;
+            weight_grad2<EPI>(make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
+                              make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])),
+                              c1, off2, D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
+            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+          }
+          tmem_st16(t_lane + 128 + 64 * h + 16 * c, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_full + h);
+      }
+      if (!ok) break;
+      ok = mbar_wait(acc_full + ab, (ii / ACB) & 1, wctx);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int e = p.csc_map[e0 + i];
-      const int kd = p.kind[e];
-      uint32_t mw0 = 0xFFFFFFFFu, mw1 = 0xFFFFFFFFu;
-      if (kd == 2) {
-        const uint2 mb = *reinterpret_cast<const uint2*>(
-            p.bitsT + static_cast<int64_t>(p.pidx[e]) * 512 + row * 4 + g * 2);
-        mw0 = mb.x;
-        mw1 = mb.y;
-      }
-      const float* vs = vec + s * 256 + g * 64;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int col = g * 64 + half * 32;
-        uint32_t sr[32], dpr[32];
-        tmem_ld32(t_lane + col, sr);
-        tmem_ld32(t_lane + 128 + col, dpr);
-        tmem_wait_ld();
-        const uint32_t mw = half ? mw1 : mw0;
-        uint32_t pk[16], dk[16];
-#pragma unroll
-        for (int cc = 0; cc < 32; cc += 2) {
-          float p0, p1, d0, d1;
-          weight_grad<EPI>(__uint_as_float(sr[cc]), __uint_as_float(dpr[cc]), c1,
-                           vs[half * 32 + cc], vs[128 + half * 32 + cc], (mw >> cc) & 1u, p0, d0);
-          weight_grad<EPI>(__uint_as_float(sr[cc + 1]), __uint_as_float(dpr[cc + 1]), c1,
-                           vs[half * 32 + cc + 1], vs[128 + half * 32 + cc + 1],
-                           (mw >> (cc + 1)) & 1u, p1, d1);
-          pk[cc >> 1] = pack_bf16x2(p0, p1);
-          dk[cc >> 1] = pack_bf16x2(d0, d1);
-        }
-        tmem_st16(t_lane + g * 64 + half * 16, pk);
-        tmem_st16(t_lane + 128 + g * 64 + half * 16, dk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-    if (ok) ok = mbar_wait(acc_full, 0, wctx);
-    ok = __all_sync(0xFFFFFFFFu, ok);
-    if (ok) {
-      tc_fence_after();
       constexpr int kOc = D / 2;
-      __nv_bfloat16* dvp = p.dv + b * p.dv_sb + static_cast<int64_t>(kg) * p.dv_sn + h * p.dv_sh + g * kOc;
-      __nv_bfloat16* dkp = p.dk + b * p.dk_sb + static_cast<int64_t>(kg) * p.dk_sn + h * p.dk_sh + g * kOc;
+      uint32_t pk[kOc / 2];
 #pragma unroll
       for (int c0 = 0; c0 < kOc; c0 += 32) {
         uint32_t acc[32];
-        tmem_ld32(t_lane + 256 + g * kOc + c0, acc);
+        tmem_ld32(t_lane + 256 + ab * D + h * kOc + c0, acc);
         tmem_wait_ld();
-        if (kg < p.Nk) store_row_bf16(dvp + c0, acc, 1.0f);
-        tmem_ld32(t_lane + 256 + D + g * kOc + c0, acc);
-        tmem_wait_ld();
-        if (kg < p.Nk) store_row_bf16(dkp + c0, acc, p.scale);
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pk[c0 / 2 + c] = pack_bf16x2(__uint_as_float(acc[2 * c]) * p.scale,
+                                       __uint_as_float(acc[2 * c + 1]) * p.scale);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + ab);
+      if (qg < p.Nq) {
+        uint4* dqp = reinterpret_cast<uint4*>(p.dq + it.b * p.dq_sb + static_cast<int64_t>(qg) * p.dq_sn +
+                                              it.h * p.dq_sh + h * kOc);
+#pragma unroll
+        for (int c = 0; c < kOc / 8; ++c)
+          dqp[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      ++ii;
     }
   }
   tc_fence_before();
@@ -405,230 +858,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, 512);
   }
 }
-
-// ---------------------------------------------------------------------------------------
-// dQ
-// ---------------------------------------------------------------------------------------
-template <int D>
-struct DqLayout {
-  static constexpr int kStages = D == 64 ? 4 : 2;
-  static constexpr int kBoxes = D / 64;
-  static constexpr int kBoxBytes = 128 * 128;
-  static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kQ = 0;
-  static constexpr int kDO = kTileBytes;
-  static constexpr int kK = 2 * kTileBytes;
-  static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBar = kV + kStages * kTileBytes;
-  // qd_full, acc_full, s_full, ds_full, kv_full[S], kv_empty[S]
-  static constexpr int kNumBars = 4 + 2 * kStages;
-  static constexpr int kMisc = kBar + 8 * kNumBars;
-  static constexpr int kBytes = kMisc + 16;
-  static constexpr int kAlloc = kBytes + 1024;
-};
-
-template <int D, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
-    dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
-              const BwdParams p) {
-  using L = DqLayout<D>;
-  constexpr int S = L::kStages;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  const int warp = warp_id(), lane = lane_id();
-  const int wi = blockIdx.x / p.H, h = blockIdx.x % p.H;
-  const int r = p.row_work[wi];
-  const int b = r / p.QT, qt = r % p.QT;
-  const int e0 = p.row_ptr[r];
-  const int n = p.row_ptr[r + 1] - e0;
-
-  if (n == 0) {
-    const int rows = min(kTile, p.Nq - qt * kTile);
-    zero_rows<D>(p.dq + b * p.dq_sb + static_cast<int64_t>(qt * kTile) * p.dq_sn + h * p.dq_sh,
-                 p.dq_sn, rows, threadIdx.x, kThreads);
-    return;
-  }
-
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* qd_full = bars + 0;
-  uint64_t* acc_full = bars + 1;
-  uint64_t* s_full = bars + 2;
-  uint64_t* ds_full = bars + 3;
-  uint64_t* kv_full = bars + 4;
-  uint64_t* kv_empty = bars + 4 + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  volatile int* drain_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
-  const WaitCtx wctx{p.status, p.wait_ns, abort_flag};
-
-  if (threadIdx.x == 0) {
-    mbar_init(qd_full, 1);
-    mbar_init(acc_full, 1);
-    mbar_init(s_full, 1);
-    mbar_init(ds_full, 8);
-    for (int i = 0; i < S; ++i) {
-      mbar_init(kv_full + i, 1);
-      mbar_init(kv_empty + i, 1);
+int num_sms() {
+  static int sms = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      sms = 148;
     }
-    *abort_flag = 0;
-    *drain_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tq);
-      tma_prefetch_desc(&tk);
-      tma_prefetch_desc(&tv);
-      tma_prefetch_desc(&tdo);
-      mbar_arrive_expect_tx(qd_full, 2 * L::kTileBytes);
-      for (int x = 0; x < L::kBoxes; ++x) {
-        tma_load_4d(smem + L::kQ + x * L::kBoxBytes, &tq, qd_full, x * 64, qt * kTile, h, b);
-        tma_load_4d(smem + L::kDO + x * L::kBoxBytes, &tdo, qd_full, x * 64, qt * kTile, h, b);
-      }
-      int issued = 0;
-      for (int j = 0; j < n; ++j) {
-        const int s = j % S;
-        if (j >= S && !mbar_wait(kv_empty + s, ((j / S) - 1) & 1, wctx)) break;
-        const int kt = p.col_idx[e0 + j];
-        mbar_arrive_expect_tx(kv_full + s, 2 * L::kTileBytes);
-        for (int x = 0; x < L::kBoxes; ++x) {
-          tma_load_4d(smem + L::kK + s * L::kTileBytes + x * L::kBoxBytes, &tk, kv_full + s,
-                      x * 64, kt * kTile, h, b);
-          tma_load_4d(smem + L::kV + s * L::kTileBytes + x * L::kBoxBytes, &tv, kv_full + s,
-                      x * 64, kt * kTile, h, b);
-        }
-        issued = j + 1;
-      }
-      if (*abort_flag) {
-        const WaitCtx drain{p.status, p.wait_ns, drain_flag};
-        mbar_wait(qd_full, 0, drain);
-        for (int j = max(0, issued - S); j < issued; ++j) mbar_wait(kv_full + j % S, (j / S) & 1, drain);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_ss = idesc_bf16_f32(128, 128, false);
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
-      const uint32_t q_base = smem_u32(smem + L::kQ);
-      const uint32_t do_base = smem_u32(smem + L::kDO);
-      const uint32_t t_dq = tmem + 256;
-      bool ok = mbar_wait(qd_full, 0, wctx);
-      tc_fence_after();
-      for (int j = 0; ok && j <= n; ++j) {
-        if (j >= 1) {
-          const int jj = j - 1, s2 = jj % S;
-          if (!(ok = mbar_wait(ds_full, jj & 1, wctx))) break;
-          tc_fence_after();
-          const uint32_t k_s = smem_u32(smem + L::kK + s2 * L::kTileBytes);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t a_col = 128 + (kk >> 2) * 64 + (kk & 3) * 8;
-            mma_ts(t_dq, tmem + a_col, smem_desc_sw128(k_s + kk * 2048, L::kBoxBytes, 1024),
-                   idesc_acc, (jj > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(kv_empty + s2);
-        }
-        if (j < n) {
-          const int s = j % S;
-          if (!(ok = mbar_wait(kv_full + s, (j / S) & 1, wctx))) break;
-          tc_fence_after();
-          const uint32_t k_s = smem_u32(smem + L::kK + s * L::kTileBytes);
-          const uint32_t v_s = smem_u32(smem + L::kV + s * L::kTileBytes);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-            mma_ss(tmem, smem_desc_sw128(q_base + off, 16, 1024),
-                   smem_desc_sw128(k_s + off, 16, 1024), idesc_ss, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-            mma_ss(tmem + 128, smem_desc_sw128(do_base + off, 16, 1024),
-                   smem_desc_sw128(v_s + off, 16, 1024), idesc_ss, kk > 0);
-          }
-          mma_commit(s_full);
-        }
-      }
-      mma_commit(acc_full);
-    }
-  } else if (warp >= kEpiWarp0) {
-    const int g = (warp - kEpiWarp0) >> 2;
-    const int wq = warp & 3;
-    const int row = wq * 32 + lane;
-    const int qg = qt * kTile + row;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const float c1 = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
-    const float off = row_offset<EPI>(p, b, h, qg);
-    const float Drow = row_D<EPI>(p, b, h, qg);
-    bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      if (ok) ok = mbar_wait(s_full, j & 1, wctx);
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      const int e = e0 + j;
-      const int kd = p.kind[e];
-      uint32_t mw0 = 0xFFFFFFFFu, mw1 = 0xFFFFFFFFu;
-      if (kd == 2) {
-        const uint2 mb = *reinterpret_cast<const uint2*>(
-            p.bits + static_cast<int64_t>(p.pidx[e]) * 512 + row * 4 + g * 2);
-        mw0 = mb.x;
-        mw1 = mb.y;
-      }
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int col = g * 64 + half * 32;
-        uint32_t sr[32], dpr[32];
-        tmem_ld32(t_lane + col, sr);
-        tmem_ld32(t_lane + 128 + col, dpr);
-        tmem_wait_ld();
-        const uint32_t mw = half ? mw1 : mw0;
-        uint32_t dk[16];
-#pragma unroll
-        for (int cc = 0; cc < 32; cc += 2) {
-          float p0, p1, d0, d1;
-          weight_grad<EPI>(__uint_as_float(sr[cc]), __uint_as_float(dpr[cc]), c1, off, Drow,
-                           (mw >> cc) & 1u, p0, d0);
-          weight_grad<EPI>(__uint_as_float(sr[cc + 1]), __uint_as_float(dpr[cc + 1]), c1, off,
-                           Drow, (mw >> (cc + 1)) & 1u, p1, d1);
-          dk[cc >> 1] = pack_bf16x2(d0, d1);
-        }
-        tmem_st16(t_lane + 128 + g * 64 + half * 16, dk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
-    }
-    if (ok) ok = mbar_wait(acc_full, 0, wctx);
-    ok = __all_sync(0xFFFFFFFFu, ok);
-    if (ok) {
-      tc_fence_after();
-      constexpr int kOc = D / 2;
-      __nv_bfloat16* dqp = p.dq + b * p.dq_sb + static_cast<int64_t>(qg) * p.dq_sn + h * p.dq_sh + g * kOc;
-#pragma unroll
-      for (int c0 = 0; c0 < kOc; c0 += 32) {
-        uint32_t acc[32];
-        tmem_ld32(t_lane + 256 + g * kOc + c0, acc);
-        tmem_wait_ld();
-        if (qg < p.Nq) store_row_bf16(dqp + c0, acc, p.scale);
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
+  });
+  return sms;
 }
 
 template <int D, int EPI>
@@ -650,6 +891,7 @@ int launch_bwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.csc_map = plan->csc_map;
   p.row_work = plan->row_work;
   p.col_work = plan->col_work;
+  p.B = plan->B;
   p.QT = plan->QT;
   p.KT = plan->KT;
   p.Nq = plan->Nq;
@@ -688,8 +930,8 @@ int launch_bwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
     if ((e = cudaFuncSetAttribute(kdkv, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   DkvLayout<D>::kAlloc)) != cudaSuccess)
       return cuda_status(e);
-    kdkv<<<static_cast<unsigned>(static_cast<int64_t>(plan->B) * plan->KT * H), kThreads,
-           DkvLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    const int items = plan->B * plan->KT * H;
+    kdkv<<<std::min(items, num_sms()), kThreads, DkvLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   if (parts & SIGATTN_BWD_DQ) {
@@ -697,8 +939,8 @@ int launch_bwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
     if ((e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   DqLayout<D>::kAlloc)) != cudaSuccess)
       return cuda_status(e);
-    kdq<<<static_cast<unsigned>(static_cast<int64_t>(plan->B) * plan->QT * H), kThreads,
-          DqLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    const int items = plan->B * plan->QT * H;
+    kdq<<<std::min(items, num_sms()), kThreads, DqLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   return SIGATTN_OK;

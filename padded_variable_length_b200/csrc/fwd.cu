@@ -4,23 +4,29 @@
 // Method: "Better Models, Faster Training: Sigmoid Attention for single-cell Foundation
 // Models", section 2A: O = sigma(Q K^T / sqrt(d) + b) V, each weight computed on its own
 // with no row normalisation; section 2C: one fused kernel that skips every tile that is
-// padding on the query or the key side.  softmax and softmax_1 (the QuietAttention page,
-// section "Proposition : softmax_1 et QuietAttention") run through the same kernel with
-// the online max / sum recombination of the FlashAttention article (section on the
-// mathematics of blockwise softmax); softmax_1 starts from a zero logit whose value row is
-// zero (m = 0, l = 1).
+// padding on the query or the key side, with the sigmoid on the hardware tanh
+// approximation.  softmax and softmax_1 (the QuietAttention page, section "Proposition :
+// softmax_1 et QuietAttention") run through the same kernel with the online max / sum
+// recombination of the FlashAttention article (section on the mathematics of blockwise
+// softmax); softmax_1 starts from a zero logit whose value row is zero (m = 0, l = 1).
 //
-// One CTA per (q-tile row of the plan, head), 384 threads:
-//   warp 0      TMA producer: Q once, then K and V tiles of each listed k-tile into a ring
-//   warp 1      TMEM allocator and MMA issuer (one thread): S = Q K^T into one of two
-//               TMEM S buffers, then O += P V with P read from TMEM
+// Persistent: one CTA per SM walks the plan's longest-first list of (q-tile row, head)
+// work items with a stride of the grid size.  All tiles of all of a CTA's items form one
+// stream: the S = Q K^T of tile t is issued before the O += P V of tile t - 1, also across
+// item boundaries, so the tensor pipe works on the next item while the epilogue finishes
+// the last one.  384 threads:
+//   warp 0      TMA producer: Q of each item (two buffers), K and V tiles into a ring
+//   warp 1      TMEM allocator and MMA issuer (one thread)
 //   warps 4-11  two epilogue warpgroups; thread = query row (TMEM lane); warpgroup g
 //               owns S columns [64g, 64g+64) and O columns [g d/2, (g+1) d/2)
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+d).  P (bf16) overwrites the first
-// half of the columns each warpgroup read, so the two warpgroups never touch each
-// other's S values.
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256, 256+d), O1 [256+d, 256+2d).  P (bf16)
+// overwrites the first half of the S columns each warpgroup read and is the TMEM A
+// operand of the PV MMA.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -41,7 +47,7 @@ struct FwdParams {
   const int32_t* pidx;
   const uint32_t* bits;
   const int32_t* row_work;
-  int QT, Nq, H;
+  int QT, Nq, H, nitems;
   float scale;
   const float* bias;
   int64_t bias_sb;
@@ -58,18 +64,34 @@ struct FwdLayout {
   static constexpr int kBoxes = D / 64;
   static constexpr int kBoxBytes = 128 * 128;  // 128 rows x 64 bf16
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kTileBytes;
+  static constexpr int kQ = 0;                  // two Q buffers
+  static constexpr int kK = 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kBar = kV + kStages * kTileBytes;
-  // barriers: q_full, o_full, pv_done, s_full[2], p_full[2], k_full[S], v_full[S], kv_empty[S]
-  static constexpr int kNumBars = 7 + 3 * kStages;
-  static constexpr int kRed = kBar + 8 * kNumBars;          // float [2][2][128] row maxima
-  static constexpr int kRedL = kRed + 2 * 2 * 128 * 4;      // float [2][128] row sums
-  static constexpr int kMisc = kRedL + 2 * 128 * 4;          // tmem base, abort flag
+  // q_full[2] q_empty[2] o_full[2] o_empty[2] s_full[2] p_full[2] pv_done
+  // k_full[S] v_full[S] kv_empty[S]
+  static constexpr int kNumBars = 13 + 3 * kStages;
+  static constexpr int kRed = kBar + 8 * kNumBars;      // float [2][2][128] row maxima
+  static constexpr int kRedL = kRed + 2 * 2 * 128 * 4;  // float [2][128] row sums
+  static constexpr int kMisc = kRedL + 2 * 128 * 4;      // tmem base, abort, drain flags
   static constexpr int kBytes = kMisc + 16;
-  static constexpr int kAlloc = kBytes + 1024;               // slack for 1024-byte alignment
+  static constexpr int kAlloc = kBytes + 1024;           // slack for 1024-byte alignment
 };
+
+struct Item {
+  int b, qt, h, e0, n;
+};
+
+__device__ __forceinline__ Item decode_item(const FwdParams& p, int w) {
+  Item it;
+  const int r = p.row_work[w / p.H];
+  it.h = w % p.H;
+  it.b = r / p.QT;
+  it.qt = r % p.QT;
+  it.e0 = p.row_ptr[r];
+  it.n = p.row_ptr[r + 1] - it.e0;
+  return it;
+}
 
 template <int D, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -81,60 +103,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
-  const int w = blockIdx.x / p.H, h = blockIdx.x % p.H;
-  const int r = p.row_work[w];
-  const int b = r / p.QT, qt = r % p.QT;
-  const int e0 = p.row_ptr[r];
-  const int n = p.row_ptr[r + 1] - e0;
-
-  if (n == 0) {
-    // No tile in this row: the whole q-tile is padding or sees no key.  O = 0.
-    const int rows = min(kTile, p.Nq - qt * kTile);
-    constexpr int kChunks = D / 8;  // 16-byte chunks per row
-    for (int i = threadIdx.x; i < rows * kChunks; i += kThreads) {
-      const int row = i / kChunks, c = i % kChunks;
-      __nv_bfloat16* dst = p.o + b * p.o_sb + static_cast<int64_t>(qt * kTile + row) * p.o_sn +
-                           h * p.o_sh + c * 8;
-      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    if (EPI != 0) {
-      const float v = EPI == 1 ? -INFINITY : 0.0f;
-      for (int i = threadIdx.x; i < rows; i += kThreads)
-        p.lse[(static_cast<int64_t>(b) * p.H + h) * p.Nq + qt * kTile + i] = v;
-    }
-    return;
-  }
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* q_full = bars + 0;
-  uint64_t* o_full = bars + 1;
-  uint64_t* pv_done = bars + 2;
-  uint64_t* s_full = bars + 3;   // [2]
-  uint64_t* p_full = bars + 5;   // [2]
-  uint64_t* k_full = bars + 7;   // [S]
-  uint64_t* v_full = bars + 7 + S;
-  uint64_t* kv_empty = bars + 7 + 2 * S;
+  uint64_t* q_full = bars + 0;    // [2]
+  uint64_t* q_empty = bars + 2;   // [2]
+  uint64_t* o_full = bars + 4;    // [2]
+  uint64_t* o_empty = bars + 6;   // [2]
+  uint64_t* s_full = bars + 8;    // [2]
+  uint64_t* p_full = bars + 10;   // [2]
+  uint64_t* pv_done = bars + 12;
+  uint64_t* k_full = bars + 13;   // [S]
+  uint64_t* v_full = bars + 13 + S;
+  uint64_t* kv_empty = bars + 13 + 2 * S;
   float* red_max = reinterpret_cast<float*>(smem + L::kRed);
   float* red_l = reinterpret_cast<float*>(smem + L::kRedL);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* drain_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
   const WaitCtx wctx{p.status, p.wait_ns, abort_flag};
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(o_full, 1);
-    mbar_init(pv_done, 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full + i, 1);
+      mbar_init(q_empty + i, 1);
+      mbar_init(o_full + i, 1);
+      mbar_init(o_empty + i, 8);
       mbar_init(s_full + i, 1);
       mbar_init(p_full + i, 8);
     }
+    mbar_init(pv_done, 1);
     for (int i = 0; i < S; ++i) {
       mbar_init(k_full + i, 1);
       mbar_init(v_full + i, 1);
       mbar_init(kv_empty + i, 1);
     }
     *abort_flag = 0;
-    *reinterpret_cast<volatile int*>(smem + L::kMisc + 8) = 0;  // drain flag
+    *drain_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
@@ -149,33 +153,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
-      mbar_arrive_expect_tx(q_full, L::kTileBytes);
-      for (int x = 0; x < L::kBoxes; ++x)
-        tma_load_4d(smem + L::kQ + x * L::kBoxBytes, &tq, q_full, x * 64, qt * kTile, h, b);
-      int issued = 0;
-      for (int j = 0; j < n; ++j) {
-        const int s = j % S;
-        if (j >= S && !mbar_wait(kv_empty + s, ((j / S) - 1) & 1, wctx)) break;
-        const int kt = p.col_idx[e0 + j];
-        mbar_arrive_expect_tx(k_full + s, L::kTileBytes);
+      int t = 0, i = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < p.nitems; w += gridDim.x) {
+        const Item it = decode_item(p, w);
+        if (it.n == 0) continue;
+        const int qb = i & 1;
+        if (i >= 2 && !(ok = mbar_wait(q_empty + qb, ((i >> 1) - 1) & 1, wctx))) break;
+        mbar_arrive_expect_tx(q_full + qb, L::kTileBytes);
         for (int x = 0; x < L::kBoxes; ++x)
-          tma_load_4d(smem + L::kK + s * L::kTileBytes + x * L::kBoxBytes, &tk, k_full + s,
-                      x * 64, kt * kTile, h, b);
-        mbar_arrive_expect_tx(v_full + s, L::kTileBytes);
-        for (int x = 0; x < L::kBoxes; ++x)
-          tma_load_4d(smem + L::kV + s * L::kTileBytes + x * L::kBoxBytes, &tv, v_full + s,
-                      x * 64, kt * kTile, h, b);
-        issued = j + 1;
+          tma_load_4d(smem + L::kQ + qb * L::kTileBytes + x * L::kBoxBytes, &tq, q_full + qb,
+                      x * 64, it.qt * kTile, it.h, it.b);
+        ++i;
+        for (int j = 0; j < it.n; ++j, ++t) {
+          const int s = t % S;
+          if (t >= S && !(ok = mbar_wait(kv_empty + s, ((t / S) - 1) & 1, wctx))) break;
+          const int kt = p.col_idx[it.e0 + j];
+          mbar_arrive_expect_tx(k_full + s, L::kTileBytes);
+          for (int x = 0; x < L::kBoxes; ++x)
+            tma_load_4d(smem + L::kK + s * L::kTileBytes + x * L::kBoxBytes, &tk, k_full + s,
+                        x * 64, kt * kTile, it.h, it.b);
+          mbar_arrive_expect_tx(v_full + s, L::kTileBytes);
+          for (int x = 0; x < L::kBoxes; ++x)
+            tma_load_4d(smem + L::kV + s * L::kTileBytes + x * L::kBoxBytes, &tv, v_full + s,
+                        x * 64, kt * kTile, it.h, it.b);
+        }
       }
       if (*abort_flag) {
         // Let the copies still in flight land before the CTA's shared memory goes away.
-        mbar_wait(q_full, 0, WaitCtx{p.status, p.wait_ns, reinterpret_cast<volatile int*>(
-                                                               smem + L::kMisc + 8)});
-        for (int j = max(0, issued - S); j < issued; ++j) {
-          const WaitCtx drain{p.status, p.wait_ns,
-                              reinterpret_cast<volatile int*>(smem + L::kMisc + 8)};
-          mbar_wait(k_full + j % S, (j / S) & 1, drain);
-          mbar_wait(v_full + j % S, (j / S) & 1, drain);
+        const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+        for (int u = max(0, i - 2); u < i; ++u) mbar_wait(q_full + (u & 1), (u >> 1) & 1, drain);
+        for (int u = max(0, t - S); u < t; ++u) {
+          mbar_wait(k_full + u % S, (u / S) & 1, drain);
+          mbar_wait(v_full + u % S, (u / S) & 1, drain);
         }
       }
     }
@@ -184,183 +194,239 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      const uint32_t q_base = smem_u32(smem + L::kQ);
-      bool ok = mbar_wait(q_full, 0, wctx);
-      tc_fence_after();
-      for (int j = 0; ok && j <= n; ++j) {
-        if (j < n) {
-          const int s = j % S;
-          if (!(ok = mbar_wait(k_full + s, (j / S) & 1, wctx))) break;
+      // the PV still to issue: its global tile, item number and place in the item
+      int pv_t = -1, pv_item = 0;
+      bool pv_first = false, pv_last = false;
+      bool ok = true;
+      auto issue_pv = [&]() -> bool {
+        const int pb = pv_t & 1, s2 = pv_t % S, ob = pv_item & 1;
+        if (!mbar_wait(p_full + pb, (pv_t >> 1) & 1, wctx)) return false;
+        if (!mbar_wait(v_full + s2, (pv_t / S) & 1, wctx)) return false;
+        if (pv_first && pv_item >= 2 && !mbar_wait(o_empty + ob, ((pv_item >> 1) - 1) & 1, wctx))
+          return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_u32(smem + L::kV + s2 * L::kTileBytes);
+        const uint32_t o_tmem = tmem + 256 + ob * D;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t a_tmem = tmem + pb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+          mma_ts(o_tmem, a_tmem, smem_desc_sw128(v_base + kk * 2048, L::kBoxBytes, 1024),
+                 idesc_pv, (pv_first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit(kv_empty + s2);
+        if (EPI != 0) mma_commit(pv_done);
+        if (pv_last) mma_commit(o_full + ob);
+        return true;
+      };
+      int t = 0, i = 0;
+      for (int w = blockIdx.x; ok && w < p.nitems; w += gridDim.x) {
+        const Item it = decode_item(p, w);
+        if (it.n == 0) continue;
+        const int qb = i & 1;
+        if (!(ok = mbar_wait(q_full + qb, (i >> 1) & 1, wctx))) break;
+        tc_fence_after();
+        const uint32_t q_base = smem_u32(smem + L::kQ + qb * L::kTileBytes);
+        for (int j = 0; j < it.n; ++j, ++t) {
+          const int s = t % S;
+          if (!(ok = mbar_wait(k_full + s, (t / S) & 1, wctx))) break;
           tc_fence_after();
           const uint32_t k_base = smem_u32(smem + L::kK + s * L::kTileBytes);
-          const uint32_t d_tmem = tmem + (j & 1) * 128;
+          const uint32_t d_tmem = tmem + (t & 1) * 128;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
             mma_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
                    smem_desc_sw128(k_base + off, 16, 1024), idesc_qk, kk > 0);
           }
-          mma_commit(s_full + (j & 1));
+          mma_commit(s_full + (t & 1));
+          if (j == it.n - 1) mma_commit(q_empty + qb);
+          if (pv_t >= 0 && !(ok = issue_pv())) break;
+          pv_t = t;
+          pv_item = i;
+          pv_first = j == 0;
+          pv_last = j == it.n - 1;
         }
-        if (j >= 1) {
-          const int jj = j - 1, s2 = jj % S, pb = jj & 1;
-          if (!(ok = mbar_wait(p_full + pb, (jj >> 1) & 1, wctx))) break;
-          if (!(ok = mbar_wait(v_full + s2, (jj / S) & 1, wctx))) break;
-          tc_fence_after();
-          const uint32_t v_base = smem_u32(smem + L::kV + s2 * L::kTileBytes);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t a_tmem = tmem + pb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
-            mma_ts(tmem + 256, a_tmem, smem_desc_sw128(v_base + kk * 2048, L::kBoxBytes, 1024),
-                   idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(kv_empty + s2);
-          if (EPI != 0) mma_commit(pv_done);
-        }
+        ++i;
       }
-      mma_commit(o_full);
+      if (ok && pv_t >= 0) issue_pv();
     }
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- epilogue
     const int g = (warp - kEpiWarp0) >> 2;  // warpgroup: S columns [64g, 64g+64)
     const int wq = warp & 3;                // TMEM lanes [32 wq, 32 wq + 32)
     const int row = wq * 32 + lane;
-    const int rg = qt * kTile + row;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const float bias_r = (p.bias != nullptr && rg < p.Nq) ? p.bias[b * p.bias_sb + rg] : 0.0f;
-    // sigmoid: sigma(x) = 0.5 + 0.5 tanh(x/2), x = scale s + bias -> (c1, c0) = halves;
-    // softmax: t = (scale s + bias) log2 e
-    const float c1 = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
-    const float c0 = EPI == 0 ? 0.5f * bias_r : bias_r * kLog2e;
-    float m_run = EPI == 2 ? 0.0f : kNegBig;  // base-2 running max (softmax modes)
-    float l_run = (EPI == 2 && g == 0) ? 1.0f : 0.0f;
+    constexpr int kOc = D / 2;  // O columns of this warpgroup
     // `ok` stays warp-uniform (tcgen05.ld/st are warp-collective).  After an abort the
-    // loop keeps running without touching TMEM so that every epilogue thread executes the
+    // loops keep running without touching TMEM so that every epilogue thread executes the
     // same sequence of named barriers (softmax modes) and nobody waits forever.
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int sb = j & 1;
-      if (ok) ok = mbar_wait(s_full + sb, (j >> 1) & 1, wctx);
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      if (ok) tc_fence_after();
-      const int e = e0 + j;
-      const int kd = p.kind[e];
-      uint32_t mw0 = 0xFFFFFFFFu, mw1 = 0xFFFFFFFFu;
-      if (kd == 2) {
-        const uint2 mb = *reinterpret_cast<const uint2*>(
-            p.bits + static_cast<int64_t>(p.pidx[e]) * 512 + row * 4 + g * 2);
-        mw0 = mb.x;
-        mw1 = mb.y;
-      }
-      uint32_t sr[64];
-      if (ok) {
-        tmem_ld32(t_lane + sb * 128 + g * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(t_lane + sb * 128 + g * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) sr[c] = 0u;
-      }
-      float pv[64];
-      if (EPI == 0) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float sg = sigmoid_tanh(__uint_as_float(sr[c]), c1, c0);
-          const uint32_t bit = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
-          pv[c] = bit ? sg : 0.0f;
+    int t = 0, i = 0;
+    for (int w = blockIdx.x; w < p.nitems; w += gridDim.x) {
+      const Item it = decode_item(p, w);
+      if (it.n == 0) {
+        // No tile in this row: the whole q-tile is padding or sees no key.  O = 0.
+        const int rows = min(kTile, p.Nq - it.qt * kTile);
+        constexpr int kChunks = D / 8;  // 16-byte chunks per row
+        const int tid = threadIdx.x - kEpiWarp0 * 32;
+        for (int c = tid; c < rows * kChunks; c += 256) {
+          const int rr = c / kChunks, ch = c % kChunks;
+          __nv_bfloat16* dst = p.o + it.b * p.o_sb +
+                               static_cast<int64_t>(it.qt * kTile + rr) * p.o_sn + it.h * p.o_sh +
+                               ch * 8;
+          *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
         }
-      } else {
-        float tmax = kNegBig;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float t = fmaf(__uint_as_float(sr[c]), c1, c0);
-          const uint32_t bit = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
-          pv[c] = bit ? t : kNegBig;
-          tmax = fmaxf(tmax, pv[c]);
+        if (EPI != 0)
+          for (int c = tid; c < rows; c += 256)
+            p.lse[(static_cast<int64_t>(it.b) * p.H + it.h) * p.Nq + it.qt * kTile + c] =
+                EPI == 1 ? -INFINITY : 0.0f;
+        continue;
+      }
+      const int ob = i & 1;
+      const int rg = it.qt * kTile + row;
+      const float bias_r =
+          (p.bias != nullptr && rg < p.Nq) ? p.bias[it.b * p.bias_sb + rg] : 0.0f;
+      // sigmoid: sigma(x) = 0.5 + 0.5 tanh(x/2), x = scale s + bias -> (c1, c0) = halves;
+      // softmax: t = (scale s + bias) log2 e
+      const float c1 = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
+      const float c0 = EPI == 0 ? 0.5f * bias_r : bias_r * kLog2e;
+      float m_run = EPI == 2 ? 0.0f : kNegBig;  // base-2 running max (softmax modes)
+      float l_run = (EPI == 2 && g == 0) ? 1.0f : 0.0f;
+      for (int j = 0; j < it.n; ++j, ++t) {
+        const int sb = t & 1;
+        if (ok) ok = mbar_wait(s_full + sb, (t >> 1) & 1, wctx);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (ok) tc_fence_after();
+        const int e = it.e0 + j;
+        const int kd = p.kind[e];
+        uint32_t mw0 = 0xFFFFFFFFu, mw1 = 0xFFFFFFFFu;
+        if (kd == 2) {
+          const uint2 mb = *reinterpret_cast<const uint2*>(
+              p.bits + static_cast<int64_t>(p.pidx[e]) * 512 + row * 4 + g * 2);
+          mw0 = mb.x;
+          mw1 = mb.y;
         }
-        red_max[(sb * 2 + g) * 128 + row] = tmax;
-        named_barrier_sync(1, 256);
-        tmax = fmaxf(tmax, red_max[(sb * 2 + (g ^ 1)) * 128 + row]);
-        // Lazy rescaling: keep the running max unless the tile's max exceeds it by more
-        // than 8 (base 2), so that exp2(t - m) stays <= 256; the result is exact either
-        // way because numerator and denominator share m.
-        const bool need = tmax > m_run + 8.0f;
-        const float m_new = need ? tmax : m_run;
-        const float alpha = ex2_approx(m_run - m_new);
-        if (ok && __any_sync(0xFFFFFFFFu, need) && j > 0) {
-          // O must not be read while PV_{j-1} may still accumulate into it.
-          ok = mbar_wait(pv_done, (j - 1) & 1, wctx);
-          ok = __all_sync(0xFFFFFFFFu, ok);
-          if (ok) {
-            tc_fence_after();
-            constexpr int kOc = D / 2;  // O columns of this warpgroup
+        uint32_t sr[64];
+        if (ok) {
+          tmem_ld32(t_lane + sb * 128 + g * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(t_lane + sb * 128 + g * 64 + 32,
+                    *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-            for (int c0o = 0; c0o < kOc; c0o += 32) {
-              uint32_t orr[32];
-              tmem_ld32(t_lane + 256 + g * kOc + c0o, orr);
-              tmem_wait_ld();
+          for (int c = 0; c < 64; ++c) sr[c] = 0u;
+        }
+        float pv[64];
+        if (EPI == 0) {
+          if (kd == 2) {
 #pragma unroll
-              for (int c = 0; c < 32; ++c)
-                orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-              tmem_st32(t_lane + 256 + g * kOc + c0o, orr);
+            for (int c = 0; c < 64; ++c) {
+              const float sg = sigmoid_tanh(__uint_as_float(sr[c]), c1, c0);
+              const uint32_t bit = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
+              pv[c] = bit ? sg : 0.0f;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) pv[c] = sigmoid_tanh(__uint_as_float(sr[c]), c1, c0);
+          }
+        } else {
+          float tmax = kNegBig;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float tt = fmaf(__uint_as_float(sr[c]), c1, c0);
+            const uint32_t bit = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
+            pv[c] = bit ? tt : kNegBig;
+            tmax = fmaxf(tmax, pv[c]);
+          }
+          red_max[(sb * 2 + g) * 128 + row] = tmax;
+          named_barrier_sync(1, 256);
+          tmax = fmaxf(tmax, red_max[(sb * 2 + (g ^ 1)) * 128 + row]);
+          // Lazy rescaling: keep the running max unless the tile's max exceeds it by more
+          // than 8 (base 2), so that exp2(t - m) stays <= 256; the result is exact either
+          // way because numerator and denominator share m.
+          const bool need = tmax > m_run + 8.0f;
+          const float m_new = need ? tmax : m_run;
+          const float alpha = ex2_approx(m_run - m_new);
+          if (ok && __any_sync(0xFFFFFFFFu, need) && j > 0) {
+            // O must not be read while PV of the previous tile may still accumulate into it.
+            ok = mbar_wait(pv_done, (t - 1) & 1, wctx);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (ok) {
+              tc_fence_after();
+#pragma unroll
+              for (int c0o = 0; c0o < kOc; c0o += 32) {
+                uint32_t orr[32];
+                tmem_ld32(t_lane + 256 + ob * D + g * kOc + c0o, orr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                  orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+                tmem_st32(t_lane + 256 + ob * D + g * kOc + c0o, orr);
+              }
             }
           }
-        }
-        l_run *= alpha;
-        m_run = m_new;
+          l_run *= alpha;
+          m_run = m_new;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float e2 = pv[c] > 0.5f * kNegBig ? ex2_approx(pv[c] - m_run) : 0.0f;
-          pv[c] = e2;
-          l_run += e2;
+          for (int c = 0; c < 64; ++c) {
+            const float e2 = pv[c] > 0.5f * kNegBig ? ex2_approx(pv[c] - m_run) : 0.0f;
+            pv[c] = e2;
+            l_run += e2;
+          }
+        }
+        if (ok) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
+          tmem_st32(t_lane + sb * 128 + g * 64, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full + sb);
+        }
+      }
+      // ---- output of this item: O (and LSE) from TMEM buffer ob
+      if (ok) ok = mbar_wait(o_full + ob, (i >> 1) & 1, wctx);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      float inv_l = 1.0f;
+      if (EPI != 0) {
+        red_l[g * 128 + row] = l_run;
+        named_barrier_sync(1, 256);
+        const float l_tot = l_run + red_l[(g ^ 1) * 128 + row];
+        named_barrier_sync(1, 256);  // red_l is rewritten by the next item
+        inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
+        if (ok && g == 0 && rg < p.Nq) {
+          const float lse = l_tot > 0.0f ? (m_run + __log2f(l_tot)) * kLn2 : -INFINITY;
+          p.lse[(static_cast<int64_t>(it.b) * p.H + it.h) * p.Nq + rg] = lse;
         }
       }
       if (ok) {
-        uint32_t pk[32];
+        tc_fence_after();
+        uint32_t pk[kOc / 2];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
-        tmem_st32(t_lane + sb * 128 + g * 64, pk);
-        tmem_wait_st();
+        for (int c0o = 0; c0o < kOc; c0o += 32) {
+          uint32_t orr[32];
+          tmem_ld32(t_lane + 256 + ob * D + g * kOc + c0o, orr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            pk[c0o / 2 + c] = pack_bf16x2(__uint_as_float(orr[2 * c]) * inv_l,
+                                          __uint_as_float(orr[2 * c + 1]) * inv_l);
+        }
+        // O buffer ob may be overwritten by item i + 2 from here on
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + sb);
-      }
-    }
-    if (ok) ok = mbar_wait(o_full, 0, wctx);
-    ok = __all_sync(0xFFFFFFFFu, ok);
-    float inv_l = 1.0f;
-    if (EPI != 0) {
-      red_l[g * 128 + row] = l_run;
-      named_barrier_sync(1, 256);
-      const float l_tot = l_run + red_l[(g ^ 1) * 128 + row];
-      inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
-      if (ok && g == 0 && rg < p.Nq) {
-        const float lse = l_tot > 0.0f ? (m_run + __log2f(l_tot)) * kLn2 : -INFINITY;
-        p.lse[(static_cast<int64_t>(b) * p.H + h) * p.Nq + rg] = lse;
-      }
-    }
-    if (ok) {
-      tc_fence_after();
-      constexpr int kOc = D / 2;
-      __nv_bfloat16* dst = p.o + b * p.o_sb + static_cast<int64_t>(rg) * p.o_sn + h * p.o_sh +
-                           g * kOc;
-#pragma unroll
-      for (int c0o = 0; c0o < kOc; c0o += 32) {
-        uint32_t orr[32];
-        tmem_ld32(t_lane + 256 + g * kOc + c0o, orr);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          pk[c] = pack_bf16x2(__uint_as_float(orr[2 * c]) * inv_l,
-                              __uint_as_float(orr[2 * c + 1]) * inv_l);
+        if (lane == 0) mbar_arrive(o_empty + ob);
         if (rg < p.Nq) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c0o);
+          uint4* d4 = reinterpret_cast<uint4*>(p.o + it.b * p.o_sb +
+                                               static_cast<int64_t>(rg) * p.o_sn + it.h * p.o_sh +
+                                               g * kOc);
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < kOc / 8; ++c)
             d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         }
       }
+      ++i;
     }
   }
   tc_fence_before();
@@ -369,6 +435,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+int num_sms() {
+  static int sms = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      sms = 148;
+    }
+  });
+  return sms;
 }
 
 template <int D, int EPI>
@@ -387,6 +467,7 @@ int launch_fwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.QT = plan->QT;
   p.Nq = plan->Nq;
   p.H = H;
+  p.nitems = plan->B * plan->QT * H;
   p.scale = scale;
   p.bias = bias;
   p.bias_sb = bias_sb;
@@ -401,8 +482,8 @@ int launch_fwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return cuda_status(e);
-  const int64_t blocks = static_cast<int64_t>(plan->B) * plan->QT * H;
-  kern<<<static_cast<unsigned>(blocks), kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
+  const int grid = std::min(p.nitems, num_sms());
+  kern<<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
 }
 
