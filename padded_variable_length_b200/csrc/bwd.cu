@@ -42,8 +42,8 @@ struct BwdParams {
   const int32_t* colT_ptr;
   const int32_t* rowT_idx;
   const int32_t* csc_map;
-  const int32_t* row_work;
-  const int32_t* col_work;
+  const int4* row_desc;
+  const int4* col_desc;
   int B, QT, KT, Nq, Nk, H;
   float scale;
   const float* bias;
@@ -164,25 +164,45 @@ struct WorkRef {
 // dK/dV: item w -> (k-tile column, head); dQ: item w -> (q-tile row, head).
 __device__ __forceinline__ WorkRef decode_col(const BwdParams& p, int w) {
   WorkRef r;
-  const int c = p.col_work[w / p.H];
+  const int4 d = p.col_desc[w / p.H];
   r.h = w % p.H;
-  r.b = c / p.KT;
-  r.t = c % p.KT;
-  r.e0 = p.colT_ptr[c];
-  r.n = p.colT_ptr[c + 1] - r.e0;
+  r.b = d.x / p.KT;
+  r.t = d.x % p.KT;
+  r.e0 = d.y;
+  r.n = d.z;
   return r;
 }
 
 __device__ __forceinline__ WorkRef decode_row(const BwdParams& p, int w) {
   WorkRef r;
-  const int q = p.row_work[w / p.H];
+  const int4 d = p.row_desc[w / p.H];
   r.h = w % p.H;
-  r.b = q / p.QT;
-  r.t = q % p.QT;
-  r.e0 = p.row_ptr[q];
-  r.n = p.row_ptr[q + 1] - r.e0;
+  r.b = d.x / p.QT;
+  r.t = d.x % p.QT;
+  r.e0 = d.y;
+  r.n = d.z;
   return r;
 }
+
+// Walks this CTA's work items (stride = grid size) with the next item's decode issued one
+// item ahead, so that its global loads overlap the current item.
+template <bool kCols>
+struct WorkIter {
+  const BwdParams& p;
+  int w, nitems;
+  WorkRef cur, nxt;
+  __device__ WorkRef dec(int ww) const { return kCols ? decode_col(p, ww) : decode_row(p, ww); }
+  __device__ WorkIter(const BwdParams& pp, int n) : p(pp), w(blockIdx.x), nitems(n) {
+    if (w < nitems) cur = dec(w);
+    if (w + static_cast<int>(gridDim.x) < nitems) nxt = dec(w + gridDim.x);
+  }
+  __device__ bool valid() const { return w < nitems; }
+  __device__ void advance() {
+    w += gridDim.x;
+    cur = nxt;
+    if (w + static_cast<int>(gridDim.x) < nitems) nxt = dec(w + gridDim.x);
+  }
+};
 
 // ---------------------------------------------------------------------------------------
 // dK / dV: one item = one k-tile column of the plan for one head; thread = key row.
@@ -202,7 +222,10 @@ struct DkvLayout {
   static constexpr int kQ = kV + kKVBufs * kTileBytes;
   static constexpr int kDO = kQ + kStages * kTileBytes;
   static constexpr int kVec = kDO + kStages * kTileBytes;  // float [S][2][128]
-  static constexpr int kBar = kVec + kStages * 2 * 128 * 4;
+  // per Q/dO stage: the tile's transposed PARTIAL bitmask and its kind, staged by the producer
+  static constexpr int kMetaBits = kVec + kStages * 2 * 128 * 4;
+  static constexpr int kMetaKind = kMetaBits + kStages * 2048;
+  static constexpr int kBar = kMetaKind + 16 * ((kStages * 4 + 15) / 16);
   // kv_full[KV] kv_empty[KV] q_full[S] q_empty[S] s_full[2] p_full[2] acc_full[A] acc_empty[A]
   static constexpr int kNumBars = 2 * kKVBufs + 2 * kStages + 4 + 2 * kAccBufs;
   static constexpr int kMisc = kBar + 8 * kNumBars;
@@ -233,6 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = p_full + 2;  // [ACB]
   uint64_t* acc_empty = acc_full + ACB;
   float* vec = reinterpret_cast<float*>(smem + L::kVec);
+  uint32_t* meta_bits = reinterpret_cast<uint32_t*>(smem + L::kMetaBits);
+  int* meta_kind = reinterpret_cast<int*>(smem + L::kMetaKind);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   volatile int* drain_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
@@ -267,10 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
+    // Lane 0 waits and issues the copies.  All 32 lanes fetch the list entries of the next
+    // 32 q-tiles in one round trip and the column vectors (bias / LSE / D of the tile's 128
+    // queries) one tile ahead, so no global load sits between two copies.
     int qc = 0, ii = 0;
     bool ok = true;
-    for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
-      const WorkRef it = decode_col(p, w);
+    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
       if (it.n == 0) continue;
       const int kb = ii % KVB;
       if (lane == 0 && ii >= KVB) ok = mbar_wait(kv_empty + kb, ((ii / KVB) - 1) & 1, wctx);
@@ -286,29 +314,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       ++ii;
-      for (int i = 0; i < it.n; ++i, ++qc) {
-        const int s = qc % S;
-        if (lane == 0 && qc >= S) ok = mbar_wait(q_empty + s, ((qc / S) - 1) & 1, wctx);
-        ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-        if (!ok) break;
-        const int qt = p.rowT_idx[it.e0 + i];
-        if (lane == 0) {
-          mbar_arrive_expect_tx(q_full + s, 2 * L::kTileBytes);
-          for (int x = 0; x < L::kBoxes; ++x) {
-            tma_load_4d(smem + L::kQ + s * L::kTileBytes + x * L::kBoxBytes, &tq, q_full + s,
-                        x * 64, qt * kTile, it.h, it.b);
-            tma_load_4d(smem + L::kDO + s * L::kTileBytes + x * L::kBoxBytes, &tdo, q_full + s,
-                        x * 64, qt * kTile, it.h, it.b);
+      // column vectors of one q-tile: lane l holds queries l, l+32, l+64, l+96
+      auto fetch_vec = [&](int qt, float (&v0)[4], float (&v1)[4]) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int qg = qt * kTile + lane + 32 * k;
+          v0[k] = row_offset<EPI>(p, it.b, it.h, qg);
+          v1[k] = row_D<EPI>(p, it.b, it.h, qg);
+        }
+      };
+      float cur0[4], cur1[4], nx0[4], nx1[4];
+      fetch_vec(p.rowT_idx[it.e0], cur0, cur1);
+      for (int i0 = 0; ok && i0 < it.n; i0 += 32) {
+        const int il = i0 + lane;
+        int qt_l = 0, kd_l = 0, pi_l = 0;
+        if (il < it.n) {
+          qt_l = p.rowT_idx[it.e0 + il];
+          const int e = p.csc_map[it.e0 + il];
+          kd_l = p.kind[e];
+          if (kd_l == 2) pi_l = p.pidx[e];
+        }
+        const int jn = min(32, it.n - i0);
+        for (int u = 0; u < jn; ++u, ++qc) {
+          const int qt = __shfl_sync(0xFFFFFFFFu, qt_l, u);
+          const int kd = __shfl_sync(0xFFFFFFFFu, kd_l, u);
+          const int pi = __shfl_sync(0xFFFFFFFFu, pi_l, u);
+          const int i = i0 + u;
+          if (i + 1 < it.n) {  // next tile's column vectors, in flight during this tile's wait
+            const int qn = (u + 1 < jn) ? __shfl_sync(0xFFFFFFFFu, qt_l, u + 1)
+                                        : p.rowT_idx[it.e0 + i + 1];
+            fetch_vec(qn, nx0, nx1);
           }
+          const int s = qc % S;
+          if (lane == 0 && qc >= S) ok = mbar_wait(q_empty + s, ((qc / S) - 1) & 1, wctx);
+          ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          if (lane == 0) {
+            meta_kind[s] = kd;
+            mbar_arrive_expect_tx(q_full + s, 2 * L::kTileBytes + (kd == 2 ? 2048 : 0));
+            for (int x = 0; x < L::kBoxes; ++x) {
+              tma_load_4d(smem + L::kQ + s * L::kTileBytes + x * L::kBoxBytes, &tq, q_full + s,
+                          x * 64, qt * kTile, it.h, it.b);
+              tma_load_4d(smem + L::kDO + s * L::kTileBytes + x * L::kBoxBytes, &tdo, q_full + s,
+                          x * 64, qt * kTile, it.h, it.b);
+            }
+            if (kd == 2)
+              bulk_load(meta_bits + s * 512, p.bitsT + static_cast<int64_t>(pi) * 512, 2048,
+                        q_full + s);
+          }
+          float* vs = vec + s * 256;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            vs[lane + 32 * k] = cur0[k];
+            vs[128 + lane + 32 * k] = cur1[k];
+            cur0[k] = nx0[k];
+            cur1[k] = nx1[k];
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(q_full + s);
         }
-        float* vs = vec + s * 256;
-        for (int cc = lane; cc < 128; cc += 32) {
-          const int qg = qt * kTile + cc;
-          vs[cc] = row_offset<EPI>(p, it.b, it.h, qg);
-          vs[128 + cc] = row_D<EPI>(p, it.b, it.h, qg);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_full + s);
       }
     }
     if (lane == 0 && *abort_flag) {
@@ -372,8 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (pend_last) mma_commit(acc_full + pend_ab);
       };
       int qc = 0, ii = 0;
-      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
-        const WorkRef it = decode_col(p, w);
+      for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+        const WorkRef it = iter.cur;
         if (it.n == 0) continue;
         const int kb = ii % KVB, ab = ii % ACB;
         if (kDeferAcc && pend_qt >= 0) {  // previous item's last tile, before new K / V
@@ -438,8 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float2 c1 = make_float2(c1s, c1s);
     bool ok = true;
     int qc = 0, ii = 0;
-    for (int w = blockIdx.x; w < nitems; w += gridDim.x) {
-      const WorkRef it = decode_col(p, w);
+    for (WorkIter<true> iter(p, nitems); iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
       if (it.n == 0) {
         // No query attends to this k-tile: dK = dV = 0 on its rows.
         const int rows = min(kTile, p.Nk - it.t * kTile);
@@ -454,17 +518,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ab = ii % ACB;
       for (int i = 0; i < it.n; ++i, ++qc) {
         const int s = qc % S;
-        const int e = p.csc_map[it.e0 + i];
-        const int kd = p.kind[e];
-        uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        if (kd == 2)
-          mb = *reinterpret_cast<const uint2*>(p.bitsT + static_cast<int64_t>(p.pidx[e]) * 512 +
-                                               row * 4 + 2 * h);
+        // q_full of the stage also publishes the kind and bitmask the producer staged
         if (ok) ok = mbar_wait(q_full + s, (qc / S) & 1, wctx);
         if (ok) ok = mbar_wait(s_full + h, qc & 1, wctx);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) break;
         tc_fence_after();
+        uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+        if (meta_kind[s] == 2)
+          mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
         const float* vs = vec + s * 256 + 64 * h;
         uint32_t sr[2][32], dpr[2][32];
         tmem_ld32(t_lane + 64 * h, sr[0]);
@@ -562,7 +624,10 @@ struct DqLayout {
   static constexpr int kDO = kQ + kQBufs * kTileBytes;
   static constexpr int kK = kDO + kQBufs * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBar = kV + kStages * kTileBytes;
+  // per K/V stage: the tile's PARTIAL bitmask and its kind, staged by the producer
+  static constexpr int kMetaBits = kV + kStages * kTileBytes;
+  static constexpr int kMetaKind = kMetaBits + kStages * 2048;
+  static constexpr int kBar = kMetaKind + 16 * ((kStages * 4 + 15) / 16);
   // qd_full[QB] qd_empty[QB] kv_full[S] kv_empty[S] s_full[2] ds_full[2] acc_full[A] acc_empty[A]
   static constexpr int kNumBars = 2 * kQBufs + 2 * kStages + 4 + 2 * kAccBufs;
   static constexpr int kMisc = kBar + 8 * kNumBars;
@@ -592,6 +657,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* ds_full = s_full + 2;    // [2] per half
   uint64_t* acc_full = ds_full + 2;  // [ACB]
   uint64_t* acc_empty = acc_full + ACB;
+  uint32_t* meta_bits = reinterpret_cast<uint32_t*>(smem + L::kMetaBits);
+  int* meta_kind = reinterpret_cast<int*>(smem + L::kMetaKind);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   volatile int* drain_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
@@ -626,40 +693,68 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      int tk_ = 0, ii = 0;
-      bool ok = true;
-      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
-        const WorkRef it = decode_row(p, w);
-        if (it.n == 0) continue;
-        const int qb = ii % QB;
-        if (ii >= QB && !(ok = mbar_wait(qd_empty + qb, ((ii / QB) - 1) & 1, wctx))) break;
-        mbar_arrive_expect_tx(qd_full + qb, 2 * L::kTileBytes);
-        for (int x = 0; x < L::kBoxes; ++x) {
-          tma_load_4d(smem + L::kQ + qb * L::kTileBytes + x * L::kBoxBytes, &tq, qd_full + qb,
-                      x * 64, it.t * kTile, it.h, it.b);
-          tma_load_4d(smem + L::kDO + qb * L::kTileBytes + x * L::kBoxBytes, &tdo, qd_full + qb,
-                      x * 64, it.t * kTile, it.h, it.b);
-        }
-        ++ii;
-        for (int j = 0; j < it.n; ++j, ++tk_) {
-          const int s = tk_ % S;
-          if (tk_ >= S && !(ok = mbar_wait(kv_empty + s, ((tk_ / S) - 1) & 1, wctx))) break;
-          const int kt = p.col_idx[it.e0 + j];
-          mbar_arrive_expect_tx(kv_full + s, 2 * L::kTileBytes);
+    // Lane 0 waits and issues the copies; all 32 lanes fetch the list entries of the next
+    // 32 k-tiles in one round trip.
+    int tk_ = 0, ii = 0;
+    bool ok = true;
+    for (WorkIter<false> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
+      if (it.n == 0) continue;
+      const int qb = ii % QB;
+      if (lane == 0) {
+        if (ii >= QB) ok = mbar_wait(qd_empty + qb, ((ii / QB) - 1) & 1, wctx);
+        if (ok) {
+          mbar_arrive_expect_tx(qd_full + qb, 2 * L::kTileBytes);
           for (int x = 0; x < L::kBoxes; ++x) {
-            tma_load_4d(smem + L::kK + s * L::kTileBytes + x * L::kBoxBytes, &tk, kv_full + s,
-                        x * 64, kt * kTile, it.h, it.b);
-            tma_load_4d(smem + L::kV + s * L::kTileBytes + x * L::kBoxBytes, &tv, kv_full + s,
-                        x * 64, kt * kTile, it.h, it.b);
+            tma_load_4d(smem + L::kQ + qb * L::kTileBytes + x * L::kBoxBytes, &tq, qd_full + qb,
+                        x * 64, it.t * kTile, it.h, it.b);
+            tma_load_4d(smem + L::kDO + qb * L::kTileBytes + x * L::kBoxBytes, &tdo, qd_full + qb,
+                        x * 64, it.t * kTile, it.h, it.b);
           }
         }
       }
-      if (*abort_flag) {
-        const WaitCtx drain{p.status, p.wait_ns, drain_flag};
-        for (int u = max(0, ii - QB); u < ii; ++u) mbar_wait(qd_full + u % QB, (u / QB) & 1, drain);
-        for (int u = max(0, tk_ - S); u < tk_; ++u) mbar_wait(kv_full + u % S, (u / S) & 1, drain);
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      ++ii;
+      for (int j0 = 0; ok && j0 < it.n; j0 += 32) {
+        const int jj = j0 + lane;
+        int kt_l = 0, kd_l = 0, pi_l = 0;
+        if (jj < it.n) {
+          kt_l = p.col_idx[it.e0 + jj];
+          kd_l = p.kind[it.e0 + jj];
+        }
+        if (kd_l == 2) pi_l = p.pidx[it.e0 + jj];
+        const int jn = min(32, it.n - j0);
+        for (int u = 0; u < jn; ++u, ++tk_) {
+          const int kt = __shfl_sync(0xFFFFFFFFu, kt_l, u);
+          const int kd = __shfl_sync(0xFFFFFFFFu, kd_l, u);
+          const int pi = __shfl_sync(0xFFFFFFFFu, pi_l, u);
+          const int s = tk_ % S;
+          if (lane == 0) {
+            if (tk_ >= S) ok = mbar_wait(kv_empty + s, ((tk_ / S) - 1) & 1, wctx);
+            if (ok) {
+              meta_kind[s] = kd;
+              mbar_arrive_expect_tx(kv_full + s, 2 * L::kTileBytes + (kd == 2 ? 2048 : 0));
+              for (int x = 0; x < L::kBoxes; ++x) {
+                tma_load_4d(smem + L::kK + s * L::kTileBytes + x * L::kBoxBytes, &tk, kv_full + s,
+                            x * 64, kt * kTile, it.h, it.b);
+                tma_load_4d(smem + L::kV + s * L::kTileBytes + x * L::kBoxBytes, &tv, kv_full + s,
+                            x * 64, kt * kTile, it.h, it.b);
+              }
+              if (kd == 2)
+                bulk_load(meta_bits + s * 512, p.bits + static_cast<int64_t>(pi) * 512, 2048,
+                          kv_full + s);
+            }
+          }
+          ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+        }
       }
+    }
+    if (lane == 0 && *abort_flag) {
+      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      for (int u = max(0, ii - QB); u < ii; ++u) mbar_wait(qd_full + u % QB, (u / QB) & 1, drain);
+      for (int u = max(0, tk_ - S); u < tk_; ++u) mbar_wait(kv_full + u % S, (u / S) & 1, drain);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -704,8 +799,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (pend_last) mma_commit(acc_full + pend_ab);
       };
       int tk_ = 0, ii = 0;
-      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
-        const WorkRef it = decode_row(p, w);
+      for (WorkIter<false> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+        const WorkRef it = iter.cur;
         if (it.n == 0) continue;
         const int qb = ii % QB, ab = ii % ACB;
         if (kDeferAcc && pend_t >= 0) {
@@ -770,8 +865,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float2 c1 = make_float2(c1s, c1s);
     bool ok = true;
     int tk_ = 0, ii = 0;
-    for (int w = blockIdx.x; w < nitems; w += gridDim.x) {
-      const WorkRef it = decode_row(p, w);
+    WorkIter<false> iter(p, nitems);
+    float off_cur = 0.0f, D_cur = 0.0f;
+    if (iter.valid()) {
+      off_cur = row_offset<EPI>(p, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
+      D_cur = row_D<EPI>(p, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
+    }
+    for (; iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
+      // the next item's row values, in flight while this one is processed
+      float off_nxt = 0.0f, D_nxt = 0.0f;
+      if (iter.w + static_cast<int>(gridDim.x) < nitems && iter.nxt.n > 0) {
+        off_nxt = row_offset<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
+        D_nxt = row_D<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
+      }
+      const float off = off_cur, Drow = D_cur;
+      off_cur = off_nxt;
+      D_cur = D_nxt;
       if (it.n == 0) {
         const int rows = min(kTile, p.Nq - it.t * kTile);
         zero_rows<D>(p.dq + it.b * p.dq_sb + static_cast<int64_t>(it.t * kTile) * p.dq_sn +
@@ -781,20 +891,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       const int ab = ii % ACB;
       const int qg = it.t * kTile + row;
-      const float off = row_offset<EPI>(p, it.b, it.h, qg);
-      const float Drow = row_D<EPI>(p, it.b, it.h, qg);
       const float2 off2 = make_float2(off, off), D2 = make_float2(Drow, Drow);
       for (int j = 0; j < it.n; ++j, ++tk_) {
-        const int e = it.e0 + j;
-        const int kd = p.kind[e];
-        uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        if (kd == 2)
-          mb = *reinterpret_cast<const uint2*>(p.bits + static_cast<int64_t>(p.pidx[e]) * 512 +
-                                               row * 4 + 2 * h);
+        const int s = tk_ % S;
+        // kv_full of the stage also publishes the kind and bitmask the producer staged
+        if (ok) ok = mbar_wait(kv_full + s, (tk_ / S) & 1, wctx);
         if (ok) ok = mbar_wait(s_full + h, tk_ & 1, wctx);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) break;
         tc_fence_after();
+        uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+        if (meta_kind[s] == 2)
+          mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
         uint32_t sr[2][32], dpr[2][32];
         tmem_ld32(t_lane + 64 * h, sr[0]);
         tmem_ld32(t_lane + 128 + 64 * h, dpr[0]);
@@ -889,8 +997,8 @@ int launch_bwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.colT_ptr = plan->colT_ptr;
   p.rowT_idx = plan->rowT_idx;
   p.csc_map = plan->csc_map;
-  p.row_work = plan->row_work;
-  p.col_work = plan->col_work;
+  p.row_desc = plan->row_desc;
+  p.col_desc = plan->col_desc;
   p.B = plan->B;
   p.QT = plan->QT;
   p.KT = plan->KT;

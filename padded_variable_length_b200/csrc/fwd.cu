@@ -46,7 +46,7 @@ struct FwdParams {
   const uint8_t* kind;
   const int32_t* pidx;
   const uint32_t* bits;
-  const int32_t* row_work;
+  const int4* row_desc;
   int QT, Nq, H, nitems;
   float scale;
   const float* bias;
@@ -67,7 +67,10 @@ struct FwdLayout {
   static constexpr int kQ = 0;                  // two Q buffers
   static constexpr int kK = 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBar = kV + kStages * kTileBytes;
+  // per K/V stage: the tile's PARTIAL bitmask (2 KB) and its kind, staged by the producer
+  static constexpr int kMetaBits = kV + kStages * kTileBytes;
+  static constexpr int kMetaKind = kMetaBits + kStages * 2048;
+  static constexpr int kBar = kMetaKind + 16 * ((kStages * 4 + 15) / 16);
   // q_full[2] q_empty[2] o_full[2] o_empty[2] s_full[2] p_full[2] pv_done
   // k_full[S] v_full[S] kv_empty[S]
   static constexpr int kNumBars = 13 + 3 * kStages;
@@ -84,14 +87,32 @@ struct Item {
 
 __device__ __forceinline__ Item decode_item(const FwdParams& p, int w) {
   Item it;
-  const int r = p.row_work[w / p.H];
+  const int4 d = p.row_desc[w / p.H];
   it.h = w % p.H;
-  it.b = r / p.QT;
-  it.qt = r % p.QT;
-  it.e0 = p.row_ptr[r];
-  it.n = p.row_ptr[r + 1] - it.e0;
+  it.b = d.x / p.QT;
+  it.qt = d.x % p.QT;
+  it.e0 = d.y;
+  it.n = d.z;
   return it;
 }
+
+// Walks this CTA's work items (stride = grid size) with the next item's decode issued one
+// item ahead, so that its global loads overlap the current item.
+struct ItemIter {
+  const FwdParams& p;
+  int w;
+  Item cur, nxt;
+  __device__ explicit ItemIter(const FwdParams& pp) : p(pp), w(blockIdx.x) {
+    if (w < p.nitems) cur = decode_item(p, w);
+    if (w + static_cast<int>(gridDim.x) < p.nitems) nxt = decode_item(p, w + gridDim.x);
+  }
+  __device__ bool valid() const { return w < p.nitems; }
+  __device__ void advance() {
+    w += gridDim.x;
+    cur = nxt;
+    if (w + static_cast<int>(gridDim.x) < p.nitems) nxt = decode_item(p, w + gridDim.x);
+  }
+};
 
 template <int D, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -115,6 +136,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_full = bars + 13;   // [S]
   uint64_t* v_full = bars + 13 + S;
   uint64_t* kv_empty = bars + 13 + 2 * S;
+  uint32_t* meta_bits = reinterpret_cast<uint32_t*>(smem + L::kMetaBits);
+  int* meta_kind = reinterpret_cast<int*>(smem + L::kMetaKind);
   float* red_max = reinterpret_cast<float*>(smem + L::kRed);
   float* red_l = reinterpret_cast<float*>(smem + L::kRedL);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -129,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(o_full + i, 1);
       mbar_init(o_empty + i, 8);
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, 8);
+      mbar_init(p_full + i, EPI == 0 ? 4 : 8);  // sigmoid: one warpgroup per tile
     }
     mbar_init(pv_done, 1);
     for (int i = 0; i < S; ++i) {
@@ -149,44 +172,74 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
+    // Lane 0 waits and issues the copies; all 32 lanes fetch the list entries of the next
+    // 32 tiles in one round trip, so index loads never sit between two copies.
     if (lane == 0) {
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
-      int t = 0, i = 0;
-      bool ok = true;
-      for (int w = blockIdx.x; ok && w < p.nitems; w += gridDim.x) {
-        const Item it = decode_item(p, w);
-        if (it.n == 0) continue;
-        const int qb = i & 1;
-        if (i >= 2 && !(ok = mbar_wait(q_empty + qb, ((i >> 1) - 1) & 1, wctx))) break;
-        mbar_arrive_expect_tx(q_full + qb, L::kTileBytes);
-        for (int x = 0; x < L::kBoxes; ++x)
-          tma_load_4d(smem + L::kQ + qb * L::kTileBytes + x * L::kBoxBytes, &tq, q_full + qb,
-                      x * 64, it.qt * kTile, it.h, it.b);
-        ++i;
-        for (int j = 0; j < it.n; ++j, ++t) {
-          const int s = t % S;
-          if (t >= S && !(ok = mbar_wait(kv_empty + s, ((t / S) - 1) & 1, wctx))) break;
-          const int kt = p.col_idx[it.e0 + j];
-          mbar_arrive_expect_tx(k_full + s, L::kTileBytes);
+    }
+    int t = 0, i = 0;
+    bool ok = true;
+    for (ItemIter iter(p); ok && iter.valid(); iter.advance()) {
+      const Item it = iter.cur;
+      if (it.n == 0) continue;
+      const int qb = i & 1;
+      if (lane == 0) {
+        if (i >= 2) ok = mbar_wait(q_empty + qb, ((i >> 1) - 1) & 1, wctx);
+        if (ok) {
+          mbar_arrive_expect_tx(q_full + qb, L::kTileBytes);
           for (int x = 0; x < L::kBoxes; ++x)
-            tma_load_4d(smem + L::kK + s * L::kTileBytes + x * L::kBoxBytes, &tk, k_full + s,
-                        x * 64, kt * kTile, it.h, it.b);
-          mbar_arrive_expect_tx(v_full + s, L::kTileBytes);
-          for (int x = 0; x < L::kBoxes; ++x)
-            tma_load_4d(smem + L::kV + s * L::kTileBytes + x * L::kBoxBytes, &tv, v_full + s,
-                        x * 64, kt * kTile, it.h, it.b);
+            tma_load_4d(smem + L::kQ + qb * L::kTileBytes + x * L::kBoxBytes, &tq, q_full + qb,
+                        x * 64, it.qt * kTile, it.h, it.b);
         }
       }
-      if (*abort_flag) {
-        // Let the copies still in flight land before the CTA's shared memory goes away.
-        const WaitCtx drain{p.status, p.wait_ns, drain_flag};
-        for (int u = max(0, i - 2); u < i; ++u) mbar_wait(q_full + (u & 1), (u >> 1) & 1, drain);
-        for (int u = max(0, t - S); u < t; ++u) {
-          mbar_wait(k_full + u % S, (u / S) & 1, drain);
-          mbar_wait(v_full + u % S, (u / S) & 1, drain);
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      ++i;
+      for (int j0 = 0; ok && j0 < it.n; j0 += 32) {
+        const int jj = j0 + lane;
+        int kt_l = 0, kd_l = 0, pi_l = 0;
+        if (jj < it.n) {
+          kt_l = p.col_idx[it.e0 + jj];
+          kd_l = p.kind[it.e0 + jj];
         }
+        if (kd_l == 2) pi_l = p.pidx[it.e0 + jj];
+        const int jn = min(32, it.n - j0);
+        for (int u = 0; u < jn; ++u, ++t) {
+          const int kt = __shfl_sync(0xFFFFFFFFu, kt_l, u);
+          const int kd = __shfl_sync(0xFFFFFFFFu, kd_l, u);
+          const int pi = __shfl_sync(0xFFFFFFFFu, pi_l, u);
+          const int s = t % S;
+          if (lane == 0) {
+            if (t >= S) ok = mbar_wait(kv_empty + s, ((t / S) - 1) & 1, wctx);
+            if (ok) {
+              meta_kind[s] = kd;
+              mbar_arrive_expect_tx(k_full + s, L::kTileBytes + (kd == 2 ? 2048 : 0));
+              for (int x = 0; x < L::kBoxes; ++x)
+                tma_load_4d(smem + L::kK + s * L::kTileBytes + x * L::kBoxBytes, &tk, k_full + s,
+                            x * 64, kt * kTile, it.h, it.b);
+              if (kd == 2)
+                bulk_load(meta_bits + s * 512, p.bits + static_cast<int64_t>(pi) * 512, 2048,
+                          k_full + s);
+              mbar_arrive_expect_tx(v_full + s, L::kTileBytes);
+              for (int x = 0; x < L::kBoxes; ++x)
+                tma_load_4d(smem + L::kV + s * L::kTileBytes + x * L::kBoxBytes, &tv, v_full + s,
+                            x * 64, kt * kTile, it.h, it.b);
+            }
+          }
+          ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+        }
+      }
+    }
+    if (lane == 0 && *abort_flag) {
+      // Let the copies still in flight land before the CTA's shared memory goes away.
+      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      for (int u = max(0, i - 2); u < i; ++u) mbar_wait(q_full + (u & 1), (u >> 1) & 1, drain);
+      for (int u = max(0, t - S); u < t; ++u) {
+        mbar_wait(k_full + u % S, (u / S) & 1, drain);
+        mbar_wait(v_full + u % S, (u / S) & 1, drain);
       }
     }
   } else if (warp == 1) {
@@ -209,7 +262,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t o_tmem = tmem + 256 + ob * D;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t a_tmem = tmem + pb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+          // sigmoid: P of keys 16kk.. at column 8kk (one warpgroup wrote the whole tile);
+          // softmax: warpgroup g wrote keys [64g, 64g+64) at columns [64g, 64g+32)
+          const uint32_t a_tmem =
+              tmem + pb * 128 + (EPI == 0 ? kk * 8 : (kk >> 2) * 64 + (kk & 3) * 8);
           mma_ts(o_tmem, a_tmem, smem_desc_sw128(v_base + kk * 2048, L::kBoxBytes, 1024),
                  idesc_pv, (pv_first && kk == 0) ? 0u : 1u);
         }
@@ -219,8 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       int t = 0, i = 0;
-      for (int w = blockIdx.x; ok && w < p.nitems; w += gridDim.x) {
-        const Item it = decode_item(p, w);
+      for (ItemIter iter(p); ok && iter.valid(); iter.advance()) {
+        const Item it = iter.cur;
         if (it.n == 0) continue;
         const int qb = i & 1;
         if (!(ok = mbar_wait(q_full + qb, (i >> 1) & 1, wctx))) break;
@@ -250,59 +306,177 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok && pv_t >= 0) issue_pv();
     }
-  } else if (warp >= kEpiWarp0) {
-    // ---------------------------------------------------------------- epilogue
-    const int g = (warp - kEpiWarp0) >> 2;  // warpgroup: S columns [64g, 64g+64)
+  } else if (EPI == 0 && warp >= kEpiWarp0) {
+    // ---------------------------------------------------------------- sigmoid epilogue
+    // Ping-pong: warpgroup g takes the tiles with t % 2 == g (S buffer g), all 128 columns,
+    // in four chunks of 32 whose TMEM loads overlap the previous chunk's math; the two
+    // warpgroups work on different tiles, so one's load / store latency hides under the
+    // other's MUFU work.  P of keys [32c, 32c+32) goes to columns [16c, 16c+16).
+    const int g = (warp - kEpiWarp0) >> 2;
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t s_base = t_lane + g * 128;
+    constexpr int kOc = D / 2;
+    const float2 c1 = make_float2(0.5f * p.scale, 0.5f * p.scale);
+    const float2 half2 = make_float2(0.5f, 0.5f);
+    bool ok = true;
+    int t = 0, i = 0;
+    auto row_bias = [&](const Item& x) {
+      const int r = x.qt * kTile + row;
+      return (p.bias != nullptr && x.n > 0 && r < p.Nq) ? p.bias[x.b * p.bias_sb + r] : 0.0f;
+    };
+    ItemIter iter(p);
+    float bias_cur = iter.valid() ? row_bias(iter.cur) : 0.0f;
+    for (; ok && iter.valid(); iter.advance()) {
+      const Item it = iter.cur;
+      // the next item's bias, in flight while this one is processed
+      const float bias_nxt =
+          iter.w + static_cast<int>(gridDim.x) < p.nitems ? row_bias(iter.nxt) : 0.0f;
+      const float bias_r = bias_cur;
+      bias_cur = bias_nxt;
+      if (it.n == 0) {
+        // No tile in this row: the whole q-tile is padding or sees no key.  O = 0.
+        const int rows = min(kTile, p.Nq - it.qt * kTile);
+        constexpr int kChunks = D / 8;
+        const int tid = threadIdx.x - kEpiWarp0 * 32;
+        for (int c = tid; c < rows * kChunks; c += 256) {
+          const int rr = c / kChunks, ch = c % kChunks;
+          *reinterpret_cast<uint4*>(p.o + it.b * p.o_sb +
+                                    static_cast<int64_t>(it.qt * kTile + rr) * p.o_sn +
+                                    it.h * p.o_sh + ch * 8) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        continue;
+      }
+      const int ob = i & 1;
+      const float2 c0 = make_float2(0.5f * bias_r, 0.5f * bias_r);
+      const int t_end = t + it.n;
+      for (int tt = t + ((t & 1) != g ? 1 : 0); tt < t_end; tt += 2) {
+        const int s = tt % S;
+        // k_full of the tile's stage also publishes the kind and bitmask the producer staged
+        if (ok) ok = mbar_wait(k_full + s, (tt / S) & 1, wctx);
+        if (ok) ok = mbar_wait(s_full + g, (tt >> 1) & 1, wctx);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const bool masked = meta_kind[s] == 2;
+        uint4 mb = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+        if (masked) mb = *reinterpret_cast<const uint4*>(meta_bits + s * 512 + row * 4);
+        uint32_t buf[2][32];
+        tmem_ld32(s_base, buf[0]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c < 3) tmem_ld32(s_base + 32 * (c + 1), buf[(c + 1) & 1]);
+          const uint32_t mw = c == 0 ? mb.x : (c == 1 ? mb.y : (c == 2 ? mb.z : mb.w));
+          uint32_t pk[16];
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            const float2 x = fma2(make_float2(__uint_as_float(buf[c & 1][cc]),
+                                              __uint_as_float(buf[c & 1][cc + 1])),
+                                  c1, c0);
+            float2 th = make_float2(tanh_approx(x.x), tanh_approx(x.y));
+            if (masked) {
+              th.x = ((mw >> cc) & 1u) ? th.x : -1.0f;
+              th.y = ((mw >> (cc + 1)) & 1u) ? th.y : -1.0f;
+            }
+            const float2 pw = fma2(th, half2, half2);
+            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
+          }
+          tmem_st16(s_base + 16 * c, pk);
+          if (c < 3) tmem_wait_ld();
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + g);
+      }
+      if (!ok) break;
+      // ---- output of this item: this warpgroup's half of the O columns
+      ok = mbar_wait(o_full + ob, (i >> 1) & 1, wctx);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t pk[kOc / 2];
+#pragma unroll
+      for (int c0o = 0; c0o < kOc; c0o += 32) {
+        uint32_t orr[32];
+        tmem_ld32(t_lane + 256 + ob * D + g * kOc + c0o, orr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pk[c0o / 2 + c] = pack_bf16x2(__uint_as_float(orr[2 * c]), __uint_as_float(orr[2 * c + 1]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_empty + ob);
+      const int rg = it.qt * kTile + row;
+      if (rg < p.Nq) {
+        uint4* d4 = reinterpret_cast<uint4*>(p.o + it.b * p.o_sb + static_cast<int64_t>(rg) * p.o_sn +
+                                             it.h * p.o_sh + g * kOc);
+#pragma unroll
+        for (int c = 0; c < kOc / 8; ++c)
+          d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      t = t_end;
+      ++i;
+    }
+  } else if (EPI != 0 && warp >= kEpiWarp0) {
+    // ---------------------------------------------------------------- softmax epilogue
+    // Column split: warpgroup g owns S columns [64g, 64g+64) of every tile and O columns
+    // [g d/2, (g+1) d/2); the row maximum is exchanged through shared memory.
+    const int g = (warp - kEpiWarp0) >> 2;
     const int wq = warp & 3;                // TMEM lanes [32 wq, 32 wq + 32)
     const int row = wq * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     constexpr int kOc = D / 2;  // O columns of this warpgroup
     // `ok` stays warp-uniform (tcgen05.ld/st are warp-collective).  After an abort the
     // loops keep running without touching TMEM so that every epilogue thread executes the
-    // same sequence of named barriers (softmax modes) and nobody waits forever.
+    // same sequence of named barriers and nobody waits forever.
     bool ok = true;
     int t = 0, i = 0;
-    for (int w = blockIdx.x; w < p.nitems; w += gridDim.x) {
-      const Item it = decode_item(p, w);
+    auto row_bias = [&](const Item& x) {
+      const int r = x.qt * kTile + row;
+      return (p.bias != nullptr && x.n > 0 && r < p.Nq) ? p.bias[x.b * p.bias_sb + r] : 0.0f;
+    };
+    ItemIter iter(p);
+    float bias_cur = iter.valid() ? row_bias(iter.cur) : 0.0f;
+    for (; iter.valid(); iter.advance()) {
+      const Item it = iter.cur;
+      const float bias_nxt =
+          iter.w + static_cast<int>(gridDim.x) < p.nitems ? row_bias(iter.nxt) : 0.0f;
+      const float bias_r = bias_cur;
+      bias_cur = bias_nxt;
       if (it.n == 0) {
-        // No tile in this row: the whole q-tile is padding or sees no key.  O = 0.
         const int rows = min(kTile, p.Nq - it.qt * kTile);
-        constexpr int kChunks = D / 8;  // 16-byte chunks per row
+        constexpr int kChunks = D / 8;
         const int tid = threadIdx.x - kEpiWarp0 * 32;
         for (int c = tid; c < rows * kChunks; c += 256) {
           const int rr = c / kChunks, ch = c % kChunks;
-          __nv_bfloat16* dst = p.o + it.b * p.o_sb +
-                               static_cast<int64_t>(it.qt * kTile + rr) * p.o_sn + it.h * p.o_sh +
-                               ch * 8;
-          *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(p.o + it.b * p.o_sb +
+                                    static_cast<int64_t>(it.qt * kTile + rr) * p.o_sn +
+                                    it.h * p.o_sh + ch * 8) = make_uint4(0u, 0u, 0u, 0u);
         }
-        if (EPI != 0)
-          for (int c = tid; c < rows; c += 256)
-            p.lse[(static_cast<int64_t>(it.b) * p.H + it.h) * p.Nq + it.qt * kTile + c] =
-                EPI == 1 ? -INFINITY : 0.0f;
+        for (int c = tid; c < rows; c += 256)
+          p.lse[(static_cast<int64_t>(it.b) * p.H + it.h) * p.Nq + it.qt * kTile + c] =
+              EPI == 1 ? -INFINITY : 0.0f;
         continue;
       }
       const int ob = i & 1;
       const int rg = it.qt * kTile + row;
-      const float bias_r =
-          (p.bias != nullptr && rg < p.Nq) ? p.bias[it.b * p.bias_sb + rg] : 0.0f;
-      // sigmoid: sigma(x) = 0.5 + 0.5 tanh(x/2), x = scale s + bias -> (c1, c0) = halves;
-      // softmax: t = (scale s + bias) log2 e
-      const float c1 = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
-      const float c0 = EPI == 0 ? 0.5f * bias_r : bias_r * kLog2e;
-      float m_run = EPI == 2 ? 0.0f : kNegBig;  // base-2 running max (softmax modes)
+      const float c1 = p.scale * kLog2e;  // t = (scale s + bias) log2 e
+      const float c0 = bias_r * kLog2e;
+      float m_run = EPI == 2 ? 0.0f : kNegBig;  // base-2 running max
       float l_run = (EPI == 2 && g == 0) ? 1.0f : 0.0f;
       for (int j = 0; j < it.n; ++j, ++t) {
-        const int sb = t & 1;
+        const int sb = t & 1, s = t % S;
+        if (ok) ok = mbar_wait(k_full + s, (t / S) & 1, wctx);
         if (ok) ok = mbar_wait(s_full + sb, (t >> 1) & 1, wctx);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (ok) tc_fence_after();
-        const int e = it.e0 + j;
-        const int kd = p.kind[e];
         uint32_t mw0 = 0xFFFFFFFFu, mw1 = 0xFFFFFFFFu;
-        if (kd == 2) {
-          const uint2 mb = *reinterpret_cast<const uint2*>(
-              p.bits + static_cast<int64_t>(p.pidx[e]) * 512 + row * 4 + g * 2);
+        if (ok && meta_kind[s] == 2) {
+          const uint2 mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + g * 2);
           mw0 = mb.x;
           mw1 = mb.y;
         }
@@ -317,62 +491,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 64; ++c) sr[c] = 0u;
         }
         float pv[64];
-        if (EPI == 0) {
-          if (kd == 2) {
+        float tmax = kNegBig;
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-              const float sg = sigmoid_tanh(__uint_as_float(sr[c]), c1, c0);
-              const uint32_t bit = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
-              pv[c] = bit ? sg : 0.0f;
-            }
-          } else {
+        for (int c = 0; c < 64; ++c) {
+          const float tt = fmaf(__uint_as_float(sr[c]), c1, c0);
+          const uint32_t bit = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
+          pv[c] = bit ? tt : kNegBig;
+          tmax = fmaxf(tmax, pv[c]);
+        }
+        red_max[(sb * 2 + g) * 128 + row] = tmax;
+        named_barrier_sync(1, 256);
+        tmax = fmaxf(tmax, red_max[(sb * 2 + (g ^ 1)) * 128 + row]);
+        // Lazy rescaling: keep the running max unless the tile's max exceeds it by more
+        // than 8 (base 2), so that exp2(t - m) stays <= 256; the result is exact either
+        // way because numerator and denominator share m.
+        const bool need = tmax > m_run + 8.0f;
+        const float m_new = need ? tmax : m_run;
+        const float alpha = ex2_approx(m_run - m_new);
+        if (ok && __any_sync(0xFFFFFFFFu, need) && j > 0) {
+          // O must not be read while PV of the previous tile may still accumulate into it.
+          ok = mbar_wait(pv_done, (t - 1) & 1, wctx);
+          ok = __all_sync(0xFFFFFFFFu, ok);
+          if (ok) {
+            tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < 64; ++c) pv[c] = sigmoid_tanh(__uint_as_float(sr[c]), c1, c0);
-          }
-        } else {
-          float tmax = kNegBig;
+            for (int c0o = 0; c0o < kOc; c0o += 32) {
+              uint32_t orr[32];
+              tmem_ld32(t_lane + 256 + ob * D + g * kOc + c0o, orr);
+              tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float tt = fmaf(__uint_as_float(sr[c]), c1, c0);
-            const uint32_t bit = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
-            pv[c] = bit ? tt : kNegBig;
-            tmax = fmaxf(tmax, pv[c]);
-          }
-          red_max[(sb * 2 + g) * 128 + row] = tmax;
-          named_barrier_sync(1, 256);
-          tmax = fmaxf(tmax, red_max[(sb * 2 + (g ^ 1)) * 128 + row]);
-          // Lazy rescaling: keep the running max unless the tile's max exceeds it by more
-          // than 8 (base 2), so that exp2(t - m) stays <= 256; the result is exact either
-          // way because numerator and denominator share m.
-          const bool need = tmax > m_run + 8.0f;
-          const float m_new = need ? tmax : m_run;
-          const float alpha = ex2_approx(m_run - m_new);
-          if (ok && __any_sync(0xFFFFFFFFu, need) && j > 0) {
-            // O must not be read while PV of the previous tile may still accumulate into it.
-            ok = mbar_wait(pv_done, (t - 1) & 1, wctx);
-            ok = __all_sync(0xFFFFFFFFu, ok);
-            if (ok) {
-              tc_fence_after();
-#pragma unroll
-              for (int c0o = 0; c0o < kOc; c0o += 32) {
-                uint32_t orr[32];
-                tmem_ld32(t_lane + 256 + ob * D + g * kOc + c0o, orr);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; ++c)
-                  orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-                tmem_st32(t_lane + 256 + ob * D + g * kOc + c0o, orr);
-              }
+              for (int c = 0; c < 32; ++c)
+                orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+              tmem_st32(t_lane + 256 + ob * D + g * kOc + c0o, orr);
             }
           }
-          l_run *= alpha;
-          m_run = m_new;
+        }
+        l_run *= alpha;
+        m_run = m_new;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float e2 = pv[c] > 0.5f * kNegBig ? ex2_approx(pv[c] - m_run) : 0.0f;
-            pv[c] = e2;
-            l_run += e2;
-          }
+        for (int c = 0; c < 64; ++c) {
+          const float e2 = pv[c] > 0.5f * kNegBig ? ex2_approx(pv[c] - m_run) : 0.0f;
+          pv[c] = e2;
+          l_run += e2;
         }
         if (ok) {
           uint32_t pk[32];
@@ -385,20 +545,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive(p_full + sb);
         }
       }
-      // ---- output of this item: O (and LSE) from TMEM buffer ob
+      // ---- output of this item: O and LSE from TMEM buffer ob
       if (ok) ok = mbar_wait(o_full + ob, (i >> 1) & 1, wctx);
       ok = __all_sync(0xFFFFFFFFu, ok);
-      float inv_l = 1.0f;
-      if (EPI != 0) {
-        red_l[g * 128 + row] = l_run;
-        named_barrier_sync(1, 256);
-        const float l_tot = l_run + red_l[(g ^ 1) * 128 + row];
-        named_barrier_sync(1, 256);  // red_l is rewritten by the next item
-        inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
-        if (ok && g == 0 && rg < p.Nq) {
-          const float lse = l_tot > 0.0f ? (m_run + __log2f(l_tot)) * kLn2 : -INFINITY;
-          p.lse[(static_cast<int64_t>(it.b) * p.H + it.h) * p.Nq + rg] = lse;
-        }
+      red_l[g * 128 + row] = l_run;
+      named_barrier_sync(1, 256);
+      const float l_tot = l_run + red_l[(g ^ 1) * 128 + row];
+      named_barrier_sync(1, 256);  // red_l is rewritten by the next item
+      const float inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
+      if (ok && g == 0 && rg < p.Nq) {
+        const float lse = l_tot > 0.0f ? (m_run + __log2f(l_tot)) * kLn2 : -INFINITY;
+        p.lse[(static_cast<int64_t>(it.b) * p.H + it.h) * p.Nq + rg] = lse;
       }
       if (ok) {
         tc_fence_after();
@@ -463,7 +620,7 @@ int launch_fwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.kind = plan->kind;
   p.pidx = plan->pidx;
   p.bits = plan->bits;
-  p.row_work = plan->row_work;
+  p.row_desc = plan->row_desc;
   p.QT = plan->QT;
   p.Nq = plan->Nq;
   p.H = H;

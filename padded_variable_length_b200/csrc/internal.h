@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/sigattn.h"
+#include "sigattn.h"
 
 // Device buffers of a tile plan.  Layouts are those of sigattn_plan_export; in addition
 // the plan keeps the transposed PARTIAL bitmasks (for kernels that own a key per thread)
@@ -28,6 +28,10 @@ struct sigattn_plan {
   uint32_t* bitsT;  // [partial * 512] the same bitmasks transposed: bit (q % 32) of word (k*4 + q/32)
   int32_t* row_work;
   int32_t* col_work;
+  // the work lists again, one 16-byte record per entry: {row or column, first list entry,
+  // number of entries, 0}, so that a kernel decodes a work item with one independent load
+  int4* row_desc;
+  int4* col_desc;
 };
 
 namespace sigattn {

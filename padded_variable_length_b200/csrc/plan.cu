@@ -346,6 +346,16 @@ __global__ void __launch_bounds__(128) k_bits_from_lengths(const int32_t* __rest
   reinterpret_cast<uint4*>(bits + static_cast<int64_t>(blockIdx.x) * 512)[q] = w;
 }
 
+// desc[k] = {work[k], ptr[work[k]], ptr[work[k] + 1] - ptr[work[k]], 0}
+__global__ void k_work_desc(const int32_t* __restrict__ work, const int32_t* __restrict__ ptr, int n,
+                            int4* __restrict__ desc) {
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) {
+    const int r = work[k];
+    const int a = ptr[r];
+    desc[k] = make_int4(r, a, ptr[r + 1] - a, 0);
+  }
+}
+
 // One CTA of 128 threads per PARTIAL block: thread k gathers column k of the bitmask.
 __global__ void __launch_bounds__(128) k_transpose_bits(const uint32_t* __restrict__ bits,
                                                         uint32_t* __restrict__ bitsT) {
@@ -403,8 +413,9 @@ struct Scratch {
 };
 
 void plan_free_buffers(sigattn_plan* p) {
-  void* ps[] = {p->row_ptr,  p->col_idx, p->kind, p->pidx,     p->colT_ptr, p->rowT_idx,
-                p->csc_map,  p->bits,    p->bitsT, p->row_work, p->col_work};
+  void* ps[] = {p->row_ptr, p->col_idx, p->kind,     p->pidx,     p->colT_ptr, p->rowT_idx,
+                p->csc_map, p->bits,    p->bitsT,    p->row_work, p->col_work, p->row_desc,
+                p->col_desc};
   for (void* q : ps)
     if (q) cudaFree(q);
 }
@@ -437,6 +448,8 @@ int finish_plan(sigattn_plan* plan, Scratch& sc, cudaStream_t stream, BitsFn bit
   SIGATTN_TRY(dev_alloc(&plan->colT_ptr, cols + 1));
   SIGATTN_TRY(dev_alloc(&plan->row_work, rows));
   SIGATTN_TRY(dev_alloc(&plan->col_work, cols));
+  SIGATTN_TRY(dev_alloc(&plan->row_desc, rows));
+  SIGATTN_TRY(dev_alloc(&plan->col_desc, cols));
   SIGATTN_TRY(scratch_alloc(&sc.row_cnt, rows, stream));
   SIGATTN_TRY(scratch_alloc(&sc.row_pcnt, rows, stream));
   SIGATTN_TRY(scratch_alloc(&sc.row_poff, rows + 1, stream));
@@ -451,6 +464,10 @@ int finish_plan(sigattn_plan* plan, Scratch& sc, cudaStream_t stream, BitsFn bit
   k_scan<<<1, 1024, 0, stream>>>(sc.col_cnt, cols, plan->colT_ptr, nullptr);
   k_sort_longest_first<<<1, 32, 0, stream>>>(sc.row_cnt, rows, plan->row_work, sc.totals + 2);
   k_sort_longest_first<<<1, 32, 0, stream>>>(sc.col_cnt, cols, plan->col_work, sc.totals + 3);
+  k_work_desc<<<grid_for(rows, 256), 256, 0, stream>>>(plan->row_work, plan->row_ptr, rows,
+                                                        plan->row_desc);
+  k_work_desc<<<grid_for(cols, 256), 256, 0, stream>>>(plan->col_work, plan->colT_ptr, cols,
+                                                        plan->col_desc);
   SIGATTN_TRY_CUDA(cudaGetLastError());
   int64_t totals[8] = {0};
   SIGATTN_TRY_CUDA(cudaMemcpyAsync(totals, sc.totals, 4 * sizeof(int64_t), cudaMemcpyDeviceToHost,
