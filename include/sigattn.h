@@ -262,6 +262,10 @@ SIGATTN_API int sigattn_selftest_wait_timeout(uint64_t ns, sigattn_stream stream
 /* Static description of an error code. */
 SIGATTN_API const char* sigattn_error_string(int code);
 
+/* Name of the CUDA error behind the most recent SIGATTN_ERR_CUDA / NOMEM returned by any
+ * call of this library (process-wide), e.g. "cudaErrorInvalidValue"; "no CUDA error" if none. */
+SIGATTN_API const char* sigattn_last_cuda_error(void);
+
 /* Library version, e.g. 100 for 0.1.0. */
 SIGATTN_API int sigattn_version(void);
 

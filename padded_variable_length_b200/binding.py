@@ -26,8 +26,10 @@ ERR = {-1: "INVALID", -2: "UNSUPPORTED", -3: "ALIGNMENT", -4: "SHAPE", -5: "CUDA
 class SigattnError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
-        super().__init__(f"{what}: sigattn error {code} ({ERR.get(code, '?')}): "
-                         f"{_lib.sigattn_error_string(code).decode()}")
+        detail = _lib.sigattn_error_string(code).decode()
+        if code in (-5, -8):
+            detail += f" [{_lib.sigattn_last_cuda_error().decode()}]"
+        super().__init__(f"{what}: sigattn error {code} ({ERR.get(code, '?')}): {detail}")
 
 
 if not os.path.exists(LIB_PATH):
@@ -79,6 +81,7 @@ _sig("sigattn_set_wait_limit_ns", ctypes.c_int, _u64)
 _sig("sigattn_selftest_wait_timeout", ctypes.c_int, _u64, _p)
 _sig("sigattn_error_string", ctypes.c_char_p, ctypes.c_int)
 _sig("sigattn_version", ctypes.c_int)
+_sig("sigattn_last_cuda_error", ctypes.c_char_p)
 
 lib = _lib
 

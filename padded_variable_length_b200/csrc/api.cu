@@ -28,8 +28,11 @@ int launch_bwd_impl(const sigattn_plan* plan, int epilogue, int H, int d, float 
                     const TensorDesc& dq, const TensorDesc& dk, const TensorDesc& dv,
                     int parts, int* status, unsigned long long wait_ns, cudaStream_t stream);
 
+std::atomic<int> g_last_cuda_error{0};
+
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return SIGATTN_OK;
+  g_last_cuda_error.store(static_cast<int>(e));
   cudaGetLastError();
   return e == cudaErrorMemoryAllocation ? SIGATTN_ERR_NOMEM : SIGATTN_ERR_CUDA;
 }
@@ -293,6 +296,11 @@ extern "C" const char* sigattn_error_string(int code) {
     case SIGATTN_ERR_NOMEM: return "device allocation failed";
     default: return "unknown error code";
   }
+}
+
+extern "C" const char* sigattn_last_cuda_error(void) {
+  const int e = g_last_cuda_error.load();
+  return e == 0 ? "no CUDA error" : cudaGetErrorName(static_cast<cudaError_t>(e));
 }
 
 extern "C" int sigattn_version(void) { return 100; }
