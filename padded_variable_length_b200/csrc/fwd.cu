@@ -609,23 +609,23 @@ int num_sms() {
 }
 
 // ------------------------------------------------------------------------------------
-// Sigmoid forward with decoupled stages.
+// Sigmoid forward: one tensor-pipe step per tile.
 //
-// The weights of sigmoid attention need no row statistics, so nothing but tensor memory
-// ties one key tile to the next.  This kernel keeps the epilogue (the MUFU-bound part)
-// fed without gaps:
-//   * P has TMEM columns of its own, so the S buffer a warpgroup has read can take the
-//     S of the tile after next while the warpgroup is still computing: the MMA issuer
-//     runs S two tiles ahead of PV (S_t is issued before O += P_{t-2} V_{t-2});
-//   * K and V have separate rings released by separate commits (K after its S MMA, V
-//     after its PV MMA), filled by two producer warps, so K runs ahead of V;
-//   * a warpgroup writes out the O of an item only after its first tile of the next
-//     item, when the last PV of that item has long completed.
-// Warps: 0 Q/K producer, 1 TMEM allocator + MMA issuer, 2 V producer (with the tile's
-// kind and PARTIAL bitmask, published by v_full), 4-11 two epilogue warpgroups; warpgroup
-// g takes the tiles t with t % 2 == g of the CTA's tile stream.
-// TMEM columns: S0 [0,128), S1 [128,256), P0 [256,320), P1 [320,384), then O: two
-// buffers of 64 columns for d = 64, one of 128 for d = 128.
+// The weights of sigmoid attention need no row statistics, so nothing but buffers ties
+// one key tile to the next, and the kernel is organised to need as few hand-offs per tile
+// as possible.  Step u of the MMA issuer, started when the epilogue has finished tile
+// u - 2, issues S_u = Q K_u^T (commit s_ready: S_u is ready and K_u consumed) and then
+// O += P_{u-2} V_{u-2} (commit step: V_{u-2} consumed).  S and P of a tile share a
+// buffer (P overwrites the columns of S its own warpgroup has read), and three such
+// buffers let the epilogue work on tile u - 1 while step u runs; the epilogue loads the
+// first half of its columns of tile u + 1 while it computes the second half of tile u.
+// Warps: 0 Q/K producer, 1 TMEM allocator + MMA issuer, 2 V producer, 3 kind / bitmask
+// producer, 4-11 two epilogue warpgroups: thread = query row = TMEM lane, warpgroup g on
+// keys [64g, 64g+64) of every tile.  The O of an item is written out after the first
+// tile of the next item, when the last PV of the item has long completed.
+// TMEM columns: S/P buffers [0,128), [128,256), [256,384); O in [384,512) (two buffers
+// of 64 columns for d = 64, one of 128 for d = 128).  P of keys 16kk.. (the A operand of
+// the kk-th K-step of the PV MMA) sits at column 64 (kk / 4) + 8 (kk % 4) of its buffer.
 template <int D>
 struct SigLayout {
   static constexpr int kBoxes = D / 64;
@@ -633,20 +633,23 @@ struct SigLayout {
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
   static constexpr int kKStages = D == 64 ? 4 : 2;
   static constexpr int kVStages = D == 64 ? 4 : 2;
+  static constexpr int kMStages = 4;
+  static constexpr int kSteps = 4;  // ring of step barriers, >= both stage counts
   static constexpr int kOBufs = D == 64 ? 2 : 1;
   static constexpr int kOCol = 384;
   static constexpr int kQ = 0;
   static constexpr int kK = 2 * kTileBytes;
   static constexpr int kV = kK + kKStages * kTileBytes;
   static constexpr int kMetaBits = kV + kVStages * kTileBytes;
-  static constexpr int kMetaKind = kMetaBits + kVStages * 2048;
-  static constexpr int kBar = kMetaKind + 16 * ((kVStages * 4 + 15) / 16);
-  // q_full[2] q_empty[2] s_full[2] s_empty[2] p_full[2] p_empty[2] o_full[2] o_empty[2]
-  // done, k_full[SK] k_empty[SK] v_full[SV] v_empty[SV]
-  static constexpr int kNumBars = 17 + 2 * kKStages + 2 * kVStages;
+  static constexpr int kMetaKind = kMetaBits + kMStages * 2048;
+  static constexpr int kBar = kMetaKind + 16 * ((kMStages * 4 + 15) / 16);
+  // q_full[2] q_empty[2] o_full[2] o_empty[2] e_done[2] done, s_ready[kSteps],
+  // step[kSteps], k_full[SK] v_full[SV] m_full[SM] m_empty[SM]
+  static constexpr int kNumBars = 11 + 2 * kSteps + kKStages + kVStages + 2 * kMStages;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kSteps >= kKStages && kSteps >= kVStages && kSteps >= 3, "step ring");
 };
 
 template <int D>
@@ -654,7 +657,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fwd_sigmoid_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const FwdParams p) {
   using L = SigLayout<D>;
-  constexpr int SK = L::kKStages, SV = L::kVStages, OB = L::kOBufs;
+  constexpr int SK = L::kKStages, SV = L::kVStages, SM = L::kMStages, NS = L::kSteps;
+  constexpr int OB = L::kOBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -663,17 +667,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 2;
-  uint64_t* s_full = bars + 4;
-  uint64_t* s_empty = bars + 6;
-  uint64_t* p_full = bars + 8;
-  uint64_t* p_empty = bars + 10;
-  uint64_t* o_full = bars + 12;
-  uint64_t* o_empty = bars + 14;
-  uint64_t* done = bars + 16;
-  uint64_t* k_full = bars + 17;
-  uint64_t* k_empty = k_full + SK;
-  uint64_t* v_full = k_empty + SK;
-  uint64_t* v_empty = v_full + SV;
+  uint64_t* o_full = bars + 4;
+  uint64_t* o_empty = bars + 6;
+  uint64_t* e_done = bars + 8;
+  uint64_t* done = bars + 10;
+  uint64_t* s_ready = bars + 11;
+  uint64_t* step = s_ready + NS;
+  uint64_t* k_full = step + NS;
+  uint64_t* v_full = k_full + SK;
+  uint64_t* m_full = v_full + SV;
+  uint64_t* m_empty = m_full + SM;
   uint32_t* meta_bits = reinterpret_cast<uint32_t*>(smem + L::kMetaBits);
   int* meta_kind = reinterpret_cast<int*>(smem + L::kMetaKind);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -685,21 +688,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(q_full + i, 1);
       mbar_init(q_empty + i, 1);
-      mbar_init(s_full + i, 1);
-      mbar_init(s_empty + i, 4);
-      mbar_init(p_full + i, 4);
-      mbar_init(p_empty + i, 1);
       mbar_init(o_full + i, 1);
       mbar_init(o_empty + i, 8);
+      mbar_init(e_done + i, 8);
     }
     mbar_init(done, 1);
-    for (int i = 0; i < SK; ++i) {
-      mbar_init(k_full + i, 1);
-      mbar_init(k_empty + i, 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(s_ready + i, 1);
+      mbar_init(step + i, 1);
     }
-    for (int i = 0; i < SV; ++i) {
-      mbar_init(v_full + i, 1);
-      mbar_init(v_empty + i, 1);
+    for (int i = 0; i < SK; ++i) mbar_init(k_full + i, 1);
+    for (int i = 0; i < SV; ++i) mbar_init(v_full + i, 1);
+    for (int i = 0; i < SM; ++i) {
+      mbar_init(m_full + i, 1);
+      mbar_init(m_empty + i, 8);
     }
     *abort_flag = 0;
     *drain_flag = 0;
@@ -711,27 +713,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 || warp == 2) {
-    // ---------------------------------------------------------------- TMA producers
-    // warp 0: Q of each item and the K ring; warp 2: the V ring with each tile's kind and
-    // bitmask.  All 32 lanes fetch the list entries of the next 32 tiles in one round
-    // trip; lane 0 waits and issues the copies.
-    const bool is_k = warp == 0;
-    if (lane == 0) {
-      tma_prefetch_desc(is_k ? &tk : &tv);
-      if (is_k) tma_prefetch_desc(&tq);
+  if (warp == 0 || warp == 2 || warp == 3) {
+    // ---------------------------------------------------------------- producers
+    // warp 0: Q of each item and the K ring (slot of tile u free after step u); warp 2:
+    // the V ring (slot of tile u free after step u + 2); warp 3: each tile's kind and
+    // PARTIAL bitmask (slot released by the epilogue).  All 32 lanes fetch the list
+    // entries of the next 32 tiles in one round trip; lane 0 waits and issues the copies.
+    const int role = warp == 0 ? 0 : (warp == 2 ? 1 : 2);
+    if (lane == 0 && role < 2) {
+      tma_prefetch_desc(role == 0 ? &tk : &tv);
+      if (role == 0) tma_prefetch_desc(&tq);
     }
-    const int NS = is_k ? SK : SV;
-    uint64_t* full = is_k ? k_full : v_full;
-    uint64_t* empty = is_k ? k_empty : v_empty;
-    const int ring = is_k ? L::kK : L::kV;
-    const CUtensorMap* map = is_k ? &tk : &tv;
+    const int NR = role == 0 ? SK : (role == 1 ? SV : SM);
+    uint64_t* full = role == 0 ? k_full : (role == 1 ? v_full : m_full);
+    const int ring = role == 0 ? L::kK : L::kV;
+    const CUtensorMap* map = role == 0 ? &tk : &tv;
     int t = 0, i = 0;
     bool ok = true;
     for (ItemIter iter(p); ok && iter.valid(); iter.advance()) {
       const Item it = iter.cur;
       if (it.n == 0) continue;
-      if (is_k) {
+      if (role == 0) {
         const int qb = i & 1;
         if (lane == 0) {
           if (i >= 2) ok = mbar_wait(q_empty + qb, ((i >> 1) - 1) & 1, wctx);
@@ -750,8 +752,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int jj = j0 + lane;
         int kt_l = 0, kd_l = 0, pi_l = 0;
         if (jj < it.n) {
-          kt_l = p.col_idx[it.e0 + jj];
-          if (!is_k) kd_l = p.kind[it.e0 + jj];
+          if (role < 2) kt_l = p.col_idx[it.e0 + jj];
+          else kd_l = p.kind[it.e0 + jj];
         }
         if (kd_l == 2) pi_l = p.pidx[it.e0 + jj];
         const int jn = min(32, it.n - j0);
@@ -759,18 +761,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int kt = __shfl_sync(0xFFFFFFFFu, kt_l, u);
           const int kd = __shfl_sync(0xFFFFFFFFu, kd_l, u);
           const int pi = __shfl_sync(0xFFFFFFFFu, pi_l, u);
-          const int s = t % NS;
+          const int s = t % NR;
           if (lane == 0) {
-            if (t >= NS) ok = mbar_wait(empty + s, ((t / NS) - 1) & 1, wctx);
+            if (t >= NR) {
+              if (role == 2) {
+                ok = mbar_wait(m_empty + s, ((t / NR) - 1) & 1, wctx);
+              } else {
+                // K of tile x is consumed by S_x, V of tile x by the PV of step x + 2
+                const int x = t - NR;
+                ok = role == 0 ? mbar_wait(s_ready + x % NS, (x / NS) & 1, wctx)
+                               : mbar_wait(step + (x + 2) % NS, ((x + 2) / NS) & 1, wctx);
+              }
+            }
             if (ok) {
-              if (!is_k) meta_kind[s] = kd;
-              mbar_arrive_expect_tx(full + s, L::kTileBytes + (kd == 2 ? 2048 : 0));
-              for (int x = 0; x < L::kBoxes; ++x)
-                tma_load_4d(smem + ring + s * L::kTileBytes + x * L::kBoxBytes, map, full + s,
-                            x * 64, kt * kTile, it.h, it.b);
-              if (kd == 2)
-                bulk_load(meta_bits + s * 512, p.bits + static_cast<int64_t>(pi) * 512, 2048,
-                          full + s);
+              if (role < 2) {
+                mbar_arrive_expect_tx(full + s, L::kTileBytes);
+                for (int x = 0; x < L::kBoxes; ++x)
+                  tma_load_4d(smem + ring + s * L::kTileBytes + x * L::kBoxBytes, map, full + s,
+                              x * 64, kt * kTile, it.h, it.b);
+              } else {
+                meta_kind[s] = kd;
+                if (kd == 2) {
+                  mbar_arrive_expect_tx(full + s, 2048);
+                  bulk_load(meta_bits + s * 512, p.bits + static_cast<int64_t>(pi) * 512, 2048,
+                            full + s);
+                } else {
+                  mbar_arrive(full + s);
+                }
+              }
             }
           }
           ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
@@ -781,36 +799,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && *abort_flag) {
       // Let the copies still in flight land before the CTA's shared memory goes away.
       const WaitCtx drain{p.status, p.wait_ns, drain_flag};
-      if (is_k)
+      if (role == 0)
         for (int u = max(0, i - 2); u < i; ++u) mbar_wait(q_full + (u & 1), (u >> 1) & 1, drain);
-      for (int u = max(0, t - NS); u < t; ++u) mbar_wait(full + u % NS, (u / NS) & 1, drain);
+      for (int u = max(0, t - NR); u < t; ++u) mbar_wait(full + u % NR, (u / NR) & 1, drain);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      // PVs still to issue (oldest first): global tile, item number, first / last of item
-      int pv_t[2] = {-1, -1}, pv_i[2] = {0, 0};
+      // the two PVs still to issue (oldest first): item number, first / last of item
+      int pv_i[2] = {0, 0};
       bool pv_first[2] = {false, false}, pv_last[2] = {false, false};
       bool ok = true;
-      auto issue_pv = [&](int t, int i, bool first, bool last) -> bool {
-        const int pb = t & 1, sv = t % SV, ob = i % OB;
-        if (!mbar_wait(p_full + pb, (t >> 1) & 1, wctx)) return false;
-        if (!mbar_wait(v_full + sv, (t / SV) & 1, wctx)) return false;
-        if (first && i >= OB && !mbar_wait(o_empty + ob, ((i / OB) - 1) & 1, wctx)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(smem + L::kV + sv * L::kTileBytes);
-        const uint32_t o_tmem = tmem + L::kOCol + ob * D;
-        const uint32_t p_tmem = tmem + 256 + pb * 64;
+      // O += P_x V_x for tile x = u - 2, after the epilogue finished tile x
+      auto wait_pv = [&](int x, int i, bool first) -> bool {
+        if (!mbar_wait(e_done + (x & 1), (x >> 1) & 1, wctx)) return false;
+        if (!mbar_wait(v_full + x % SV, (x / SV) & 1, wctx)) return false;
+        if (first && i >= OB && !mbar_wait(o_empty + i % OB, ((i / OB) - 1) & 1, wctx))
+          return false;
+        return true;
+      };
+      auto issue_pv = [&](int x, int i, bool first) {
+        const uint32_t v_base = smem_u32(smem + L::kV + (x % SV) * L::kTileBytes);
+        const uint32_t o_tmem = tmem + L::kOCol + (i % OB) * D;
+        const uint32_t p_tmem = tmem + (x % 3) * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_base + kk * 2048, L::kBoxBytes, 1024),
-                 idesc_pv, (first && kk == 0) ? 0u : 1u);
-        mma_commit(v_empty + sv);
-        mma_commit(p_empty + pb);
-        if (last) mma_commit(o_full + ob);
-        return true;
+          mma_ts(o_tmem, p_tmem + (kk >> 2) * 64 + (kk & 3) * 8,
+                 smem_desc_sw128(v_base + kk * 2048, L::kBoxBytes, 1024), idesc_pv,
+                 (first && kk == 0) ? 0u : 1u);
       };
       int t = 0, i = 0;
       for (ItemIter iter(p); ok && iter.valid(); iter.advance()) {
@@ -820,35 +838,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(q_full + qb, (i >> 1) & 1, wctx))) break;
         const uint32_t q_base = smem_u32(smem + L::kQ + qb * L::kTileBytes);
         for (int j = 0; j < it.n; ++j, ++t) {
-          const int s = t % SK, sb = t & 1;
+          const int s = t % SK;
           if (!(ok = mbar_wait(k_full + s, (t / SK) & 1, wctx))) break;
-          if (t >= 2 && !(ok = mbar_wait(s_empty + sb, ((t >> 1) - 1) & 1, wctx))) break;
+          if (t >= 2 && !(ok = wait_pv(t - 2, pv_i[0], pv_first[0]))) break;
           tc_fence_after();
           const uint32_t k_base = smem_u32(smem + L::kK + s * L::kTileBytes);
-          const uint32_t d_tmem = tmem + sb * 128;
+          const uint32_t d_tmem = tmem + (t % 3) * 128;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
             mma_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
                    smem_desc_sw128(k_base + off, 16, 1024), idesc_qk, kk > 0);
           }
-          mma_commit(s_full + sb);
-          mma_commit(k_empty + s);
+          mma_commit(s_ready + t % NS);
+          if (t >= 2) issue_pv(t - 2, pv_i[0], pv_first[0]);
+          mma_commit(step + t % NS);
+          if (t >= 2 && pv_last[0]) mma_commit(o_full + pv_i[0] % OB);
           if (j == it.n - 1) mma_commit(q_empty + qb);
-          if (pv_t[0] >= 0 && !(ok = issue_pv(pv_t[0], pv_i[0], pv_first[0], pv_last[0]))) break;
-          pv_t[0] = pv_t[1];
           pv_i[0] = pv_i[1];
           pv_first[0] = pv_first[1];
           pv_last[0] = pv_last[1];
-          pv_t[1] = t;
           pv_i[1] = i;
           pv_first[1] = j == 0;
           pv_last[1] = j == it.n - 1;
         }
         ++i;
       }
-      for (int u = 0; ok && u < 2; ++u)
-        if (pv_t[u] >= 0) ok = issue_pv(pv_t[u], pv_i[u], pv_first[u], pv_last[u]);
+      // the last two steps: PV only
+      for (int u = t; ok && u < t + 2; ++u) {
+        if (u >= 2) {
+          if (!(ok = wait_pv(u - 2, pv_i[0], pv_first[0]))) break;
+          tc_fence_after();
+          issue_pv(u - 2, pv_i[0], pv_first[0]);
+          mma_commit(step + u % NS);
+          if (pv_last[0]) mma_commit(o_full + pv_i[0] % OB);
+        }
+        pv_i[0] = pv_i[1];
+        pv_first[0] = pv_first[1];
+        pv_last[0] = pv_last[1];
+      }
       // every MMA complete before the TMEM is released
       mma_commit(done);
       const WaitCtx drain{p.status, p.wait_ns, drain_flag};
@@ -856,15 +884,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- epilogue
-    // Thread = query row (TMEM lane).  A tile is read in four chunks of 32 columns whose
-    // TMEM loads overlap the previous chunk's math; P of keys [32c, 32c+32) goes to the
-    // warpgroup's P columns [16c, 16c+16).
+    // Warpgroup g, thread = query row: keys [64g, 64g+64) of every tile, loaded as two
+    // chunks of 32 columns; P of keys [64g + 32c, +32) overwrites columns [64g + 16c, +16).
     const int g = (warp - kEpiWarp0) >> 2;
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const uint32_t s_base = t_lane + g * 128;
-    const uint32_t p_base = t_lane + 256 + g * 64;
     constexpr int kOc = D / 2;  // O columns written by this warpgroup
     const float2 c1 = make_float2(0.5f * p.scale, 0.5f * p.scale);
     const float2 half2 = make_float2(0.5f, 0.5f);
@@ -931,68 +956,69 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const float2 c0 = make_float2(0.5f * bias_r, 0.5f * bias_r);
-      const int t_end = t + it.n;
-      for (int tt = t + ((t & 1) != g ? 1 : 0); tt < t_end; tt += 2) {
-        const int sv = tt % SV;
-        // v_full of the tile's V stage also publishes the kind and bitmask staged with it
-        if (ok) ok = mbar_wait(s_full + g, (tt >> 1) & 1, wctx);
-        if (ok) ok = mbar_wait(v_full + sv, (tt / SV) & 1, wctx);
-        ok = __all_sync(0xFFFFFFFFu, ok);
-        if (!ok) break;
+      // Keys [64g, 64g+32) of a tile are chunk A, [64g+32, 64g+64) chunk B.  Chunk A of the
+      // next tile of the item is loaded while chunk B of this one is computed.
+      uint32_t ca[32], cb[32];
+      bool masked = false;
+      uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+      // waits for S and the kind / bitmask of tile u, then starts loading its chunk A
+      auto fetch = [&](int u) -> bool {
+        bool w = mbar_wait(s_ready + u % NS, (u / NS) & 1, wctx);
+        w = w && mbar_wait(m_full + u % SM, (u / SM) & 1, wctx);
+        w = __all_sync(0xFFFFFFFFu, w);
+        if (!w) return false;
         tc_fence_after();
-        const bool masked = meta_kind[sv] == 2;
-        uint4 mb = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
-        if (masked) mb = *reinterpret_cast<const uint4*>(meta_bits + sv * 512 + row * 4);
-        uint32_t buf[2][32];
-        tmem_ld32(s_base, buf[0]);
-        tmem_wait_ld();
+        masked = meta_kind[u % SM] == 2;
+        mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+        if (masked) mb = *reinterpret_cast<const uint2*>(meta_bits + (u % SM) * 512 + row * 4 + g * 2);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(m_empty + u % SM);
+        tmem_ld32(t_lane + (u % 3) * 128 + g * 64, ca);
+        return true;
+      };
+      auto weights = [&](const uint32_t (&sv)[32], uint32_t mw, uint32_t (&pk)[16]) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c < 3) tmem_ld32(s_base + 32 * (c + 1), buf[(c + 1) & 1]);
-          const uint32_t mw = c == 0 ? mb.x : (c == 1 ? mb.y : (c == 2 ? mb.z : mb.w));
-          uint32_t pk[16];
-#pragma unroll
-          for (int cc = 0; cc < 32; cc += 2) {
-            const float2 x = fma2(make_float2(__uint_as_float(buf[c & 1][cc]),
-                                              __uint_as_float(buf[c & 1][cc + 1])),
-                                  c1, c0);
-            float2 th = make_float2(tanh_approx(x.x), tanh_approx(x.y));
-            if (masked) {
-              th.x = ((mw >> cc) & 1u) ? th.x : -1.0f;
-              th.y = ((mw >> (cc + 1)) & 1u) ? th.y : -1.0f;
-            }
-            const float2 pw = fma2(th, half2, half2);
-            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
+        for (int cc = 0; cc < 32; cc += 2) {
+          const float2 x = fma2(make_float2(__uint_as_float(sv[cc]), __uint_as_float(sv[cc + 1])),
+                                c1, c0);
+          float2 th = make_float2(tanh_approx(x.x), tanh_approx(x.y));
+          if (masked) {
+            th.x = ((mw >> cc) & 1u) ? th.x : -1.0f;
+            th.y = ((mw >> (cc + 1)) & 1u) ? th.y : -1.0f;
           }
-          if (c == 0 && tt >= 2) {
-            // P buffer g is free once O += P V of this warpgroup's previous tile completed
-            ok = mbar_wait(p_empty + g, ((tt >> 1) - 1) & 1, wctx);
-            ok = __all_sync(0xFFFFFFFFu, ok);
-            if (!ok) break;
-            tc_fence_after();
-          }
-          tmem_st16(p_base + 16 * c, pk);
-          if (c < 3) tmem_wait_ld();
-          if (c == 2) {
-            // all of S read: the MMA may overwrite this buffer with the tile after next
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_empty + g);
-          }
+          const float2 pw = fma2(th, half2, half2);
+          pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
         }
-        if (!ok) break;
+      };
+      if (!(ok = fetch(t))) break;
+      for (int j = 0; j < it.n; ++j, ++t) {
+        const uint32_t sp = t_lane + (t % 3) * 128 + g * 64;
+        tmem_wait_ld();  // chunk A
+        tmem_ld32(sp + 32, cb);
+        uint32_t pk[16];
+        weights(ca, mb.x, pk);
+        tmem_st16(sp, pk);
+        tmem_wait_ld();  // chunk B
+        const bool masked_t = masked;
+        const uint32_t mw_b = mb.y;
+        if (j + 1 < it.n && !(ok = fetch(t + 1))) break;
+        {
+          const bool m_next = masked;
+          masked = masked_t;
+          weights(cb, mw_b, pk);
+          masked = m_next;
+        }
+        tmem_st16(sp + 16, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + g);
+        if (lane == 0) mbar_arrive(e_done + (t & 1));
         if (pend) flush_o();
       }
       if (!ok) break;
-      if (pend) flush_o();
       pend = true;
       pit = it;
       pi = i;
-      t = t_end;
       ++i;
     }
     if (ok && pend) flush_o();
