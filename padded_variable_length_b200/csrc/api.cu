@@ -125,11 +125,13 @@ __global__ void k_wait_selftest(int* status, unsigned long long limit_ns) {
     abort_flag = 0;
     fence_barrier_init();
   }
+  __syncwarp();
   __syncthreads();
   if (threadIdx.x == 0) {
     const WaitCtx w{status, limit_ns, &abort_flag};
     mbar_wait(&bar, 0, w);
   }
+  __syncwarp();
   __syncthreads();
 }
 

@@ -284,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *drain_flag = 0;
     fence_barrier_init();
   }
+  __syncwarp();
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
@@ -600,6 +601,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++ii;
     }
   }
+  // Single-lane roles (MMA issue, copy issue) end at different times than the rest of
+  // their warp: reconverge every warp before the CTA-wide barrier, which counts warps.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -685,6 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *drain_flag = 0;
     fence_barrier_init();
   }
+  __syncwarp();
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
@@ -959,6 +964,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++ii;
     }
   }
+  // Single-lane roles (MMA issue, copy issue) end at different times than the rest of
+  // their warp: reconverge every warp before the CTA-wide barrier, which counts warps.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *drain_flag = 0;
     fence_barrier_init();
   }
+  __syncwarp();
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
@@ -586,6 +587,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++i;
     }
   }
+  // Single-lane roles (MMA issue, copy issue) end at different times than the rest of
+  // their warp: reconverge every warp before the CTA-wide barrier, which counts warps.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -609,20 +613,19 @@ int num_sms() {
 }
 
 // ------------------------------------------------------------------------------------
-// Sigmoid forward: one tensor-pipe step per tile.
+// Sigmoid forward.
 //
 // The weights of sigmoid attention need no row statistics, so nothing but buffers ties
-// one key tile to the next, and the kernel is organised to need as few hand-offs per tile
-// as possible.  Step u of the MMA issuer, started when the epilogue has finished tile
-// u - 2, issues S_u = Q K_u^T (commit s_ready: S_u is ready and K_u consumed) and then
-// O += P_{u-2} V_{u-2} (commit step: V_{u-2} consumed).  S and P of a tile share a
-// buffer (P overwrites the columns of S its own warpgroup has read), and three such
-// buffers let the epilogue work on tile u - 1 while step u runs; the epilogue loads the
-// first half of its columns of tile u + 1 while it computes the second half of tile u.
+// one key tile to the next.  S and P of a tile share a TMEM buffer (P overwrites columns
+// of S already read), and there are three such buffers: the MMA issuer computes S_t as
+// soon as O += P_{t-3} V_{t-3}, the last user of that buffer, is issued, i.e. once the
+// epilogue has finished tile t - 3.  One commit per MMA group: s_ready (S_t ready, K_t
+// consumed) and step (V_t consumed).
 // Warps: 0 Q/K producer, 1 TMEM allocator + MMA issuer, 2 V producer, 3 kind / bitmask
-// producer, 4-11 two epilogue warpgroups: thread = query row = TMEM lane, warpgroup g on
-// keys [64g, 64g+64) of every tile.  The O of an item is written out after the first
-// tile of the next item, when the last PV of the item has long completed.
+// producer, 4-11 two epilogue warpgroups that take alternate tiles (thread = query row =
+// TMEM lane).  The O of an item is written out after the first tile of the next item,
+// when the last PV of the item has long completed; warpgroup g writes O columns
+// [g d/2, (g+1) d/2).
 // TMEM columns: S/P buffers [0,128), [128,256), [256,384); O in [384,512) (two buffers
 // of 64 columns for d = 64, one of 128 for d = 128).  P of keys 16kk.. (the A operand of
 // the kk-th K-step of the PV MMA) sits at column 64 (kk / 4) + 8 (kk % 4) of its buffer.
@@ -643,9 +646,9 @@ struct SigLayout {
   static constexpr int kMetaBits = kV + kVStages * kTileBytes;
   static constexpr int kMetaKind = kMetaBits + kMStages * 2048;
   static constexpr int kBar = kMetaKind + 16 * ((kMStages * 4 + 15) / 16);
-  // q_full[2] q_empty[2] o_full[2] o_empty[2] e_done[2] done, s_ready[kSteps],
+  // q_full[2] q_empty[2] o_full[2] o_empty[2] e_done[4] done, s_ready[kSteps],
   // step[kSteps], k_full[SK] v_full[SV] m_full[SM] m_empty[SM]
-  static constexpr int kNumBars = 11 + 2 * kSteps + kKStages + kVStages + 2 * kMStages;
+  static constexpr int kNumBars = 13 + 2 * kSteps + kKStages + kVStages + 2 * kMStages;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -670,8 +673,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_full = bars + 4;
   uint64_t* o_empty = bars + 6;
   uint64_t* e_done = bars + 8;
-  uint64_t* done = bars + 10;
-  uint64_t* s_ready = bars + 11;
+  uint64_t* done = bars + 12;
+  uint64_t* s_ready = bars + 13;
   uint64_t* step = s_ready + NS;
   uint64_t* k_full = step + NS;
   uint64_t* v_full = k_full + SK;
@@ -690,8 +693,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(q_empty + i, 1);
       mbar_init(o_full + i, 1);
       mbar_init(o_empty + i, 8);
-      mbar_init(e_done + i, 8);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(e_done + i, 4);
     mbar_init(done, 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(s_ready + i, 1);
@@ -701,12 +704,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < SV; ++i) mbar_init(v_full + i, 1);
     for (int i = 0; i < SM; ++i) {
       mbar_init(m_full + i, 1);
-      mbar_init(m_empty + i, 8);
+      mbar_init(m_empty + i, 4);
     }
     *abort_flag = 0;
     *drain_flag = 0;
     fence_barrier_init();
   }
+  __syncwarp();
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
@@ -767,10 +771,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (role == 2) {
                 ok = mbar_wait(m_empty + s, ((t / NR) - 1) & 1, wctx);
               } else {
-                // K of tile x is consumed by S_x, V of tile x by the PV of step x + 2
+                // K of tile x is consumed by S_x (s_ready), V of tile x by its PV (step)
                 const int x = t - NR;
-                ok = role == 0 ? mbar_wait(s_ready + x % NS, (x / NS) & 1, wctx)
-                               : mbar_wait(step + (x + 2) % NS, ((x + 2) / NS) & 1, wctx);
+                ok = mbar_wait((role == 0 ? s_ready : step) + x % NS, (x / NS) & 1, wctx);
               }
             }
             if (ok) {
@@ -808,74 +811,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      // the two PVs still to issue (oldest first): item number, first / last of item
-      int pv_i[2] = {0, 0};
-      bool pv_first[2] = {false, false}, pv_last[2] = {false, false};
+      // FIFO of the (up to three) tiles whose PV is still to issue, oldest first:
+      // item number << 2 | first of item << 1 | last of item
+      int pq0 = 0, pq1 = 0, pq2 = 0;
       bool ok = true;
-      // O += P_x V_x for tile x = u - 2, after the epilogue finished tile x
-      auto wait_pv = [&](int x, int i, bool first) -> bool {
-        if (!mbar_wait(e_done + (x & 1), (x >> 1) & 1, wctx)) return false;
-        if (!mbar_wait(v_full + x % SV, (x / SV) & 1, wctx)) return false;
-        if (first && i >= OB && !mbar_wait(o_empty + i % OB, ((i / OB) - 1) & 1, wctx))
+      // The issue path is kept short (it shares its sub-partition's issue slots with two
+      // epilogue warps): descriptors are (lo, hi) halves stepped by constant offsets, ring
+      // positions are masks of power-of-two stage counts, buffer t % 3 a running counter.
+      constexpr uint32_t kHiKm = sw128_desc_hi(1024);       // Q, K: K-major, SBO 1024
+      constexpr uint32_t kHiMn = sw128_desc_hi(1024);       // V: MN-major, SBO 1024
+      const uint32_t q_lo0 = sw128_desc_lo(smem_u32(smem + L::kQ), 16);
+      const uint32_t k_lo0 = sw128_desc_lo(smem_u32(smem + L::kK), 16);
+      const uint32_t v_lo0 = sw128_desc_lo(smem_u32(smem + L::kV), L::kBoxBytes);
+      constexpr uint32_t kTileLo = L::kTileBytes >> 4;
+      static_assert((SK & (SK - 1)) == 0 && (SV & (SV - 1)) == 0 && NS == 4, "ring sizes");
+      // O += P_x V_x for the oldest tile x of the FIFO (buffer b3 = x % 3), once the
+      // epilogue has finished it; commits step(x)
+      auto pv = [&](int x, uint32_t b3) -> bool {
+        const int i = pq0 >> 2;
+        const bool first = (pq0 & 2) != 0, last = (pq0 & 1) != 0;
+        pq0 = pq1;
+        pq1 = pq2;
+        const int sv = x & (SV - 1);
+        if (!mbar_wait(e_done + (x & 3), (x >> 2) & 1, wctx)) return false;
+        if (!mbar_wait(v_full + sv, (x / SV) & 1, wctx)) return false;
+        const int ob = OB == 1 ? 0 : (i & 1);
+        if (first && i >= OB && !mbar_wait(o_empty + ob, ((i / OB) - 1) & 1, wctx))
           return false;
+        tc_fence_after();
+        const uint32_t v_lo = v_lo0 + sv * kTileLo;
+        const uint32_t o_tmem = tmem + L::kOCol + ob * D;
+        const uint32_t p_tmem = tmem + b3 * 128;
+        mma_ts_lh(o_tmem, p_tmem, v_lo, kHiMn, idesc_pv, first ? 0u : 1u);
+#pragma unroll
+        for (int kk = 1; kk < 8; ++kk)
+          mma_ts_lh(o_tmem, p_tmem + (kk >> 2) * 64 + (kk & 3) * 8, v_lo + kk * 128, kHiMn,
+                    idesc_pv, 1u);
+        mma_commit(step + (x & 3));
+        if (last) mma_commit(o_full + ob);
         return true;
       };
-      auto issue_pv = [&](int x, int i, bool first) {
-        const uint32_t v_base = smem_u32(smem + L::kV + (x % SV) * L::kTileBytes);
-        const uint32_t o_tmem = tmem + L::kOCol + (i % OB) * D;
-        const uint32_t p_tmem = tmem + (x % 3) * 128;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(o_tmem, p_tmem + (kk >> 2) * 64 + (kk & 3) * 8,
-                 smem_desc_sw128(v_base + kk * 2048, L::kBoxBytes, 1024), idesc_pv,
-                 (first && kk == 0) ? 0u : 1u);
-      };
       int t = 0, i = 0;
+      uint32_t b3 = 0;  // t % 3
       for (ItemIter iter(p); ok && iter.valid(); iter.advance()) {
         const Item it = iter.cur;
         if (it.n == 0) continue;
         const int qb = i & 1;
         if (!(ok = mbar_wait(q_full + qb, (i >> 1) & 1, wctx))) break;
-        const uint32_t q_base = smem_u32(smem + L::kQ + qb * L::kTileBytes);
+        const uint32_t q_lo = q_lo0 + qb * kTileLo;
         for (int j = 0; j < it.n; ++j, ++t) {
-          const int s = t % SK;
+          // S_t goes to the buffer of tile t - 3: its PV first (the pipe runs in order)
+          if (t >= 3 && !(ok = pv(t - 3, b3))) break;
+          const int s = t & (SK - 1);
           if (!(ok = mbar_wait(k_full + s, (t / SK) & 1, wctx))) break;
-          if (t >= 2 && !(ok = wait_pv(t - 2, pv_i[0], pv_first[0]))) break;
           tc_fence_after();
-          const uint32_t k_base = smem_u32(smem + L::kK + s * L::kTileBytes);
-          const uint32_t d_tmem = tmem + (t % 3) * 128;
+          const uint32_t k_lo = k_lo0 + s * kTileLo;
+          const uint32_t d_tmem = tmem + b3 * 128;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-            mma_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
-                   smem_desc_sw128(k_base + off, 16, 1024), idesc_qk, kk > 0);
+            const uint32_t off = (kk >> 2) * (L::kBoxBytes >> 4) + (kk & 3) * 2;
+            mma_ss_lh(d_tmem, q_lo + off, k_lo + off, kHiKm, idesc_qk, kk > 0 ? 1u : 0u);
           }
-          mma_commit(s_ready + t % NS);
-          if (t >= 2) issue_pv(t - 2, pv_i[0], pv_first[0]);
-          mma_commit(step + t % NS);
-          if (t >= 2 && pv_last[0]) mma_commit(o_full + pv_i[0] % OB);
+          mma_commit(s_ready + (t & 3));
           if (j == it.n - 1) mma_commit(q_empty + qb);
-          pv_i[0] = pv_i[1];
-          pv_first[0] = pv_first[1];
-          pv_last[0] = pv_last[1];
-          pv_i[1] = i;
-          pv_first[1] = j == 0;
-          pv_last[1] = j == it.n - 1;
+          const int info = (i << 2) | (j == 0 ? 2 : 0) | (j == it.n - 1 ? 1 : 0);
+          if (t == 0) pq0 = info;
+          else if (t == 1) pq1 = info;
+          else pq2 = info;
+          b3 = b3 == 2 ? 0 : b3 + 1;
         }
         ++i;
       }
-      // the last two steps: PV only
-      for (int u = t; ok && u < t + 2; ++u) {
-        if (u >= 2) {
-          if (!(ok = wait_pv(u - 2, pv_i[0], pv_first[0]))) break;
-          tc_fence_after();
-          issue_pv(u - 2, pv_i[0], pv_first[0]);
-          mma_commit(step + u % NS);
-          if (pv_last[0]) mma_commit(o_full + pv_i[0] % OB);
-        }
-        pv_i[0] = pv_i[1];
-        pv_first[0] = pv_first[1];
-        pv_last[0] = pv_last[1];
+      // the last PVs: tile x uses buffer x % 3; b3 is t % 3 here
+      for (int x = max(0, t - 3); ok && x < t; ++x) {
+        const uint32_t bx = static_cast<uint32_t>((x - t + 3) % 3 + static_cast<int>(b3)) % 3;
+        ok = pv(x, bx);
       }
       // every MMA complete before the TMEM is released
       mma_commit(done);
@@ -884,8 +894,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- epilogue
-    // Warpgroup g, thread = query row: keys [64g, 64g+64) of every tile, loaded as two
-    // chunks of 32 columns; P of keys [64g + 32c, +32) overwrites columns [64g + 16c, +16).
+    // Ping-pong: warpgroup g takes the tiles t with t % 2 == g, all 128 keys, in four
+    // chunks of 32 columns whose TMEM loads overlap the previous chunk's math; while one
+    // warpgroup waits, loads or stores, the other keeps the MUFU busy.  Thread = query row.
+    // P of chunk c (keys [32c, 32c+32)) overwrites columns 64 (c / 2) + 16 (c % 2) + [0, 16)
+    // of the tile's buffer, which belong to chunk 0 or 2, already read.
     const int g = (warp - kEpiWarp0) >> 2;
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
@@ -956,73 +969,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const float2 c0 = make_float2(0.5f * bias_r, 0.5f * bias_r);
-      // Keys [64g, 64g+32) of a tile are chunk A, [64g+32, 64g+64) chunk B.  Chunk A of the
-      // next tile of the item is loaded while chunk B of this one is computed.
-      uint32_t ca[32], cb[32];
-      bool masked = false;
-      uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-      // waits for S and the kind / bitmask of tile u, then starts loading its chunk A
-      auto fetch = [&](int u) -> bool {
-        bool w = mbar_wait(s_ready + u % NS, (u / NS) & 1, wctx);
-        w = w && mbar_wait(m_full + u % SM, (u / SM) & 1, wctx);
-        w = __all_sync(0xFFFFFFFFu, w);
-        if (!w) return false;
+      const int t_end = t + it.n;
+      for (int tt = t + ((t & 1) != g ? 1 : 0); tt < t_end; tt += 2) {
+        const int ms = tt % SM;
+        if (ok) ok = mbar_wait(s_ready + tt % NS, (tt / NS) & 1, wctx);
+        if (ok) ok = mbar_wait(m_full + ms, (tt / SM) & 1, wctx);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
         tc_fence_after();
-        masked = meta_kind[u % SM] == 2;
-        mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        if (masked) mb = *reinterpret_cast<const uint2*>(meta_bits + (u % SM) * 512 + row * 4 + g * 2);
+        const bool masked = meta_kind[ms] == 2;
+        uint4 mb = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+        if (masked) mb = *reinterpret_cast<const uint4*>(meta_bits + ms * 512 + row * 4);
+        const uint32_t sp = t_lane + (tt % 3) * 128;
+        uint32_t buf[2][32];
+        tmem_ld32(sp, buf[0]);
         __syncwarp();
-        if (lane == 0) mbar_arrive(m_empty + u % SM);
-        tmem_ld32(t_lane + (u % 3) * 128 + g * 64, ca);
-        return true;
-      };
-      auto weights = [&](const uint32_t (&sv)[32], uint32_t mw, uint32_t (&pk)[16]) {
+        if (lane == 0) mbar_arrive(m_empty + ms);
+        tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < 32; cc += 2) {
-          const float2 x = fma2(make_float2(__uint_as_float(sv[cc]), __uint_as_float(sv[cc + 1])),
-                                c1, c0);
-          float2 th = make_float2(tanh_approx(x.x), tanh_approx(x.y));
-          if (masked) {
-            th.x = ((mw >> cc) & 1u) ? th.x : -1.0f;
-            th.y = ((mw >> (cc + 1)) & 1u) ? th.y : -1.0f;
+        for (int c = 0; c < 4; ++c) {
+          if (c < 3) tmem_ld32(sp + 32 * (c + 1), buf[(c + 1) & 1]);
+          const uint32_t mw = c == 0 ? mb.x : (c == 1 ? mb.y : (c == 2 ? mb.z : mb.w));
+          uint32_t pk[16];
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            const float2 x = fma2(make_float2(__uint_as_float(buf[c & 1][cc]),
+                                              __uint_as_float(buf[c & 1][cc + 1])),
+                                  c1, c0);
+            float2 th = make_float2(tanh_approx(x.x), tanh_approx(x.y));
+            if (masked) {
+              th.x = ((mw >> cc) & 1u) ? th.x : -1.0f;
+              th.y = ((mw >> (cc + 1)) & 1u) ? th.y : -1.0f;
+            }
+            const float2 pw = fma2(th, half2, half2);
+            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
           }
-          const float2 pw = fma2(th, half2, half2);
-          pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
+          tmem_st16(sp + (c >> 1) * 64 + (c & 1) * 16, pk);
+          if (c < 3) tmem_wait_ld();
         }
-      };
-      if (!(ok = fetch(t))) break;
-      for (int j = 0; j < it.n; ++j, ++t) {
-        const uint32_t sp = t_lane + (t % 3) * 128 + g * 64;
-        tmem_wait_ld();  // chunk A
-        tmem_ld32(sp + 32, cb);
-        uint32_t pk[16];
-        weights(ca, mb.x, pk);
-        tmem_st16(sp, pk);
-        tmem_wait_ld();  // chunk B
-        const bool masked_t = masked;
-        const uint32_t mw_b = mb.y;
-        if (j + 1 < it.n && !(ok = fetch(t + 1))) break;
-        {
-          const bool m_next = masked;
-          masked = masked_t;
-          weights(cb, mw_b, pk);
-          masked = m_next;
-        }
-        tmem_st16(sp + 16, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(e_done + (t & 1));
+        if (lane == 0) mbar_arrive(e_done + (tt & 3));
         if (pend) flush_o();
       }
       if (!ok) break;
+      if (pend) flush_o();
       pend = true;
       pit = it;
       pi = i;
+      t = t_end;
       ++i;
     }
     if (ok && pend) flush_o();
   }
+  // Single-lane roles (MMA issue, copy issue) end at different times than the rest of
+  // their warp: reconverge every warp before the CTA-wide barrier, which counts warps.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
