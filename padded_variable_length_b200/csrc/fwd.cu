@@ -808,16 +808,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issue loop on warp-uniform values; lane 0 waits on barriers
+    // (the result is broadcast) and an elected lane issues each MMA and commit.
+    {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
       // FIFO of the (up to three) tiles whose PV is still to issue, oldest first:
       // item number << 2 | first of item << 1 | last of item
       int pq0 = 0, pq1 = 0, pq2 = 0;
       bool ok = true;
-      // The issue path is kept short (it shares its sub-partition's issue slots with two
-      // epilogue warps): descriptors are (lo, hi) halves stepped by constant offsets, ring
-      // positions are masks of power-of-two stage counts, buffer t % 3 a running counter.
+      // The issue path is kept short: descriptors are (lo, hi) halves stepped by constant
+      // offsets, ring positions are masks of power-of-two stage counts, buffer t % 3 a
+      // running counter.
       constexpr uint32_t kHiKm = sw128_desc_hi(1024);       // Q, K: K-major, SBO 1024
       constexpr uint32_t kHiMn = sw128_desc_hi(1024);       // V: MN-major, SBO 1024
       const uint32_t q_lo0 = sw128_desc_lo(smem_u32(smem + L::kQ), 16);
@@ -833,22 +835,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         pq0 = pq1;
         pq1 = pq2;
         const int sv = x & (SV - 1);
-        if (!mbar_wait(e_done + (x & 3), (x >> 2) & 1, wctx)) return false;
-        if (!mbar_wait(v_full + sv, (x / SV) & 1, wctx)) return false;
+        if (!mbar_wait_w(e_done + (x & 3), (x >> 2) & 1, wctx)) return false;
+        if (!mbar_wait_w(v_full + sv, (x / SV) & 1, wctx)) return false;
         const int ob = OB == 1 ? 0 : (i & 1);
-        if (first && i >= OB && !mbar_wait(o_empty + ob, ((i / OB) - 1) & 1, wctx))
+        if (first && i >= OB && !mbar_wait_w(o_empty + ob, ((i / OB) - 1) & 1, wctx))
           return false;
         tc_fence_after();
         const uint32_t v_lo = v_lo0 + sv * kTileLo;
         const uint32_t o_tmem = tmem + L::kOCol + ob * D;
         const uint32_t p_tmem = tmem + b3 * 128;
-        mma_ts_lh(o_tmem, p_tmem, v_lo, kHiMn, idesc_pv, first ? 0u : 1u);
+        mma_ts_lh_w(o_tmem, p_tmem, v_lo, kHiMn, idesc_pv, first ? 0u : 1u);
 #pragma unroll
         for (int kk = 1; kk < 8; ++kk)
-          mma_ts_lh(o_tmem, p_tmem + (kk >> 2) * 64 + (kk & 3) * 8, v_lo + kk * 128, kHiMn,
+          mma_ts_lh_w(o_tmem, p_tmem + (kk >> 2) * 64 + (kk & 3) * 8, v_lo + kk * 128, kHiMn,
                     idesc_pv, 1u);
-        mma_commit(step + (x & 3));
-        if (last) mma_commit(o_full + ob);
+        mma_commit_w(step + (x & 3));
+        if (last) mma_commit_w(o_full + ob);
         return true;
       };
       int t = 0, i = 0;
@@ -857,23 +859,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = iter.cur;
         if (it.n == 0) continue;
         const int qb = i & 1;
-        if (!(ok = mbar_wait(q_full + qb, (i >> 1) & 1, wctx))) break;
+        if (!(ok = mbar_wait_w(q_full + qb, (i >> 1) & 1, wctx))) break;
         const uint32_t q_lo = q_lo0 + qb * kTileLo;
         for (int j = 0; j < it.n; ++j, ++t) {
           // S_t goes to the buffer of tile t - 3: its PV first (the pipe runs in order)
           if (t >= 3 && !(ok = pv(t - 3, b3))) break;
           const int s = t & (SK - 1);
-          if (!(ok = mbar_wait(k_full + s, (t / SK) & 1, wctx))) break;
+          if (!(ok = mbar_wait_w(k_full + s, (t / SK) & 1, wctx))) break;
           tc_fence_after();
           const uint32_t k_lo = k_lo0 + s * kTileLo;
           const uint32_t d_tmem = tmem + b3 * 128;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * (L::kBoxBytes >> 4) + (kk & 3) * 2;
-            mma_ss_lh(d_tmem, q_lo + off, k_lo + off, kHiKm, idesc_qk, kk > 0 ? 1u : 0u);
+            mma_ss_lh_w(d_tmem, q_lo + off, k_lo + off, kHiKm, idesc_qk, kk > 0 ? 1u : 0u);
           }
-          mma_commit(s_ready + (t & 3));
-          if (j == it.n - 1) mma_commit(q_empty + qb);
+          mma_commit_w(s_ready + (t & 3));
+          if (j == it.n - 1) mma_commit_w(q_empty + qb);
           const int info = (i << 2) | (j == 0 ? 2 : 0) | (j == it.n - 1 ? 1 : 0);
           if (t == 0) pq0 = info;
           else if (t == 1) pq1 = info;
@@ -888,9 +890,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = pv(x, bx);
       }
       // every MMA complete before the TMEM is released
-      mma_commit(done);
+      mma_commit_w(done);
       const WaitCtx drain{p.status, p.wait_ns, drain_flag};
-      mbar_wait(done, 0, drain);
+      mbar_wait_w(done, 0, drain);
     }
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- epilogue
