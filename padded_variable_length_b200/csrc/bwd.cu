@@ -383,7 +383,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // d = 64: the whole warp runs the issue loop on warp-uniform values (lane 0 waits on
+    // barriers, the result is broadcast; an elected lane issues), which shortens the issue
+    // path.  d = 128 (MMA-bound, waits in the middle of each tile) issues from lane 0.
+    constexpr bool kW = D == 64;
+    if (kW || lane == 0) {
+      constexpr uint32_t kHi = sw128_desc_hi(1024);
       constexpr uint32_t idesc_half = idesc_bf16_f32(128, 64, false);  // S^T / dP^T halves
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);     // dV / dK
       // d = 64 (three Q / dO stages): the dV / dK MMAs of half h of a tile are issued just
@@ -395,9 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       // accumulating MMAs of half h of the q-tile with global index qt_, stage s, buffer ab
       auto acc_half = [&](int h, int qt_, int s, int ab, bool first, int item) -> bool {
-        if (!mbar_wait(p_full + h, qt_ & 1, wctx)) return false;
+        if (!mbar_wait_x<kW>(p_full + h, qt_ & 1, wctx)) return false;
         if (h == 0 && first && item >= ACB &&
-            !mbar_wait(acc_empty + ab, ((item / ACB) - 1) & 1, wctx))
+            !mbar_wait_x<kW>(acc_empty + ab, ((item / ACB) - 1) & 1, wctx))
           return false;
         tc_fence_after();
         const uint32_t q_s = smem_u32(smem + L::kQ + s * L::kTileBytes);
@@ -407,10 +412,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 4; ++kk) {
           const uint32_t acc = (first && h == 0 && kk == 0) ? 0u : 1u;
           const uint32_t boff = (4 * h + kk) * 2048;  // query rows 64h + 16kk
-          mma_ts(t_dv, tmem + 64 * h + kk * 8,
-                 smem_desc_sw128(do_s + boff, L::kBoxBytes, 1024), idesc_acc, acc);
-          mma_ts(t_dk, tmem + 128 + 64 * h + kk * 8,
-                 smem_desc_sw128(q_s + boff, L::kBoxBytes, 1024), idesc_acc, acc);
+          mma_ts_lh_x<kW>(t_dv, tmem + 64 * h + kk * 8, sw128_desc_lo(do_s + boff, L::kBoxBytes),
+                          kHi, idesc_acc, acc);
+          mma_ts_lh_x<kW>(t_dk, tmem + 128 + 64 * h + kk * 8,
+                          sw128_desc_lo(q_s + boff, L::kBoxBytes), kHi, idesc_acc, acc);
         }
         return true;
       };
@@ -418,23 +423,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + 64 * h, smem_desc_sw128(k_base + off, 16, 1024),
-                 smem_desc_sw128(q_s + off + h * 8192, 16, 1024), idesc_half, kk > 0);
+          mma_ss_lh_x<kW>(tmem + 64 * h, sw128_desc_lo(k_base + off, 16),
+                          sw128_desc_lo(q_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + 128 + 64 * h, smem_desc_sw128(v_base + off, 16, 1024),
-                 smem_desc_sw128(do_s + off + h * 8192, 16, 1024), idesc_half, kk > 0);
+          mma_ss_lh_x<kW>(tmem + 128 + 64 * h, sw128_desc_lo(v_base + off, 16),
+                          sw128_desc_lo(do_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
         }
-        mma_commit(s_full + h);
+        mma_commit_x<kW>(s_full + h);
       };
       // the q-tile whose accumulating MMAs are deferred (kDeferAcc)
       int pend_qt = -1, pend_s = 0, pend_ab = 0, pend_item = 0;
       bool pend_first = false, pend_last = false;
       auto finish_pending = [&]() {
-        mma_commit(q_empty + pend_s);
-        if (pend_last) mma_commit(acc_full + pend_ab);
+        mma_commit_x<kW>(q_empty + pend_s);
+        if (pend_last) mma_commit_x<kW>(acc_full + pend_ab);
       };
       int qc = 0, ii = 0;
       for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
@@ -448,13 +453,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           finish_pending();
           pend_qt = -1;
         }
-        if (!(ok = mbar_wait(kv_full + kb, (ii / KVB) & 1, wctx))) break;
+        if (!(ok = mbar_wait_x<kW>(kv_full + kb, (ii / KVB) & 1, wctx))) break;
         tc_fence_after();
         const uint32_t k_base = smem_u32(smem + L::kK + kb * L::kTileBytes);
         const uint32_t v_base = smem_u32(smem + L::kV + kb * L::kTileBytes);
         for (int i = 0; i < it.n; ++i, ++qc) {
           const int s = qc % S;
-          if (!(ok = mbar_wait(q_full + s, (qc / S) & 1, wctx))) break;
+          if (!(ok = mbar_wait_x<kW>(q_full + s, (qc / S) & 1, wctx))) break;
           tc_fence_after();
           const uint32_t q_s = smem_u32(smem + L::kQ + s * L::kTileBytes);
           const uint32_t do_s = smem_u32(smem + L::kDO + s * L::kTileBytes);
@@ -467,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             if (pend_qt >= 0) finish_pending();
-            if (i == it.n - 1) mma_commit(kv_empty + kb);
+            if (i == it.n - 1) mma_commit_x<kW>(kv_empty + kb);
             pend_qt = qc;
             pend_s = s;
             pend_ab = ab;
@@ -479,10 +484,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             sdp_half(1, k_base, v_base, q_s, do_s);
             if (!(ok = acc_half(0, qc, s, ab, i == 0, ii) && acc_half(1, qc, s, ab, i == 0, ii)))
               break;
-            mma_commit(q_empty + s);
+            mma_commit_x<kW>(q_empty + s);
             if (i == it.n - 1) {
-              mma_commit(acc_full + ab);
-              mma_commit(kv_empty + kb);
+              mma_commit_x<kW>(acc_full + ab);
+              mma_commit_x<kW>(kv_empty + kb);
             }
           }
         }
@@ -763,22 +768,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // d = 64: the whole warp runs the issue loop on warp-uniform values (lane 0 waits on
+    // barriers, the result is broadcast; an elected lane issues), which shortens the issue
+    // path.  d = 128 (MMA-bound, waits in the middle of each tile) issues from lane 0.
+    constexpr bool kW = D == 64;
+    if (kW || lane == 0) {
+      constexpr uint32_t kHi = sw128_desc_hi(1024);
       constexpr uint32_t idesc_half = idesc_bf16_f32(128, 64, false);  // S / dP halves
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);     // dQ
       constexpr bool kDeferAcc = D == 64;  // as in the dK / dV kernel
       bool ok = true;
       auto acc_half = [&](int h, int t_, int s, int ab, bool first, int item) -> bool {
-        if (!mbar_wait(ds_full + h, t_ & 1, wctx)) return false;
+        if (!mbar_wait_x<kW>(ds_full + h, t_ & 1, wctx)) return false;
         if (h == 0 && first && item >= ACB &&
-            !mbar_wait(acc_empty + ab, ((item / ACB) - 1) & 1, wctx))
+            !mbar_wait_x<kW>(acc_empty + ab, ((item / ACB) - 1) & 1, wctx))
           return false;
         tc_fence_after();
         const uint32_t k_s = smem_u32(smem + L::kK + s * L::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + 256 + ab * D, tmem + 128 + 64 * h + kk * 8,
-                 smem_desc_sw128(k_s + (4 * h + kk) * 2048, L::kBoxBytes, 1024), idesc_acc,
+          mma_ts_lh_x<kW>(tmem + 256 + ab * D, tmem + 128 + 64 * h + kk * 8,
+                          sw128_desc_lo(k_s + (4 * h + kk) * 2048, L::kBoxBytes), kHi, idesc_acc,
                  (first && h == 0 && kk == 0) ? 0u : 1u);
         return true;
       };
@@ -786,22 +796,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + 64 * h, smem_desc_sw128(q_base + off, 16, 1024),
-                 smem_desc_sw128(k_s + off + h * 8192, 16, 1024), idesc_half, kk > 0);
+          mma_ss_lh_x<kW>(tmem + 64 * h, sw128_desc_lo(q_base + off, 16),
+                          sw128_desc_lo(k_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + 128 + 64 * h, smem_desc_sw128(do_base + off, 16, 1024),
-                 smem_desc_sw128(v_s + off + h * 8192, 16, 1024), idesc_half, kk > 0);
+          mma_ss_lh_x<kW>(tmem + 128 + 64 * h, sw128_desc_lo(do_base + off, 16),
+                          sw128_desc_lo(v_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
         }
-        mma_commit(s_full + h);
+        mma_commit_x<kW>(s_full + h);
       };
       int pend_t = -1, pend_s = 0, pend_ab = 0, pend_item = 0;
       bool pend_first = false, pend_last = false;
       auto finish_pending = [&]() {
-        mma_commit(kv_empty + pend_s);
-        if (pend_last) mma_commit(acc_full + pend_ab);
+        mma_commit_x<kW>(kv_empty + pend_s);
+        if (pend_last) mma_commit_x<kW>(acc_full + pend_ab);
       };
       int tk_ = 0, ii = 0;
       for (WorkIter<false> iter(p, nitems); ok && iter.valid(); iter.advance()) {
@@ -815,13 +825,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           finish_pending();
           pend_t = -1;
         }
-        if (!(ok = mbar_wait(qd_full + qb, (ii / QB) & 1, wctx))) break;
+        if (!(ok = mbar_wait_x<kW>(qd_full + qb, (ii / QB) & 1, wctx))) break;
         tc_fence_after();
         const uint32_t q_base = smem_u32(smem + L::kQ + qb * L::kTileBytes);
         const uint32_t do_base = smem_u32(smem + L::kDO + qb * L::kTileBytes);
         for (int j = 0; j < it.n; ++j, ++tk_) {
           const int s = tk_ % S;
-          if (!(ok = mbar_wait(kv_full + s, (tk_ / S) & 1, wctx))) break;
+          if (!(ok = mbar_wait_x<kW>(kv_full + s, (tk_ / S) & 1, wctx))) break;
           tc_fence_after();
           const uint32_t k_s = smem_u32(smem + L::kK + s * L::kTileBytes);
           const uint32_t v_s = smem_u32(smem + L::kV + s * L::kTileBytes);
@@ -834,7 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             if (pend_t >= 0) finish_pending();
-            if (j == it.n - 1) mma_commit(qd_empty + qb);
+            if (j == it.n - 1) mma_commit_x<kW>(qd_empty + qb);
             pend_t = tk_;
             pend_s = s;
             pend_ab = ab;
@@ -846,10 +856,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             sdp_half(1, q_base, do_base, k_s, v_s);
             if (!(ok = acc_half(0, tk_, s, ab, j == 0, ii) && acc_half(1, tk_, s, ab, j == 0, ii)))
               break;
-            mma_commit(kv_empty + s);
+            mma_commit_x<kW>(kv_empty + s);
             if (j == it.n - 1) {
-              mma_commit(acc_full + ab);
-              mma_commit(qd_empty + qb);
+              mma_commit_x<kW>(acc_full + ab);
+              mma_commit_x<kW>(qd_empty + qb);
             }
           }
         }

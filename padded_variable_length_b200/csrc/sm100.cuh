@@ -451,4 +451,29 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Issue helpers that pick the whole-warp (W = true: every lane runs the loop, lane 0
+// waits, an elected lane issues) or the single-lane form at compile time.
+template <bool W>
+__device__ __forceinline__ bool mbar_wait_x(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  if constexpr (W) return mbar_wait_w(bar, parity, w);
+  else return mbar_wait(bar, parity, w);
+}
+template <bool W>
+__device__ __forceinline__ void mma_commit_x(uint64_t* bar) {
+  if constexpr (W) mma_commit_w(bar);
+  else mma_commit(bar);
+}
+template <bool W>
+__device__ __forceinline__ void mma_ss_lh_x(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                            uint32_t hi, uint32_t idesc, uint32_t accumulate) {
+  if constexpr (W) mma_ss_lh_w(d_tmem, a_lo, b_lo, hi, idesc, accumulate);
+  else mma_ss_lh(d_tmem, a_lo, b_lo, hi, idesc, accumulate);
+}
+template <bool W>
+__device__ __forceinline__ void mma_ts_lh_x(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                            uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+  if constexpr (W) mma_ts_lh_w(d_tmem, a_tmem, b_lo, b_hi, idesc, accumulate);
+  else mma_ts_lh(d_tmem, a_tmem, b_lo, b_hi, idesc, accumulate);
+}
+
 }  // namespace sigattn
