@@ -206,14 +206,22 @@ struct WorkIter {
 
 // ---------------------------------------------------------------------------------------
 // dK / dV: one item = one k-tile column of the plan for one head; thread = key row.
-// TMEM: S^T half h [64h, 64h+64), dP^T half h [128+64h, ...), then per accumulator buffer a:
-// dV [256 + 2Da, +D), dK [256 + 2Da + D, +D).
+// d = 128 TMEM: S^T half h [64h, 64h+64), dP^T half h [128+64h, ...), dV [256, 384),
+// dK [384, 512).
+// d = 64 ("unit" schedule): a unit is one query half of one tile, u = 2 (tile) + half, and
+// warpgroup h takes the units of half h.  Three unit buffers rotate: S^T of unit u in
+// [128 (u % 3), +64), dP^T in [128 (u % 3) + 64, +64); P^T and dS^T overwrite the first 32
+// columns of each.  The MMA issuer computes S^T / dP^T of unit u right after the dV / dK
+// MMAs of unit u - 3, the last user of that buffer, so they are ready a tile and a half
+// before the epilogue needs them.  dV [384, 448), dK [448, 512) (one accumulator: the
+// epilogue reads an item's dV / dK after its first unit of the next item).
 // ---------------------------------------------------------------------------------------
 template <int D>
 struct DkvLayout {
-  static constexpr int kStages = D == 64 ? 3 : 2;   // Q / dO ring
+  static constexpr bool kUnits = D == 64;
+  static constexpr int kStages = kUnits ? 4 : 2;  // Q / dO ring
   static constexpr int kKVBufs = D == 64 ? 2 : 1;   // K / V of consecutive items
-  static constexpr int kAccBufs = D == 64 ? 2 : 1;  // dV / dK accumulators in TMEM
+  static constexpr int kAccBufs = 1;                // dV / dK accumulators in TMEM
   static constexpr int kBoxes = D / 64;
   static constexpr int kBoxBytes = 128 * 128;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
@@ -226,8 +234,10 @@ struct DkvLayout {
   static constexpr int kMetaBits = kVec + kStages * 2 * 128 * 4;
   static constexpr int kMetaKind = kMetaBits + kStages * 2048;
   static constexpr int kBar = kMetaKind + 16 * ((kStages * 4 + 15) / 16);
-  // kv_full[KV] kv_empty[KV] q_full[S] q_empty[S] s_full[2] p_full[2] acc_full[A] acc_empty[A]
-  static constexpr int kNumBars = 2 * kKVBufs + 2 * kStages + 4 + 2 * kAccBufs;
+  // kv_full[KV] kv_empty[KV] q_full[S] q_empty[S] s_full[NR] p_full[NR] acc_full[A] acc_empty[A]
+  // (NR = 4 unit slots for d = 64, one per half for d = 128)
+  static constexpr int kRing = kUnits ? 4 : 2;
+  static constexpr int kNumBars = 2 * kKVBufs + 2 * kStages + 2 * kRing + 2 * kAccBufs;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -251,9 +261,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* kv_empty = kv_full + KVB;
   uint64_t* q_full = kv_empty + KVB;
   uint64_t* q_empty = q_full + S;
-  uint64_t* s_full = q_empty + S;   // [2] per half
-  uint64_t* p_full = s_full + 2;    // [2] per half
-  uint64_t* acc_full = p_full + 2;  // [ACB]
+  constexpr int NR = L::kRing;
+  uint64_t* s_full = q_empty + S;    // [NR] per unit slot (d = 64) or per half
+  uint64_t* p_full = s_full + NR;    // [NR]
+  uint64_t* acc_full = p_full + NR;  // [ACB]
   uint64_t* acc_empty = acc_full + ACB;
   float* vec = reinterpret_cast<float*>(smem + L::kVec);
   uint32_t* meta_bits = reinterpret_cast<uint32_t*>(smem + L::kMetaBits);
@@ -272,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(q_full + i, 2);  // TMA bytes + the producer warp's column vectors
       mbar_init(q_empty + i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NR; ++i) {
       mbar_init(s_full + i, 1);
       mbar_init(p_full + i, 4);  // the four warps of one epilogue warpgroup
     }
@@ -381,6 +392,86 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = max(0, ii - KVB); u < ii; ++u) mbar_wait(kv_full + u % KVB, (u / KVB) & 1, drain);
       for (int u = max(0, qc - S); u < qc; ++u) mbar_wait(q_full + u % S, (u / S) & 1, drain);
     }
+  } else if (warp == 1 && L::kUnits) {
+    // ---------------------------------------------------------------- MMA issuer (units)
+    // The whole warp runs the issue loop on warp-uniform values; lane 0 waits on barriers
+    // (the result is broadcast) and an elected lane issues.  Unit u: S^T / dP^T of query
+    // half u % 2 of tile u / 2; issue order dV / dK of unit u - 3, then S^T / dP^T of u.
+    constexpr uint32_t kHi = sw128_desc_hi(1024);
+    constexpr uint32_t idesc_half = idesc_bf16_f32(128, 64, false);  // S^T / dP^T halves
+    constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);     // dV / dK
+    constexpr uint32_t kT = L::kTileBytes >> 4;
+    const uint32_t k_lo0 = sw128_desc_lo(smem_u32(smem + L::kK), 16);
+    const uint32_t v_lo0 = sw128_desc_lo(smem_u32(smem + L::kV), 16);
+    const uint32_t q_lo0 = sw128_desc_lo(smem_u32(smem + L::kQ), 16);
+    const uint32_t do_lo0 = sw128_desc_lo(smem_u32(smem + L::kDO), 16);
+    const uint32_t q_mn0 = sw128_desc_lo(smem_u32(smem + L::kQ), L::kBoxBytes);
+    const uint32_t do_mn0 = sw128_desc_lo(smem_u32(smem + L::kDO), L::kBoxBytes);
+    static_assert(!L::kUnits || (S == 4 && KVB == 2 && ACB == 1 && NR == 4), "unit rings");
+    // FIFO of the (up to three) units whose dV / dK MMAs are still to issue, oldest first:
+    // stage | half << 2 | first of item << 3 | last of item << 4 | item << 5
+    int f0 = 0, f1 = 0, f2 = 0;
+    bool ok = true;
+    // dV += P^T dO, dK += dS^T Q for unit x (buffer b = x % 3), once its warpgroup is done
+    auto acc = [&](int x, uint32_t b) -> bool {
+      const int info = f0;
+      f0 = f1;
+      f1 = f2;
+      const int s = info & 3, hh = (info >> 2) & 1, item = info >> 5;
+      const bool first = ((info >> 3) & 1) != 0, last = ((info >> 4) & 1) != 0;
+      if (!mbar_wait_w(p_full + (x & 3), (x >> 2) & 1, wctx)) return false;
+      if (first && item >= 1 && !mbar_wait_w(acc_empty, (item - 1) & 1, wctx)) return false;
+      tc_fence_after();
+      const uint32_t pt = tmem + b * 128;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t a = (first && kk == 0) ? 0u : 1u;
+        const uint32_t rows = (4 * hh + kk) * 128;  // query rows 64 hh + 16 kk (2 KB each)
+        mma_ts_lh_w(tmem + 384, pt + kk * 8, do_mn0 + s * kT + rows, kHi, idesc_acc, a);
+        mma_ts_lh_w(tmem + 448, pt + 64 + kk * 8, q_mn0 + s * kT + rows, kHi, idesc_acc, a);
+      }
+      if (hh == 1) mma_commit_w(q_empty + s);
+      if (last) mma_commit_w(acc_full);
+      return true;
+    };
+    int qc = 0, ii = 0, u = 0;
+    uint32_t b3 = 0;  // u % 3
+    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
+      if (it.n == 0) continue;
+      const int kb = ii & 1;
+      if (!(ok = mbar_wait_w(kv_full + kb, (ii >> 1) & 1, wctx))) break;
+      const uint32_t k_lo = k_lo0 + kb * kT, v_lo = v_lo0 + kb * kT;
+      for (int i = 0; ok && i < it.n; ++i, ++qc) {
+        const int s = qc & 3;
+        if (!(ok = mbar_wait_w(q_full + s, (qc >> 2) & 1, wctx))) break;
+        for (int hh = 0; hh < 2; ++hh, ++u) {
+          // S^T / dP^T of unit u go to the buffer of unit u - 3: its dV / dK MMAs first
+          if (u >= 3 && !(ok = acc(u - 3, b3))) break;
+          tc_fence_after();
+          const uint32_t st = tmem + b3 * 128;
+          const uint32_t qh = q_lo0 + s * kT + hh * 512, dh = do_lo0 + s * kT + hh * 512;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss_lh_w(st, k_lo + kk * 2, qh + kk * 2, kHi, idesc_half, kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss_lh_w(st + 64, v_lo + kk * 2, dh + kk * 2, kHi, idesc_half, kk > 0 ? 1u : 0u);
+          mma_commit_w(s_full + (u & 3));
+          const int info = s | (hh << 2) | ((i == 0 && hh == 0) ? 8 : 0) |
+                           ((i == it.n - 1 && hh == 1) ? 16 : 0) | (ii << 5);
+          if (u == 0) f0 = info;
+          else if (u == 1) f1 = info;
+          else f2 = info;
+          b3 = b3 == 2 ? 0 : b3 + 1;
+        }
+      }
+      if (!ok) break;
+      mma_commit_w(kv_empty + kb);  // K / V feed only S^T / dP^T
+      ++ii;
+    }
+    for (int x = max(0, u - 3); ok && x < u; ++x)
+      ok = acc(x, static_cast<uint32_t>((static_cast<int>(b3) + 3 + x - u) % 3));
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     // d = 64: the whole warp runs the issue loop on warp-uniform values (lane 0 waits on
@@ -498,6 +589,126 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc_half(1, pend_qt, pend_s, pend_ab, pend_first, pend_item))
         finish_pending();
     }
+  } else if (warp >= kEpiWarp0 && L::kUnits) {
+    // ---------------------------------------------------------------- epilogue (units)
+    const int h = (warp - kEpiWarp0) >> 2;  // query half of every tile
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;  // key row of the tile
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float c1s = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
+    const float2 c1 = make_float2(c1s, c1s);
+    constexpr int kOc = D / 2;  // dV / dK columns written by this warpgroup
+    bool ok = true;
+    // dV / dK of the last item with tiles, written out after the first unit of the next
+    bool pend = false;
+    WorkRef pit{};
+    int pi = 0;
+    auto flush = [&]() {
+      pend = false;
+      ok = ok && mbar_wait(acc_full, pi & 1, wctx);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) return;
+      tc_fence_after();
+      uint32_t pv[kOc / 2], pkk[kOc / 2];
+      {
+        uint32_t acc[32];
+        tmem_ld32(t_lane + 384 + h * kOc, acc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pv[c] = pack_bf16x2(__uint_as_float(acc[2 * c]), __uint_as_float(acc[2 * c + 1]));
+        tmem_ld32(t_lane + 448 + h * kOc, acc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pkk[c] = pack_bf16x2(__uint_as_float(acc[2 * c]) * p.scale,
+                               __uint_as_float(acc[2 * c + 1]) * p.scale);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      const int kg = pit.t * kTile + row;
+      if (kg < p.Nk) {
+        uint4* dvp = reinterpret_cast<uint4*>(p.dv + pit.b * p.dv_sb +
+                                              static_cast<int64_t>(kg) * p.dv_sn + pit.h * p.dv_sh +
+                                              h * kOc);
+        uint4* dkp = reinterpret_cast<uint4*>(p.dk + pit.b * p.dk_sb +
+                                              static_cast<int64_t>(kg) * p.dk_sn + pit.h * p.dk_sh +
+                                              h * kOc);
+#pragma unroll
+        for (int c = 0; c < kOc / 8; ++c) {
+          dvp[c] = make_uint4(pv[4 * c], pv[4 * c + 1], pv[4 * c + 2], pv[4 * c + 3]);
+          dkp[c] = make_uint4(pkk[4 * c], pkk[4 * c + 1], pkk[4 * c + 2], pkk[4 * c + 3]);
+        }
+      }
+    };
+    int qc = 0, ii = 0;
+    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
+      if (it.n == 0) {
+        // No query attends to this k-tile: dK = dV = 0 on its rows.
+        if (pend) flush();
+        const int rows = min(kTile, p.Nk - it.t * kTile);
+        const int tid = threadIdx.x - kEpiWarp0 * 32;
+        zero_rows<D>(p.dk + it.b * p.dk_sb + static_cast<int64_t>(it.t * kTile) * p.dk_sn +
+                         it.h * p.dk_sh, p.dk_sn, rows, tid, 256);
+        zero_rows<D>(p.dv + it.b * p.dv_sb + static_cast<int64_t>(it.t * kTile) * p.dv_sn +
+                         it.h * p.dv_sh, p.dv_sn, rows, tid, 256);
+        continue;
+      }
+      for (int i = 0; i < it.n; ++i, ++qc) {
+        const int s = qc & 3, u = 2 * qc + h;
+        // q_full of the stage also publishes the kind, bitmask and column vectors
+        if (ok) ok = mbar_wait(q_full + s, (qc >> 2) & 1, wctx);
+        if (ok) ok = mbar_wait(s_full + (u & 3), (u >> 2) & 1, wctx);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+        if (meta_kind[s] == 2)
+          mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
+        const float* vs = vec + s * 256 + 64 * h;
+        const uint32_t base = t_lane + (u % 3) * 128;
+        uint32_t sr[2][32], dpr[2][32];
+        tmem_ld32(base, sr[0]);
+        tmem_ld32(base + 64, dpr[0]);
+        tmem_wait_ld();
+        tmem_ld32(base + 32, sr[1]);
+        tmem_ld32(base + 96, dpr[1]);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (c == 1) tmem_wait_ld();
+          const uint32_t mw = c ? mb.y : mb.x;
+          uint32_t pk[16], dk[16];
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            float2 pw, ds;
+            const float2 off2 = *reinterpret_cast<const float2*>(vs + 32 * c + cc);
+            const float2 D2 = EPI == 0 ? make_float2(0.0f, 0.0f)
+                                       : *reinterpret_cast<const float2*>(vs + 128 + 32 * c + cc);
+            weight_grad2<EPI>(
+                make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
+                make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])), c1, off2,
+                D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
+            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
+            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+          }
+          tmem_st16(base + 16 * c, pk);
+          tmem_st16(base + 64 + 16 * c, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + (u & 3));
+        if (pend) flush();
+      }
+      if (!ok) break;
+      pend = true;
+      pit = it;
+      pi = ii;
+      ++ii;
+    }
+    if (ok && pend) flush();
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- epilogue
     const int h = (warp - kEpiWarp0) >> 2;  // query half of every tile
@@ -619,11 +830,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------------------------------
 // dQ: one item = one q-tile row of the plan for one head; thread = query row.
-// TMEM: S half h [64h, 64h+64), dP half h [128+64h, ...), dQ buffer a [256 + Da, +D).
+// d = 128 TMEM: S half h [64h, 64h+64), dP half h [128+64h, ...), dQ [256, 384).
+// d = 64: the unit schedule of the dK / dV kernel, with units = key halves of a tile:
+// S of unit u in [128 (u % 3), +64), dP in [128 (u % 3) + 64, +64) (dS overwrites its
+// first 32 columns); dQ buffer a in [384 + 64a, +64).
 // ---------------------------------------------------------------------------------------
 template <int D>
 struct DqLayout {
-  static constexpr int kStages = D == 64 ? 3 : 2;   // K / V ring
+  static constexpr bool kUnits = D == 64;
+  static constexpr int kStages = kUnits ? 4 : 2;    // K / V ring
   static constexpr int kQBufs = D == 64 ? 2 : 1;    // Q / dO of consecutive items
   static constexpr int kAccBufs = D == 64 ? 2 : 1;  // dQ accumulators in TMEM
   static constexpr int kBoxes = D / 64;
@@ -637,8 +852,10 @@ struct DqLayout {
   static constexpr int kMetaBits = kV + kStages * kTileBytes;
   static constexpr int kMetaKind = kMetaBits + kStages * 2048;
   static constexpr int kBar = kMetaKind + 16 * ((kStages * 4 + 15) / 16);
-  // qd_full[QB] qd_empty[QB] kv_full[S] kv_empty[S] s_full[2] ds_full[2] acc_full[A] acc_empty[A]
-  static constexpr int kNumBars = 2 * kQBufs + 2 * kStages + 4 + 2 * kAccBufs;
+  // qd_full[QB] qd_empty[QB] kv_full[S] kv_empty[S] s_full[NR] ds_full[NR] acc_full[A]
+  // acc_empty[A] (NR = 4 unit slots for d = 64, one per half for d = 128)
+  static constexpr int kRing = kUnits ? 4 : 2;
+  static constexpr int kNumBars = 2 * kQBufs + 2 * kStages + 2 * kRing + 2 * kAccBufs;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -662,9 +879,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* qd_empty = qd_full + QB;
   uint64_t* kv_full = qd_empty + QB;
   uint64_t* kv_empty = kv_full + S;
-  uint64_t* s_full = kv_empty + S;   // [2] per half
-  uint64_t* ds_full = s_full + 2;    // [2] per half
-  uint64_t* acc_full = ds_full + 2;  // [ACB]
+  constexpr int NR = L::kRing;
+  uint64_t* s_full = kv_empty + S;    // [NR] per unit slot (d = 64) or per half
+  uint64_t* ds_full = s_full + NR;    // [NR]
+  uint64_t* acc_full = ds_full + NR;  // [ACB]
   uint64_t* acc_empty = acc_full + ACB;
   uint32_t* meta_bits = reinterpret_cast<uint32_t*>(smem + L::kMetaBits);
   int* meta_kind = reinterpret_cast<int*>(smem + L::kMetaKind);
@@ -682,7 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(kv_full + i, 1);
       mbar_init(kv_empty + i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NR; ++i) {
       mbar_init(s_full + i, 1);
       mbar_init(ds_full + i, 4);
     }
@@ -766,6 +984,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = max(0, ii - QB); u < ii; ++u) mbar_wait(qd_full + u % QB, (u / QB) & 1, drain);
       for (int u = max(0, tk_ - S); u < tk_; ++u) mbar_wait(kv_full + u % S, (u / S) & 1, drain);
     }
+  } else if (warp == 1 && L::kUnits) {
+    // ---------------------------------------------------------------- MMA issuer (units)
+    // As in the dK / dV kernel: whole-warp issue; unit u = key half u % 2 of k-tile u / 2;
+    // dQ MMAs of unit u - 3, then S / dP of unit u.
+    constexpr uint32_t kHi = sw128_desc_hi(1024);
+    constexpr uint32_t idesc_half = idesc_bf16_f32(128, 64, false);  // S / dP halves
+    constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);     // dQ
+    constexpr uint32_t kT = L::kTileBytes >> 4;
+    const uint32_t q_lo0 = sw128_desc_lo(smem_u32(smem + L::kQ), 16);
+    const uint32_t do_lo0 = sw128_desc_lo(smem_u32(smem + L::kDO), 16);
+    const uint32_t k_lo0 = sw128_desc_lo(smem_u32(smem + L::kK), 16);
+    const uint32_t v_lo0 = sw128_desc_lo(smem_u32(smem + L::kV), 16);
+    const uint32_t k_mn0 = sw128_desc_lo(smem_u32(smem + L::kK), L::kBoxBytes);
+    static_assert(!L::kUnits || (S == 4 && QB == 2 && ACB == 2 && NR == 4), "unit rings");
+    // FIFO of the (up to three) units whose dQ MMAs are still to issue, oldest first:
+    // stage | half << 2 | first of item << 3 | last of item << 4 | item << 5
+    int f0 = 0, f1 = 0, f2 = 0;
+    bool ok = true;
+    // dQ += dS K for unit x (buffer b = x % 3), once its warpgroup is done
+    auto acc = [&](int x, uint32_t b) -> bool {
+      const int info = f0;
+      f0 = f1;
+      f1 = f2;
+      const int s = info & 3, hh = (info >> 2) & 1, item = info >> 5, ab = item & 1;
+      const bool first = ((info >> 3) & 1) != 0, last = ((info >> 4) & 1) != 0;
+      if (!mbar_wait_w(ds_full + (x & 3), (x >> 2) & 1, wctx)) return false;
+      if (first && item >= 2 && !mbar_wait_w(acc_empty + ab, ((item >> 1) - 1) & 1, wctx))
+        return false;
+      tc_fence_after();
+      const uint32_t pt = tmem + b * 128 + 64;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts_lh_w(tmem + 384 + ab * D, pt + kk * 8, k_mn0 + s * kT + (4 * hh + kk) * 128, kHi,
+                    idesc_acc, (first && kk == 0) ? 0u : 1u);
+      if (hh == 1) mma_commit_w(kv_empty + s);
+      if (last) mma_commit_w(acc_full + ab);
+      return true;
+    };
+    int tc = 0, ii = 0, u = 0;
+    uint32_t b3 = 0;  // u % 3
+    for (WorkIter<false> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
+      if (it.n == 0) continue;
+      const int qb = ii & 1;
+      if (!(ok = mbar_wait_w(qd_full + qb, (ii >> 1) & 1, wctx))) break;
+      const uint32_t q_lo = q_lo0 + qb * kT, do_lo = do_lo0 + qb * kT;
+      for (int j = 0; ok && j < it.n; ++j, ++tc) {
+        const int s = tc & 3;
+        if (!(ok = mbar_wait_w(kv_full + s, (tc >> 2) & 1, wctx))) break;
+        for (int hh = 0; hh < 2; ++hh, ++u) {
+          // S / dP of unit u go to the buffer of unit u - 3: its dQ MMAs first
+          if (u >= 3 && !(ok = acc(u - 3, b3))) break;
+          tc_fence_after();
+          const uint32_t st = tmem + b3 * 128;
+          const uint32_t kh = k_lo0 + s * kT + hh * 512, vh = v_lo0 + s * kT + hh * 512;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss_lh_w(st, q_lo + kk * 2, kh + kk * 2, kHi, idesc_half, kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss_lh_w(st + 64, do_lo + kk * 2, vh + kk * 2, kHi, idesc_half, kk > 0 ? 1u : 0u);
+          mma_commit_w(s_full + (u & 3));
+          const int info = s | (hh << 2) | ((j == 0 && hh == 0) ? 8 : 0) |
+                           ((j == it.n - 1 && hh == 1) ? 16 : 0) | (ii << 5);
+          if (u == 0) f0 = info;
+          else if (u == 1) f1 = info;
+          else f2 = info;
+          b3 = b3 == 2 ? 0 : b3 + 1;
+        }
+      }
+      if (!ok) break;
+      mma_commit_w(qd_empty + qb);  // Q / dO feed only S / dP
+      ++ii;
+    }
+    for (int x = max(0, u - 3); ok && x < u; ++x)
+      ok = acc(x, static_cast<uint32_t>((static_cast<int>(b3) + 3 + x - u) % 3));
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     // d = 64: the whole warp runs the issue loop on warp-uniform values (lane 0 waits on
@@ -870,6 +1164,123 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc_half(1, pend_t, pend_s, pend_ab, pend_first, pend_item))
         finish_pending();
     }
+  } else if (warp >= kEpiWarp0 && L::kUnits) {
+    // ---------------------------------------------------------------- epilogue (units)
+    const int h = (warp - kEpiWarp0) >> 2;  // key half of every tile
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float c1s = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
+    const float2 c1 = make_float2(c1s, c1s);
+    constexpr int kOc = D / 2;  // dQ columns written by this warpgroup
+    bool ok = true;
+    // dQ of the last item with tiles, written out after the first unit of the next item
+    bool pend = false;
+    WorkRef pit{};
+    int pi = 0;
+    auto flush = [&]() {
+      pend = false;
+      const int ab = pi & 1;
+      ok = ok && mbar_wait(acc_full + ab, (pi >> 1) & 1, wctx);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) return;
+      tc_fence_after();
+      uint32_t pk[kOc / 2];
+      {
+        uint32_t acc[32];
+        tmem_ld32(t_lane + 384 + ab * D + h * kOc, acc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pk[c] = pack_bf16x2(__uint_as_float(acc[2 * c]) * p.scale,
+                              __uint_as_float(acc[2 * c + 1]) * p.scale);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + ab);
+      const int qg = pit.t * kTile + row;
+      if (qg < p.Nq) {
+        uint4* dqp = reinterpret_cast<uint4*>(p.dq + pit.b * p.dq_sb +
+                                              static_cast<int64_t>(qg) * p.dq_sn + pit.h * p.dq_sh +
+                                              h * kOc);
+#pragma unroll
+        for (int c = 0; c < kOc / 8; ++c)
+          dqp[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+    };
+    int tc = 0, ii = 0;
+    WorkIter<false> iter(p, nitems);
+    float off_cur = 0.0f, D_cur = 0.0f;
+    if (iter.valid()) {
+      off_cur = row_offset<EPI>(p, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
+      D_cur = row_D<EPI>(p, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
+    }
+    for (; ok && iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
+      // the next item's row values, in flight while this one is processed
+      float off_nxt = 0.0f, D_nxt = 0.0f;
+      if (iter.w + static_cast<int>(gridDim.x) < nitems && iter.nxt.n > 0) {
+        off_nxt = row_offset<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
+        D_nxt = row_D<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
+      }
+      const float off = off_cur, Drow = D_cur;
+      off_cur = off_nxt;
+      D_cur = D_nxt;
+      if (it.n == 0) {
+        if (pend) flush();
+        const int rows = min(kTile, p.Nq - it.t * kTile);
+        zero_rows<D>(p.dq + it.b * p.dq_sb + static_cast<int64_t>(it.t * kTile) * p.dq_sn +
+                         it.h * p.dq_sh, p.dq_sn, rows, threadIdx.x - kEpiWarp0 * 32, 256);
+        continue;
+      }
+      const float2 off2 = make_float2(off, off), D2 = make_float2(Drow, Drow);
+      for (int j = 0; j < it.n; ++j, ++tc) {
+        const int s = tc & 3, u = 2 * tc + h;
+        // kv_full of the stage also publishes the kind and bitmask the producer staged
+        if (ok) ok = mbar_wait(kv_full + s, (tc >> 2) & 1, wctx);
+        if (ok) ok = mbar_wait(s_full + (u & 3), (u >> 2) & 1, wctx);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+        if (meta_kind[s] == 2)
+          mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
+        const uint32_t base = t_lane + (u % 3) * 128;
+        uint32_t sr[2][32], dpr[2][32];
+        tmem_ld32(base, sr[0]);
+        tmem_ld32(base + 64, dpr[0]);
+        tmem_wait_ld();
+        tmem_ld32(base + 32, sr[1]);
+        tmem_ld32(base + 96, dpr[1]);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (c == 1) tmem_wait_ld();
+          const uint32_t mw = c ? mb.y : mb.x;
+          uint32_t dk[16];
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            float2 pw, ds;
+            weight_grad2<EPI>(
+                make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
+                make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])), c1, off2,
+                D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
+            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+          }
+          tmem_st16(base + 64 + 16 * c, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_full + (u & 3));
+        if (pend) flush();
+      }
+      if (!ok) break;
+      pend = true;
+      pit = it;
+      pi = ii;
+      ++ii;
+    }
+    if (ok && pend) flush();
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- epilogue
     const int h = (warp - kEpiWarp0) >> 2;  // key half of every tile
