@@ -383,13 +383,12 @@ __device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
       : "memory");
 }
 
-// Bounded wait for a whole warp: lane 0 waits, the result is shared with the warp.
+// Bounded wait for a whole converged warp: every lane runs the same wait loop.  try_wait,
+// the cycle counter and the abort flag are read by one instruction for the whole warp, so
+// the lanes see the same values and leave the loop together; no lane-0 branch, shuffle or
+// reconvergence sits on the issue path.
 __device__ __forceinline__ bool mbar_wait_w(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
-  bool ok = true;
-  if (lane_id() == 0) ok = mbar_wait(bar, parity, w);
-  ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-  __syncwarp();
-  return ok;
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, w));
 }
 
 // ------------------------------------------------------------------------------------
