@@ -150,12 +150,11 @@ __global__ void d_preprocess_kernel(const __nv_bfloat16* __restrict__ o, int64_t
 // Shared pieces of the two gradient kernels.
 //
 // Both are persistent (one CTA per SM, static stride over the plan's longest-first work
-// list) and split every 128 x 128 tile into two column halves: epilogue warpgroup h owns
-// half h, with its own "S ready" and "P ready" barriers.  The MMA thread interleaves the
-// halves: the accumulating MMAs of half h of the previous tile, then S / dP of half h of
-// the current tile.  While one warpgroup recomputes the weights of its half, the tensor
-// pipe works on the other half, and the two warpgroups' latencies interleave instead of
-// coinciding.
+// list) and split every 128 x 128 tile into two halves along the walked axis: epilogue
+// warpgroup h owns half h.  d = 64 runs the "unit" schedule (three rotating TMEM buffers,
+// the MMAs of a half-tile issued three halves ahead, see the dK / dV layout); d = 128 keeps
+// one buffer per half and interleaves the halves.  The MMA issuer is a whole warp issuing
+// from warp-uniform values.
 // ---------------------------------------------------------------------------------------
 struct WorkRef {
   int b, t, h, e0, n;  // batch, tile index on the item's own axis, head, list range
@@ -473,27 +472,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = max(0, u - 3); ok && x < u; ++x)
       ok = acc(x, static_cast<uint32_t>((static_cast<int>(b3) + 3 + x - u) % 3));
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    // d = 64: the whole warp runs the issue loop on warp-uniform values (lane 0 waits on
-    // barriers, the result is broadcast; an elected lane issues), which shortens the issue
-    // path.  d = 128 (MMA-bound, waits in the middle of each tile) issues from lane 0.
-    constexpr bool kW = D == 64;
-    if (kW || lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer (d = 128)
+    // Whole-warp issue (see the unit schedule).  Per q-tile: S^T / dP^T of both halves, then
+    // the dV / dK MMAs of half 0 and half 1 once the matching epilogue warpgroup is done,
+    // which frees the tile's Q / dO stage one tile earlier and keeps the next loads ahead
+    // of the MMAs.
+    {
       constexpr uint32_t kHi = sw128_desc_hi(1024);
       constexpr uint32_t idesc_half = idesc_bf16_f32(128, 64, false);  // S^T / dP^T halves
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);     // dV / dK
-      // d = 64 (three Q / dO stages): the dV / dK MMAs of half h of a tile are issued just
-      // before the S^T / dP^T of half h of the next tile, so the tensor pipe moves on to the
-      // next tile while the other warpgroup still works.  d = 128 (two stages, MMA-bound):
-      // a tile's accumulating MMAs follow its own S^T / dP^T, which frees its Q / dO stage
-      // one tile earlier and keeps the next loads ahead of the MMAs.
-      constexpr bool kDeferAcc = D == 64;
       bool ok = true;
       // accumulating MMAs of half h of the q-tile with global index qt_, stage s, buffer ab
       auto acc_half = [&](int h, int qt_, int s, int ab, bool first, int item) -> bool {
-        if (!mbar_wait_x<kW>(p_full + h, qt_ & 1, wctx)) return false;
+        if (!mbar_wait_w(p_full + h, qt_ & 1, wctx)) return false;
         if (h == 0 && first && item >= ACB &&
-            !mbar_wait_x<kW>(acc_empty + ab, ((item / ACB) - 1) & 1, wctx))
+            !mbar_wait_w(acc_empty + ab, ((item / ACB) - 1) & 1, wctx))
           return false;
         tc_fence_after();
         const uint32_t q_s = smem_u32(smem + L::kQ + s * L::kTileBytes);
@@ -503,10 +496,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 4; ++kk) {
           const uint32_t acc = (first && h == 0 && kk == 0) ? 0u : 1u;
           const uint32_t boff = (4 * h + kk) * 2048;  // query rows 64h + 16kk
-          mma_ts_lh_x<kW>(t_dv, tmem + 64 * h + kk * 8, sw128_desc_lo(do_s + boff, L::kBoxBytes),
-                          kHi, idesc_acc, acc);
-          mma_ts_lh_x<kW>(t_dk, tmem + 128 + 64 * h + kk * 8,
-                          sw128_desc_lo(q_s + boff, L::kBoxBytes), kHi, idesc_acc, acc);
+          mma_ts_lh_w(t_dv, tmem + 64 * h + kk * 8, sw128_desc_lo(do_s + boff, L::kBoxBytes),
+                      kHi, idesc_acc, acc);
+          mma_ts_lh_w(t_dk, tmem + 128 + 64 * h + kk * 8, sw128_desc_lo(q_s + boff, L::kBoxBytes),
+                      kHi, idesc_acc, acc);
         }
         return true;
       };
@@ -514,80 +507,44 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          mma_ss_lh_x<kW>(tmem + 64 * h, sw128_desc_lo(k_base + off, 16),
-                          sw128_desc_lo(q_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
+          mma_ss_lh_w(tmem + 64 * h, sw128_desc_lo(k_base + off, 16),
+                      sw128_desc_lo(q_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          mma_ss_lh_x<kW>(tmem + 128 + 64 * h, sw128_desc_lo(v_base + off, 16),
-                          sw128_desc_lo(do_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
+          mma_ss_lh_w(tmem + 128 + 64 * h, sw128_desc_lo(v_base + off, 16),
+                      sw128_desc_lo(do_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
         }
-        mma_commit_x<kW>(s_full + h);
-      };
-      // the q-tile whose accumulating MMAs are deferred (kDeferAcc)
-      int pend_qt = -1, pend_s = 0, pend_ab = 0, pend_item = 0;
-      bool pend_first = false, pend_last = false;
-      auto finish_pending = [&]() {
-        mma_commit_x<kW>(q_empty + pend_s);
-        if (pend_last) mma_commit_x<kW>(acc_full + pend_ab);
+        mma_commit_w(s_full + h);
       };
       int qc = 0, ii = 0;
       for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
         const WorkRef it = iter.cur;
         if (it.n == 0) continue;
         const int kb = ii % KVB, ab = ii % ACB;
-        if (kDeferAcc && pend_qt >= 0) {  // previous item's last tile, before new K / V
-          if (!(ok = acc_half(0, pend_qt, pend_s, pend_ab, pend_first, pend_item) &&
-                     acc_half(1, pend_qt, pend_s, pend_ab, pend_first, pend_item)))
-            break;
-          finish_pending();
-          pend_qt = -1;
-        }
-        if (!(ok = mbar_wait_x<kW>(kv_full + kb, (ii / KVB) & 1, wctx))) break;
+        if (!(ok = mbar_wait_w(kv_full + kb, (ii / KVB) & 1, wctx))) break;
         tc_fence_after();
         const uint32_t k_base = smem_u32(smem + L::kK + kb * L::kTileBytes);
         const uint32_t v_base = smem_u32(smem + L::kV + kb * L::kTileBytes);
         for (int i = 0; i < it.n; ++i, ++qc) {
           const int s = qc % S;
-          if (!(ok = mbar_wait_x<kW>(q_full + s, (qc / S) & 1, wctx))) break;
+          if (!(ok = mbar_wait_w(q_full + s, (qc / S) & 1, wctx))) break;
           tc_fence_after();
           const uint32_t q_s = smem_u32(smem + L::kQ + s * L::kTileBytes);
           const uint32_t do_s = smem_u32(smem + L::kDO + s * L::kTileBytes);
-          if (kDeferAcc) {
-            for (int h = 0; h < 2 && ok; ++h) {
-              if (pend_qt >= 0 &&
-                  !(ok = acc_half(h, pend_qt, pend_s, pend_ab, pend_first, pend_item)))
-                break;
-              sdp_half(h, k_base, v_base, q_s, do_s);
-            }
-            if (!ok) break;
-            if (pend_qt >= 0) finish_pending();
-            if (i == it.n - 1) mma_commit_x<kW>(kv_empty + kb);
-            pend_qt = qc;
-            pend_s = s;
-            pend_ab = ab;
-            pend_item = ii;
-            pend_first = i == 0;
-            pend_last = i == it.n - 1;
-          } else {
-            sdp_half(0, k_base, v_base, q_s, do_s);
-            sdp_half(1, k_base, v_base, q_s, do_s);
-            if (!(ok = acc_half(0, qc, s, ab, i == 0, ii) && acc_half(1, qc, s, ab, i == 0, ii)))
-              break;
-            mma_commit_x<kW>(q_empty + s);
-            if (i == it.n - 1) {
-              mma_commit_x<kW>(acc_full + ab);
-              mma_commit_x<kW>(kv_empty + kb);
-            }
+          sdp_half(0, k_base, v_base, q_s, do_s);
+          sdp_half(1, k_base, v_base, q_s, do_s);
+          if (!(ok = acc_half(0, qc, s, ab, i == 0, ii) && acc_half(1, qc, s, ab, i == 0, ii)))
+            break;
+          mma_commit_w(q_empty + s);
+          if (i == it.n - 1) {
+            mma_commit_w(acc_full + ab);
+            mma_commit_w(kv_empty + kb);
           }
         }
         ++ii;
       }
-      if (kDeferAcc && ok && pend_qt >= 0 &&
-          acc_half(0, pend_qt, pend_s, pend_ab, pend_first, pend_item) &&
-          acc_half(1, pend_qt, pend_s, pend_ab, pend_first, pend_item))
-        finish_pending();
     }
   } else if (warp >= kEpiWarp0 && L::kUnits) {
     // ---------------------------------------------------------------- epilogue (units)
@@ -1061,108 +1018,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = max(0, u - 3); ok && x < u; ++x)
       ok = acc(x, static_cast<uint32_t>((static_cast<int>(b3) + 3 + x - u) % 3));
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    // d = 64: the whole warp runs the issue loop on warp-uniform values (lane 0 waits on
-    // barriers, the result is broadcast; an elected lane issues), which shortens the issue
-    // path.  d = 128 (MMA-bound, waits in the middle of each tile) issues from lane 0.
-    constexpr bool kW = D == 64;
-    if (kW || lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer (d = 128)
+    // Whole-warp issue; per k-tile: S / dP of both halves, then the dQ MMAs of each half
+    // once the matching epilogue warpgroup is done.
+    {
       constexpr uint32_t kHi = sw128_desc_hi(1024);
       constexpr uint32_t idesc_half = idesc_bf16_f32(128, 64, false);  // S / dP halves
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);     // dQ
-      constexpr bool kDeferAcc = D == 64;  // as in the dK / dV kernel
       bool ok = true;
       auto acc_half = [&](int h, int t_, int s, int ab, bool first, int item) -> bool {
-        if (!mbar_wait_x<kW>(ds_full + h, t_ & 1, wctx)) return false;
+        if (!mbar_wait_w(ds_full + h, t_ & 1, wctx)) return false;
         if (h == 0 && first && item >= ACB &&
-            !mbar_wait_x<kW>(acc_empty + ab, ((item / ACB) - 1) & 1, wctx))
+            !mbar_wait_w(acc_empty + ab, ((item / ACB) - 1) & 1, wctx))
           return false;
         tc_fence_after();
         const uint32_t k_s = smem_u32(smem + L::kK + s * L::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts_lh_x<kW>(tmem + 256 + ab * D, tmem + 128 + 64 * h + kk * 8,
-                          sw128_desc_lo(k_s + (4 * h + kk) * 2048, L::kBoxBytes), kHi, idesc_acc,
-                 (first && h == 0 && kk == 0) ? 0u : 1u);
+          mma_ts_lh_w(tmem + 256 + ab * D, tmem + 128 + 64 * h + kk * 8,
+                      sw128_desc_lo(k_s + (4 * h + kk) * 2048, L::kBoxBytes), kHi, idesc_acc,
+                      (first && h == 0 && kk == 0) ? 0u : 1u);
         return true;
       };
       auto sdp_half = [&](int h, uint32_t q_base, uint32_t do_base, uint32_t k_s, uint32_t v_s) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          mma_ss_lh_x<kW>(tmem + 64 * h, sw128_desc_lo(q_base + off, 16),
-                          sw128_desc_lo(k_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
+          mma_ss_lh_w(tmem + 64 * h, sw128_desc_lo(q_base + off, 16),
+                      sw128_desc_lo(k_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          mma_ss_lh_x<kW>(tmem + 128 + 64 * h, sw128_desc_lo(do_base + off, 16),
-                          sw128_desc_lo(v_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
+          mma_ss_lh_w(tmem + 128 + 64 * h, sw128_desc_lo(do_base + off, 16),
+                      sw128_desc_lo(v_s + off + h * 8192, 16), kHi, idesc_half, kk > 0);
         }
-        mma_commit_x<kW>(s_full + h);
-      };
-      int pend_t = -1, pend_s = 0, pend_ab = 0, pend_item = 0;
-      bool pend_first = false, pend_last = false;
-      auto finish_pending = [&]() {
-        mma_commit_x<kW>(kv_empty + pend_s);
-        if (pend_last) mma_commit_x<kW>(acc_full + pend_ab);
+        mma_commit_w(s_full + h);
       };
       int tk_ = 0, ii = 0;
       for (WorkIter<false> iter(p, nitems); ok && iter.valid(); iter.advance()) {
         const WorkRef it = iter.cur;
         if (it.n == 0) continue;
         const int qb = ii % QB, ab = ii % ACB;
-        if (kDeferAcc && pend_t >= 0) {
-          if (!(ok = acc_half(0, pend_t, pend_s, pend_ab, pend_first, pend_item) &&
-                     acc_half(1, pend_t, pend_s, pend_ab, pend_first, pend_item)))
-            break;
-          finish_pending();
-          pend_t = -1;
-        }
-        if (!(ok = mbar_wait_x<kW>(qd_full + qb, (ii / QB) & 1, wctx))) break;
+        if (!(ok = mbar_wait_w(qd_full + qb, (ii / QB) & 1, wctx))) break;
         tc_fence_after();
         const uint32_t q_base = smem_u32(smem + L::kQ + qb * L::kTileBytes);
         const uint32_t do_base = smem_u32(smem + L::kDO + qb * L::kTileBytes);
         for (int j = 0; j < it.n; ++j, ++tk_) {
           const int s = tk_ % S;
-          if (!(ok = mbar_wait_x<kW>(kv_full + s, (tk_ / S) & 1, wctx))) break;
+          if (!(ok = mbar_wait_w(kv_full + s, (tk_ / S) & 1, wctx))) break;
           tc_fence_after();
           const uint32_t k_s = smem_u32(smem + L::kK + s * L::kTileBytes);
           const uint32_t v_s = smem_u32(smem + L::kV + s * L::kTileBytes);
-          if (kDeferAcc) {
-            for (int h = 0; h < 2 && ok; ++h) {
-              if (pend_t >= 0 &&
-                  !(ok = acc_half(h, pend_t, pend_s, pend_ab, pend_first, pend_item)))
-                break;
-              sdp_half(h, q_base, do_base, k_s, v_s);
-            }
-            if (!ok) break;
-            if (pend_t >= 0) finish_pending();
-            if (j == it.n - 1) mma_commit_x<kW>(qd_empty + qb);
-            pend_t = tk_;
-            pend_s = s;
-            pend_ab = ab;
-            pend_item = ii;
-            pend_first = j == 0;
-            pend_last = j == it.n - 1;
-          } else {
-            sdp_half(0, q_base, do_base, k_s, v_s);
-            sdp_half(1, q_base, do_base, k_s, v_s);
-            if (!(ok = acc_half(0, tk_, s, ab, j == 0, ii) && acc_half(1, tk_, s, ab, j == 0, ii)))
-              break;
-            mma_commit_x<kW>(kv_empty + s);
-            if (j == it.n - 1) {
-              mma_commit_x<kW>(acc_full + ab);
-              mma_commit_x<kW>(qd_empty + qb);
-            }
+          sdp_half(0, q_base, do_base, k_s, v_s);
+          sdp_half(1, q_base, do_base, k_s, v_s);
+          if (!(ok = acc_half(0, tk_, s, ab, j == 0, ii) && acc_half(1, tk_, s, ab, j == 0, ii)))
+            break;
+          mma_commit_w(kv_empty + s);
+          if (j == it.n - 1) {
+            mma_commit_w(acc_full + ab);
+            mma_commit_w(qd_empty + qb);
           }
         }
         ++ii;
       }
-      if (kDeferAcc && ok && pend_t >= 0 &&
-          acc_half(0, pend_t, pend_s, pend_ab, pend_first, pend_item) &&
-          acc_half(1, pend_t, pend_s, pend_ab, pend_first, pend_item))
-        finish_pending();
     }
   } else if (warp >= kEpiWarp0 && L::kUnits) {
     // ---------------------------------------------------------------- epilogue (units)

@@ -258,32 +258,10 @@ __device__ __forceinline__ uint32_t sw128_desc_lo(uint32_t saddr, uint32_t lbo_b
   return ((saddr & 0x3FFFF) >> 4) | (((lbo_bytes >> 4) & 0x3FFF) << 16);
 }
 
-// mma_ss / mma_ts with the descriptors given as (lo, hi) halves sharing one hi word.
-__device__ __forceinline__ void mma_ss_lh(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
-                                          uint32_t hi, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-      "mov.b64 da, {%1, %3};\n\tmov.b64 db, {%2, %3};\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_ts_lh(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
-                                          uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
-      "mov.b64 db, {%2, %3};\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Whole-warp forms of mma_ss_lh / mma_ts_lh: every lane runs the issue loop with the same
-// (warp-uniform) operands, one lane elected by elect.sync issues.  Issuing from uniform
-// values is markedly cheaper than from one lane's registers.
+// MMAs with the descriptors given as (lo, hi) halves sharing one hi word, issued by a whole
+// warp: every lane runs the issue loop with the same (warp-uniform) operands and one lane
+// elected by elect.sync issues.  Issuing from uniform values is markedly cheaper than from
+// one lane's registers (12 MMAs + commit: 408 instead of 686 cycles, measured on B200).
 __device__ __forceinline__ void mma_ss_lh_w(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
                                             uint32_t hi, uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -315,66 +293,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
 }
 
 // ------------------------------------------------------------------------------------
-// Warp-wide issue: the whole warp runs the role's loop with warp-uniform values (so the
-// compiler keeps the operands in uniform registers) and elect.sync picks one lane (the
-// lowest, always the same one) to issue each asynchronous instruction.
+// Whole-warp forms of commit and wait (see mma_ss_lh_w)
 // ------------------------------------------------------------------------------------
-__device__ __forceinline__ void tma_load_4d_w(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
-                                              int x, int y, int z, int w) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-      "@e cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];\n\t}" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void bulk_load_w(void* smem_dst, const void* gsrc, uint32_t bytes,
-                                            uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-      "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      "\n\t}" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx_w(uint64_t* bar, uint32_t bytes) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-      "@e mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(
-          smem_u32(bar)),
-      "r"(bytes)
-      : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_w(uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-      "@e mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n\t}" ::"r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 __device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
@@ -448,31 +368,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
-}
-
-// Issue helpers that pick the whole-warp (W = true: every lane runs the loop, lane 0
-// waits, an elected lane issues) or the single-lane form at compile time.
-template <bool W>
-__device__ __forceinline__ bool mbar_wait_x(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
-  if constexpr (W) return mbar_wait_w(bar, parity, w);
-  else return mbar_wait(bar, parity, w);
-}
-template <bool W>
-__device__ __forceinline__ void mma_commit_x(uint64_t* bar) {
-  if constexpr (W) mma_commit_w(bar);
-  else mma_commit(bar);
-}
-template <bool W>
-__device__ __forceinline__ void mma_ss_lh_x(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
-                                            uint32_t hi, uint32_t idesc, uint32_t accumulate) {
-  if constexpr (W) mma_ss_lh_w(d_tmem, a_lo, b_lo, hi, idesc, accumulate);
-  else mma_ss_lh(d_tmem, a_lo, b_lo, hi, idesc, accumulate);
-}
-template <bool W>
-__device__ __forceinline__ void mma_ts_lh_x(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
-                                            uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
-  if constexpr (W) mma_ts_lh_w(d_tmem, a_tmem, b_lo, b_hi, idesc, accumulate);
-  else mma_ts_lh(d_tmem, a_tmem, b_lo, b_hi, idesc, accumulate);
 }
 
 }  // namespace sigattn
