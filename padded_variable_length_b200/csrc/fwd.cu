@@ -1,5 +1,5 @@
-// Forward kernel: fused tiled sigmoid (or softmax / softmax_1) attention over the tile
-// list of a plan, sm_100a.
+// Forward kernels: fused tiled sigmoid (fwd_sigmoid_kernel, below) and softmax / softmax_1
+// (fwd_kernel) attention over the tile list of a plan, sm_100a.
 //
 // Method: "Better Models, Faster Training: Sigmoid Attention for single-cell Foundation
 // Models", section 2A: O = sigma(Q K^T / sqrt(d) + b) V, each weight computed on its own
@@ -12,11 +12,11 @@
 //
 // Persistent: one CTA per SM walks the plan's longest-first list of (q-tile row, head)
 // work items with a stride of the grid size.  All tiles of all of a CTA's items form one
-// stream: the S = Q K^T of tile t is issued before the O += P V of tile t - 1, also across
-// item boundaries, so the tensor pipe works on the next item while the epilogue finishes
-// the last one.  384 threads:
+// stream.  fwd_kernel (softmax modes): the S = Q K^T of tile t is issued before the
+// O += P V of tile t - 1, also across item boundaries, so the tensor pipe works on the
+// next item while the epilogue finishes the last one.  384 threads:
 //   warp 0      TMA producer: Q of each item (two buffers), K and V tiles into a ring
-//   warp 1      TMEM allocator and MMA issuer (one thread)
+//   warp 1      TMEM allocator and MMA issuer (whole warp, one elected lane issues)
 //   warps 4-11  two epilogue warpgroups; thread = query row (TMEM lane); warpgroup g
 //               owns S columns [64g, 64g+64) and O columns [g d/2, (g+1) d/2)
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256, 256+d), O1 [256+d, 256+2d).  P (bf16)
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(o_full + i, 1);
       mbar_init(o_empty + i, 8);
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, EPI == 0 ? 4 : 8);  // sigmoid: one warpgroup per tile
+      mbar_init(p_full + i, 8);
     }
     mbar_init(pv_done, 1);
     for (int i = 0; i < S; ++i) {
@@ -245,7 +245,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // Whole-warp issue from warp-uniform values (see mma_ss_lh_w).
+    {
+      constexpr uint32_t kHi = sw128_desc_hi(1024);
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
       // the PV still to issue: its global tile, item number and place in the item
@@ -254,25 +256,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       auto issue_pv = [&]() -> bool {
         const int pb = pv_t & 1, s2 = pv_t % S, ob = pv_item & 1;
-        if (!mbar_wait(p_full + pb, (pv_t >> 1) & 1, wctx)) return false;
-        if (!mbar_wait(v_full + s2, (pv_t / S) & 1, wctx)) return false;
-        if (pv_first && pv_item >= 2 && !mbar_wait(o_empty + ob, ((pv_item >> 1) - 1) & 1, wctx))
+        if (!mbar_wait_w(p_full + pb, (pv_t >> 1) & 1, wctx)) return false;
+        if (!mbar_wait_w(v_full + s2, (pv_t / S) & 1, wctx)) return false;
+        if (pv_first && pv_item >= 2 && !mbar_wait_w(o_empty + ob, ((pv_item >> 1) - 1) & 1, wctx))
           return false;
         tc_fence_after();
         const uint32_t v_base = smem_u32(smem + L::kV + s2 * L::kTileBytes);
         const uint32_t o_tmem = tmem + 256 + ob * D;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          // sigmoid: P of keys 16kk.. at column 8kk (one warpgroup wrote the whole tile);
-          // softmax: warpgroup g wrote keys [64g, 64g+64) at columns [64g, 64g+32)
-          const uint32_t a_tmem =
-              tmem + pb * 128 + (EPI == 0 ? kk * 8 : (kk >> 2) * 64 + (kk & 3) * 8);
-          mma_ts(o_tmem, a_tmem, smem_desc_sw128(v_base + kk * 2048, L::kBoxBytes, 1024),
-                 idesc_pv, (pv_first && kk == 0) ? 0u : 1u);
+          // warpgroup g wrote the P of keys [64g, 64g+64) at columns [64g, 64g+32)
+          const uint32_t a_tmem = tmem + pb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+          mma_ts_lh_w(o_tmem, a_tmem, sw128_desc_lo(v_base + kk * 2048, L::kBoxBytes), kHi,
+                      idesc_pv, (pv_first && kk == 0) ? 0u : 1u);
         }
-        mma_commit(kv_empty + s2);
-        if (EPI != 0) mma_commit(pv_done);
-        if (pv_last) mma_commit(o_full + ob);
+        mma_commit_w(kv_empty + s2);
+        if (EPI != 0) mma_commit_w(pv_done);
+        if (pv_last) mma_commit_w(o_full + ob);
         return true;
       };
       int t = 0, i = 0;
@@ -280,23 +280,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = iter.cur;
         if (it.n == 0) continue;
         const int qb = i & 1;
-        if (!(ok = mbar_wait(q_full + qb, (i >> 1) & 1, wctx))) break;
+        if (!(ok = mbar_wait_w(q_full + qb, (i >> 1) & 1, wctx))) break;
         tc_fence_after();
         const uint32_t q_base = smem_u32(smem + L::kQ + qb * L::kTileBytes);
         for (int j = 0; j < it.n; ++j, ++t) {
           const int s = t % S;
-          if (!(ok = mbar_wait(k_full + s, (t / S) & 1, wctx))) break;
+          if (!(ok = mbar_wait_w(k_full + s, (t / S) & 1, wctx))) break;
           tc_fence_after();
           const uint32_t k_base = smem_u32(smem + L::kK + s * L::kTileBytes);
           const uint32_t d_tmem = tmem + (t & 1) * 128;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-            mma_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
-                   smem_desc_sw128(k_base + off, 16, 1024), idesc_qk, kk > 0);
+            mma_ss_lh_w(d_tmem, sw128_desc_lo(q_base + off, 16), sw128_desc_lo(k_base + off, 16),
+                        kHi, idesc_qk, kk > 0);
           }
-          mma_commit(s_full + (t & 1));
-          if (j == it.n - 1) mma_commit(q_empty + qb);
+          mma_commit_w(s_full + (t & 1));
+          if (j == it.n - 1) mma_commit_w(q_empty + qb);
           if (pv_t >= 0 && !(ok = issue_pv())) break;
           pv_t = t;
           pv_item = i;
@@ -307,122 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok && pv_t >= 0) issue_pv();
     }
-  } else if (EPI == 0 && warp >= kEpiWarp0) {
-    // ---------------------------------------------------------------- sigmoid epilogue
-    // Ping-pong: warpgroup g takes the tiles with t % 2 == g (S buffer g), all 128 columns,
-    // in four chunks of 32 whose TMEM loads overlap the previous chunk's math; the two
-    // warpgroups work on different tiles, so one's load / store latency hides under the
-    // other's MUFU work.  P of keys [32c, 32c+32) goes to columns [16c, 16c+16).
-    const int g = (warp - kEpiWarp0) >> 2;
-    const int wq = warp & 3;
-    const int row = wq * 32 + lane;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const uint32_t s_base = t_lane + g * 128;
-    constexpr int kOc = D / 2;
-    const float2 c1 = make_float2(0.5f * p.scale, 0.5f * p.scale);
-    const float2 half2 = make_float2(0.5f, 0.5f);
-    bool ok = true;
-    int t = 0, i = 0;
-    auto row_bias = [&](const Item& x) {
-      const int r = x.qt * kTile + row;
-      return (p.bias != nullptr && x.n > 0 && r < p.Nq) ? p.bias[x.b * p.bias_sb + r] : 0.0f;
-    };
-    ItemIter iter(p);
-    float bias_cur = iter.valid() ? row_bias(iter.cur) : 0.0f;
-    for (; ok && iter.valid(); iter.advance()) {
-      const Item it = iter.cur;
-      // the next item's bias, in flight while this one is processed
-      const float bias_nxt =
-          iter.w + static_cast<int>(gridDim.x) < p.nitems ? row_bias(iter.nxt) : 0.0f;
-      const float bias_r = bias_cur;
-      bias_cur = bias_nxt;
-      if (it.n == 0) {
-        // No tile in this row: the whole q-tile is padding or sees no key.  O = 0.
-        const int rows = min(kTile, p.Nq - it.qt * kTile);
-        constexpr int kChunks = D / 8;
-        const int tid = threadIdx.x - kEpiWarp0 * 32;
-        for (int c = tid; c < rows * kChunks; c += 256) {
-          const int rr = c / kChunks, ch = c % kChunks;
-          *reinterpret_cast<uint4*>(p.o + it.b * p.o_sb +
-                                    static_cast<int64_t>(it.qt * kTile + rr) * p.o_sn +
-                                    it.h * p.o_sh + ch * 8) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        continue;
-      }
-      const int ob = i & 1;
-      const float2 c0 = make_float2(0.5f * bias_r, 0.5f * bias_r);
-      const int t_end = t + it.n;
-      for (int tt = t + ((t & 1) != g ? 1 : 0); tt < t_end; tt += 2) {
-        const int s = tt % S;
-        // k_full of the tile's stage also publishes the kind and bitmask the producer staged
-        if (ok) ok = mbar_wait(k_full + s, (tt / S) & 1, wctx);
-        if (ok) ok = mbar_wait(s_full + g, (tt >> 1) & 1, wctx);
-        ok = __all_sync(0xFFFFFFFFu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        const bool masked = meta_kind[s] == 2;
-        uint4 mb = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
-        if (masked) mb = *reinterpret_cast<const uint4*>(meta_bits + s * 512 + row * 4);
-        uint32_t buf[2][32];
-        tmem_ld32(s_base, buf[0]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c < 3) tmem_ld32(s_base + 32 * (c + 1), buf[(c + 1) & 1]);
-          const uint32_t mw = c == 0 ? mb.x : (c == 1 ? mb.y : (c == 2 ? mb.z : mb.w));
-          uint32_t pk[16];
-#pragma unroll
-          for (int cc = 0; cc < 32; cc += 2) {
-            const float2 x = fma2(make_float2(__uint_as_float(buf[c & 1][cc]),
-                                              __uint_as_float(buf[c & 1][cc + 1])),
-                                  c1, c0);
-            float2 th = make_float2(tanh_approx(x.x), tanh_approx(x.y));
-            if (masked) {
-              th.x = ((mw >> cc) & 1u) ? th.x : -1.0f;
-              th.y = ((mw >> (cc + 1)) & 1u) ? th.y : -1.0f;
-            }
-            const float2 pw = fma2(th, half2, half2);
-            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
-          }
-          tmem_st16(s_base + 16 * c, pk);
-          if (c < 3) tmem_wait_ld();
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + g);
-      }
-      if (!ok) break;
-      // ---- output of this item: this warpgroup's half of the O columns
-      ok = mbar_wait(o_full + ob, (i >> 1) & 1, wctx);
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t pk[kOc / 2];
-#pragma unroll
-      for (int c0o = 0; c0o < kOc; c0o += 32) {
-        uint32_t orr[32];
-        tmem_ld32(t_lane + 256 + ob * D + g * kOc + c0o, orr);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          pk[c0o / 2 + c] = pack_bf16x2(__uint_as_float(orr[2 * c]), __uint_as_float(orr[2 * c + 1]));
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(o_empty + ob);
-      const int rg = it.qt * kTile + row;
-      if (rg < p.Nq) {
-        uint4* d4 = reinterpret_cast<uint4*>(p.o + it.b * p.o_sb + static_cast<int64_t>(rg) * p.o_sn +
-                                             it.h * p.o_sh + g * kOc);
-#pragma unroll
-        for (int c = 0; c < kOc / 8; ++c)
-          d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      t = t_end;
-      ++i;
-    }
-  } else if (EPI != 0 && warp >= kEpiWarp0) {
+  } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- softmax epilogue
     // Column split: warpgroup g owns S columns [64g, 64g+64) of every tile and O columns
     // [g d/2, (g+1) d/2); the row maximum is exchanged through shared memory.
@@ -1077,14 +962,17 @@ int launch_fwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.lse = lse;
   p.status = status;
   p.wait_ns = wait_ns;
-  if constexpr (EPI == 0) return launch_fwd_sigmoid_t<D>(p, tq, tk, tv, stream);
-  auto kern = fwd_kernel<D, EPI>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-  if (e != cudaSuccess) return cuda_status(e);
-  const int grid = std::min(p.nitems, num_sms());
-  kern<<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
-  return cuda_status(cudaGetLastError());
+  if constexpr (EPI == 0) {
+    return launch_fwd_sigmoid_t<D>(p, tq, tk, tv, stream);
+  } else {
+    auto kern = fwd_kernel<D, EPI>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return cuda_status(e);
+    const int grid = std::min(p.nitems, num_sms());
+    kern<<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
+    return cuda_status(cudaGetLastError());
+  }
 }
 
 }  // namespace
