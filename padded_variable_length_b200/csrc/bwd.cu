@@ -149,7 +149,7 @@ __global__ void d_preprocess_kernel(const __nv_bfloat16* __restrict__ o, int64_t
 // ---------------------------------------------------------------------------------------
 // Shared pieces of the two gradient kernels.
 //
-// Both are persistent (one CTA per SM, static stride over the plan's longest-first work
+// Both are persistent (one CTA per SM, snake order over the plan's longest-first work
 // list) and split every 128 x 128 tile into two halves along the walked axis: epilogue
 // warpgroup h owns half h.  d = 64 runs the "unit" schedule (three rotating TMEM buffers,
 // the MMAs of a half-tile issued three halves ahead, see the dK / dV layout); d = 128 keeps
@@ -183,23 +183,26 @@ __device__ __forceinline__ WorkRef decode_row(const BwdParams& p, int w) {
   return r;
 }
 
-// Walks this CTA's work items (stride = grid size) with the next item's decode issued one
-// item ahead, so that its global loads overlap the current item.
+// Walks this CTA's work items (snake order, see snake_item) with the next item's decode
+// issued one item ahead, so that its global loads overlap the current item.
 template <bool kCols>
 struct WorkIter {
   const BwdParams& p;
-  int w, nitems;
+  int k, w, wn, nitems;  // round, this item, next item, list length
   WorkRef cur, nxt;
   __device__ WorkRef dec(int ww) const { return kCols ? decode_col(p, ww) : decode_row(p, ww); }
-  __device__ WorkIter(const BwdParams& pp, int n) : p(pp), w(blockIdx.x), nitems(n) {
+  __device__ WorkIter(const BwdParams& pp, int n)
+      : p(pp), k(0), w(snake_item(0)), wn(snake_item(1)), nitems(n) {
     if (w < nitems) cur = dec(w);
-    if (w + static_cast<int>(gridDim.x) < nitems) nxt = dec(w + gridDim.x);
+    if (wn < nitems) nxt = dec(wn);
   }
   __device__ bool valid() const { return w < nitems; }
   __device__ void advance() {
-    w += gridDim.x;
+    ++k;
+    w = wn;
+    wn = snake_item(k + 1);
     cur = nxt;
-    if (w + static_cast<int>(gridDim.x) < nitems) nxt = dec(w + gridDim.x);
+    if (wn < nitems) nxt = dec(wn);
   }
 };
 
@@ -1138,7 +1141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WorkRef it = iter.cur;
       // the next item's row values, in flight while this one is processed
       float off_nxt = 0.0f, D_nxt = 0.0f;
-      if (iter.w + static_cast<int>(gridDim.x) < nitems && iter.nxt.n > 0) {
+      if (iter.wn < nitems && iter.nxt.n > 0) {
         off_nxt = row_offset<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
         D_nxt = row_D<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
       }
@@ -1220,7 +1223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WorkRef it = iter.cur;
       // the next item's row values, in flight while this one is processed
       float off_nxt = 0.0f, D_nxt = 0.0f;
-      if (iter.w + static_cast<int>(gridDim.x) < nitems && iter.nxt.n > 0) {
+      if (iter.wn < nitems && iter.nxt.n > 0) {
         off_nxt = row_offset<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
         D_nxt = row_D<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
       }

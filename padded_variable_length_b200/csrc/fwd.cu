@@ -11,10 +11,11 @@
 // softmax); softmax_1 starts from a zero logit whose value row is zero (m = 0, l = 1).
 //
 // Persistent: one CTA per SM walks the plan's longest-first list of (q-tile row, head)
-// work items with a stride of the grid size.  All tiles of all of a CTA's items form one
-// stream.  fwd_kernel (softmax modes): the S = Q K^T of tile t is issued before the
-// O += P V of tile t - 1, also across item boundaries, so the tensor pipe works on the
-// next item while the epilogue finishes the last one.  384 threads:
+// work items in snake order (even rounds forward, odd rounds backward over the grid).
+// All tiles of all of a CTA's items form one stream.  fwd_kernel (softmax modes): the
+// S = Q K^T of tile t is issued before the O += P V of tile t - 1, also across item
+// boundaries, so the tensor pipe works on the next item while the epilogue finishes the
+// last one.  384 threads:
 //   warp 0      TMA producer: Q of each item (two buffers), K and V tiles into a ring
 //   warp 1      TMEM allocator and MMA issuer (whole warp, one elected lane issues)
 //   warps 4-11  two epilogue warpgroups; thread = query row (TMEM lane); warpgroup g
@@ -96,21 +97,24 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p, int w) {
   return it;
 }
 
-// Walks this CTA's work items (stride = grid size) with the next item's decode issued one
-// item ahead, so that its global loads overlap the current item.
+// Walks this CTA's work items (snake order, see snake_item) with the next item's decode
+// issued one item ahead, so that its global loads overlap the current item.
 struct ItemIter {
   const FwdParams& p;
-  int w;
+  int k, w, wn;  // round, this item, next item
   Item cur, nxt;
-  __device__ explicit ItemIter(const FwdParams& pp) : p(pp), w(blockIdx.x) {
+  __device__ explicit ItemIter(const FwdParams& pp)
+      : p(pp), k(0), w(snake_item(0)), wn(snake_item(1)) {
     if (w < p.nitems) cur = decode_item(p, w);
-    if (w + static_cast<int>(gridDim.x) < p.nitems) nxt = decode_item(p, w + gridDim.x);
+    if (wn < p.nitems) nxt = decode_item(p, wn);
   }
   __device__ bool valid() const { return w < p.nitems; }
   __device__ void advance() {
-    w += gridDim.x;
+    ++k;
+    w = wn;
+    wn = snake_item(k + 1);
     cur = nxt;
-    if (w + static_cast<int>(gridDim.x) < p.nitems) nxt = decode_item(p, w + gridDim.x);
+    if (wn < p.nitems) nxt = decode_item(p, wn);
   }
 };
 
@@ -330,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (; iter.valid(); iter.advance()) {
       const Item it = iter.cur;
       const float bias_nxt =
-          iter.w + static_cast<int>(gridDim.x) < p.nitems ? row_bias(iter.nxt) : 0.0f;
+          iter.wn < p.nitems ? row_bias(iter.nxt) : 0.0f;
       const float bias_r = bias_cur;
       bias_cur = bias_nxt;
       if (it.n == 0) {
@@ -838,7 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = iter.cur;
       // the next item's bias, in flight while this one is processed
       const float bias_nxt =
-          iter.w + static_cast<int>(gridDim.x) < p.nitems ? row_bias(iter.nxt) : 0.0f;
+          iter.wn < p.nitems ? row_bias(iter.nxt) : 0.0f;
       const float bias_r = bias_cur;
       bias_cur = bias_nxt;
       if (it.n == 0) {

@@ -33,6 +33,15 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
+// Item of round k of a persistent CTA's walk over a work list sorted longest-first: the
+// CTAs take the items of even rounds in order and those of odd rounds in reverse ("snake"
+// order), which evens out the work per CTA better than a plain stride (single-cell batch:
+// at most 84 tiles per CTA instead of 89, mean 80.9).  Increasing in k for every CTA.
+__device__ __forceinline__ int snake_item(int k) {
+  const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  return k * g + ((k & 1) ? g - 1 - c : c);
+}
+
 // ------------------------------------------------------------------------------------
 // mbarrier
 // ------------------------------------------------------------------------------------
