@@ -77,3 +77,32 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+def test_more_argument_checks_without_device(lib):
+    P = ctypes.c_void_p
+    strides = (ctypes.c_int64 * 3)(0, 0, 0)
+    lib.sigattn_last_cuda_error.restype = ctypes.c_char_p
+    assert lib.sigattn_last_cuda_error() == b"no CUDA error"
+    bwd_args = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float] + [P, P] * 5 + \
+        [P, ctypes.c_int64, P, P] + [P, P] * 3
+    lib.sigattn_bwd.argtypes = bwd_args + [P]
+    lib.sigattn_bwd_ex.argtypes = bwd_args + [ctypes.c_int, P]
+    t = [P(16), strides] * 5
+    tail = [None, 0, None, None] + [P(16), strides] * 3
+    # no plan
+    assert lib.sigattn_bwd(None, 0, 1, 64, 0.125, *t, *tail, None) == -1
+    # a plan pointer that is never dereferenced: the part mask and the epilogue are checked
+    # first, the head dimension next
+    assert lib.sigattn_bwd_ex(P(16), 0, 1, 64, 0.125, *t, *tail, 0, None) == -1
+    assert lib.sigattn_bwd_ex(P(16), 0, 1, 64, 0.125, *t, *tail, 8, None) == -1
+    assert lib.sigattn_bwd_ex(P(16), 3, 1, 64, 0.125, *t, *tail, 7, None) == -1
+    assert lib.sigattn_bwd_ex(P(16), 0, 1, 96, 0.125, *t, *tail, 7, None) == -2
+    # softmax modes need LSE and the D workspace
+    assert lib.sigattn_bwd_ex(P(16), 1, 1, 64, 0.125, *t, *tail, 7, None) == -1
+    # the allocation-free form rejects a missing plan the same way
+    lib.sigattn_bwd_noalloc.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_float] + [P, P] * 5 + [P, ctypes.c_int64, P] + \
+        [P, P] * 3 + [P]
+    assert lib.sigattn_bwd_noalloc(None, 0, 1, 64, 0.125, *t, None, 0, None,
+                                   *([P(16), strides] * 3), None) == -1
