@@ -239,7 +239,7 @@ struct DkvLayout {
   // kv_full[KV] kv_empty[KV] q_full[S] q_empty[S] s_full[NR] p_full[NR] acc_full[A] acc_empty[A]
   // (NR = 4 unit slots for d = 64, one per half for d = 128)
   static constexpr int kRing = kUnits ? 4 : 2;
-  static constexpr int kNumBars = 2 * kKVBufs + 2 * kStages + 2 * kRing + 2 * kAccBufs;
+  static constexpr int kNumBars = 2 * kKVBufs + 2 * kStages + 2 * kRing + 2 * kAccBufs + 1;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -268,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_full + NR;    // [NR]
   uint64_t* acc_full = p_full + NR;  // [ACB]
   uint64_t* acc_empty = acc_full + ACB;
+  uint64_t* done = acc_empty + ACB;  // all MMAs complete (end of the kernel)
   float* vec = reinterpret_cast<float*>(smem + L::kVec);
   uint32_t* meta_bits = reinterpret_cast<uint32_t*>(smem + L::kMetaBits);
   int* meta_kind = reinterpret_cast<int*>(smem + L::kMetaKind);
@@ -293,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(acc_full + i, 1);
       mbar_init(acc_empty + i, 8);
     }
+    mbar_init(done, 1);
     *abort_flag = 0;
     *drain_flag = 0;
     fence_barrier_init();
@@ -474,6 +476,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = max(0, u - 3); ok && x < u; ++x)
       ok = acc(x, static_cast<uint32_t>((static_cast<int>(b3) + 3 + x - u) % 3));
+    // every MMA complete before the TMEM is released (also after an abort)
+    mma_commit_w(done);
+    {
+      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      mbar_wait_w(done, 0, drain);
+    }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (d = 128)
     // Whole-warp issue (see the unit schedule).  Per q-tile: S^T / dP^T of both halves, then
@@ -548,6 +556,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++ii;
       }
+    }
+    // every MMA complete before the TMEM is released (also after an abort)
+    mma_commit_w(done);
+    {
+      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      mbar_wait_w(done, 0, drain);
     }
   } else if (warp >= kEpiWarp0 && L::kUnits) {
     // ---------------------------------------------------------------- epilogue (units)
@@ -815,7 +829,7 @@ struct DqLayout {
   // qd_full[QB] qd_empty[QB] kv_full[S] kv_empty[S] s_full[NR] ds_full[NR] acc_full[A]
   // acc_empty[A] (NR = 4 unit slots for d = 64, one per half for d = 128)
   static constexpr int kRing = kUnits ? 4 : 2;
-  static constexpr int kNumBars = 2 * kQBufs + 2 * kStages + 2 * kRing + 2 * kAccBufs;
+  static constexpr int kNumBars = 2 * kQBufs + 2 * kStages + 2 * kRing + 2 * kAccBufs + 1;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -844,6 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* ds_full = s_full + NR;    // [NR]
   uint64_t* acc_full = ds_full + NR;  // [ACB]
   uint64_t* acc_empty = acc_full + ACB;
+  uint64_t* done = acc_empty + ACB;  // all MMAs complete (end of the kernel)
   uint32_t* meta_bits = reinterpret_cast<uint32_t*>(smem + L::kMetaBits);
   int* meta_kind = reinterpret_cast<int*>(smem + L::kMetaKind);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -868,6 +883,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(acc_full + i, 1);
       mbar_init(acc_empty + i, 8);
     }
+    mbar_init(done, 1);
     *abort_flag = 0;
     *drain_flag = 0;
     fence_barrier_init();
@@ -1020,6 +1036,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = max(0, u - 3); ok && x < u; ++x)
       ok = acc(x, static_cast<uint32_t>((static_cast<int>(b3) + 3 + x - u) % 3));
+    // every MMA complete before the TMEM is released (also after an abort)
+    mma_commit_w(done);
+    {
+      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      mbar_wait_w(done, 0, drain);
+    }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (d = 128)
     // Whole-warp issue; per k-tile: S / dP of both halves, then the dQ MMAs of each half
@@ -1085,6 +1107,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++ii;
       }
+    }
+    // every MMA complete before the TMEM is released (also after an abort)
+    mma_commit_w(done);
+    {
+      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      mbar_wait_w(done, 0, drain);
     }
   } else if (warp >= kEpiWarp0 && L::kUnits) {
     // ---------------------------------------------------------------- epilogue (units)
