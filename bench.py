@@ -34,6 +34,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from padded_variable_length_b200 import workloads as W  # noqa: E402
+from padded_variable_length_b200.replicas import (  # noqa: E402
+    job_throughput, max_over_ranks, replica_seed)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 EPI_BY_NAME = {"sigmoid": W.SIGMOID, "softmax": W.SOFTMAX, "softmax1": W.SOFTMAX1}
@@ -184,7 +186,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     epi = EPI_BY_NAME[args.epilogue]
     w = W.config(args.config, epilogue=epi)
     w.backward = True
-    w.seed = w.seed + 7919 * rank  # each replica its own data; the lengths stay those of the config
+    w.seed = replica_seed(w.seed, rank)
     t = W.tensors(w, with_grad=True)
     stream = torch.cuda.current_stream()
     d = {k: v.to(dev) for k, v in t.items()}
@@ -269,15 +271,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     dkdv_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
     dq_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
-    total_ms = fwd_ms + dkdv_ms + dq_ms
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(fwd_ms + dkdv_ms + dq_ms, dev)
 
     ff = fwd_flops(w)
     step_flops = 3.5 * ff
-    value = world * step_flops * args.steps / (total_ms / 1e3) / 1e12
+    value = job_throughput(world, step_flops, args.steps, total_ms)
     peaks, peak_src = load_peaks()
     peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     K = args.steps
@@ -376,11 +374,8 @@ def run_e2e(Bd, w, t, epi, dev, stream, args, world):
     ms = e0.elapsed_time(e1)
     for p in plans:
         p.close()
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
-    value = world * 3.5 * fwd_flops(w) * steps / (ms / 1e3) / 1e12
+    ms = max_over_ranks(ms, dev)
+    value = job_throughput(world, 3.5 * fwd_flops(w), steps, ms)
     return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps}
 
