@@ -142,3 +142,27 @@ def tile_list(mask: np.ndarray) -> dict:
 def tile_list_from_lengths(lengths, npad: int) -> dict:
     """The tile list of a padded batch, block by block from the lengths."""
     return _tile_list(*_length_blocks(lengths, npad))
+
+
+def row_runs(t: dict):
+    """Runs of a tile list (the dict of tile_list / tile_list_from_lengths): for each q-tile
+    row, the maximal ranges of consecutive k-tiles of one kind ("Binary Block Masking",
+    section "Comment ça marche ?", consecutive non-zero blocks).  Returns run_ptr int32
+    [B*QT + 1] and runs int32 [nruns, 4] = {first k-tile, number of tiles, kind, first CSR
+    entry}, rows in order, runs in ascending k-tile order; found by walking each row's
+    entries one by one."""
+    run_ptr = [0]
+    runs = []
+    for r in range(len(t["row_ptr"]) - 1):
+        e0, e1 = int(t["row_ptr"][r]), int(t["row_ptr"][r + 1])
+        e = e0
+        while e < e1:
+            start = e
+            while (e + 1 < e1 and t["col_idx"][e + 1] == t["col_idx"][e] + 1
+                   and t["kind"][e + 1] == t["kind"][start]):
+                e += 1
+            runs.append([int(t["col_idx"][start]), e - start + 1, int(t["kind"][start]), start])
+            e += 1
+        run_ptr.append(len(runs))
+    return (np.asarray(run_ptr, dtype=np.int32),
+            np.asarray(runs, dtype=np.int32).reshape(-1, 4))

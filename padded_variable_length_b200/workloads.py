@@ -160,6 +160,77 @@ def config(idx: int, seed: Optional[int] = None, epilogue: int = SIGMOID) -> Wor
     raise ValueError(f"no workload {idx}")
 
 
+def longformer_mask(n: int, radius: int, n_global: int) -> np.ndarray:
+    """Longformer-style element mask of one row of n tokens: token i sees token j iff
+    |i - j| <= radius (a sliding window) or either of them is one of the first n_global
+    tokens (global tokens see everything and are seen by everything)."""
+    i = np.arange(n)
+    local = np.abs(i[:, None] - i[None, :]) <= radius
+    glob = (i[:, None] < n_global) | (i[None, :] < n_global)
+    return (local | glob).astype(np.uint8)
+
+
+def tree_parents(rng: np.random.Generator, nodes: int, max_children: int = 4) -> np.ndarray:
+    """A random token tree of `nodes` nodes in breadth-first order: parent[0] = -1 (the root)
+    and every later node hangs under an earlier node that has fewer than max_children
+    children, picked uniformly -- the shape of the candidate trees that parallel decoding
+    verifies in one pass."""
+    parent = np.full(nodes, -1, dtype=np.int64)
+    children = np.zeros(nodes, dtype=np.int64)
+    for k in range(1, nodes):
+        open_nodes = np.flatnonzero(children[:k] < max_children)
+        pk = int(rng.choice(open_nodes))
+        parent[k] = pk
+        children[pk] += 1
+    return parent
+
+
+def tree_mask(prefix: int, parent: np.ndarray) -> np.ndarray:
+    """Element mask of a causal prefix followed by a token tree: prefix token i sees the
+    prefix tokens j <= i; tree node k (token prefix + k) sees the whole prefix and the tree
+    nodes on its path to the root (itself included), nothing else."""
+    nodes = parent.shape[0]
+    n = prefix + nodes
+    m = np.zeros((n, n), dtype=np.uint8)
+    m[:prefix, :prefix] = np.tril(np.ones((prefix, prefix), dtype=np.uint8))
+    m[prefix:, :prefix] = 1
+    for k in range(nodes):
+        a = k
+        while a >= 0:
+            m[prefix + k, prefix + a] = 1
+            a = int(parent[a])
+    return m
+
+
+def mask_family(kind: str, seed: Optional[int] = None, epilogue: int = SIGMOID, B: int = 4,
+                H: int = 16, d: int = 128) -> Workload:
+    """The other block-mask families through the element-mask planner ("Binary Block
+    Masking", section on applications: tree attention masks, packed fine-tuning, Longformer
+    masks); synthetic shapes, the n of b = -log n being each query's number of keys.
+
+    longformer  B rows of N = 8192 tokens, sliding window of radius 256, 32 global tokens
+    tree        B rows of N = 4096 tokens: a causal prefix of 3840 and a random token tree of
+                256 nodes (at most 4 children per node)
+    packed      B rows of N = 8192 tokens of causal documents (the packed-documents workload)
+    """
+    if kind == "packed":
+        return config(4, seed=seed, epilogue=epilogue)
+    if seed is None:
+        seed = 2000 + {"longformer": 1, "tree": 2}[kind]
+    rng = np.random.default_rng(seed)
+    masks = []
+    for _ in range(B):
+        if kind == "longformer":
+            masks.append(longformer_mask(8192, 256, 32))
+        elif kind == "tree":
+            masks.append(tree_mask(3840, tree_parents(rng, 256)))
+        else:
+            raise ValueError(kind)
+    m = np.stack(masks)
+    counts = m.sum(axis=2, dtype=np.int64).astype(np.int32)
+    return masked_workload(kind, m, counts, H=H, d=d, epilogue=epilogue, backward=True, seed=seed)
+
+
 CONFIG_IDS = (1, 2, 3, 4, 5)
 
 

@@ -468,3 +468,62 @@ def test_planted_missing_D_term_in_softmax_backward_is_caught():
         ds = p * (do @ v.T)                      # forgot - D_i
         return scale * ds @ k, scale * ds.T @ q, p.T @ do
     assert _fd_check(A.SOFTMAX, 3, bwd=bad_bwd) > 1e-3
+
+
+# ----------------------------------------------------------------------------------------
+# the other mask families (Longformer, token trees)
+# ----------------------------------------------------------------------------------------
+
+def test_longformer_mask_counts():
+    n, r, g = 300, 17, 5
+    m = W.longformer_mask(n, r, g)
+    i = np.arange(n)
+    # a non-global row sees its window (clipped at the ends) plus the g global tokens
+    # that lie outside the window
+    for row in (g, 100, n - 1):
+        lo, hi = max(0, row - r), min(n - 1, row + r)
+        outside = sum(1 for j in range(g) if j < lo or j > hi)
+        assert m[row].sum() == (hi - lo + 1) + outside
+    assert np.all(m[:g] == 1) and np.all(m[:, :g] == 1)
+    assert np.array_equal(m, m.T)
+    assert m[50, 50 + r] == 1 and m[50, 50 + r + 1] == 0
+
+
+def test_tree_mask_is_ancestor_closure():
+    rng = np.random.default_rng(3)
+    parent = W.tree_parents(rng, 40, max_children=3)
+    assert parent[0] == -1 and np.all(parent[1:] < np.arange(1, 40)) and np.all(parent[1:] >= 0)
+    assert np.bincount(parent[1:], minlength=40).max() <= 3
+    P = 25
+    m = W.tree_mask(P, parent)
+    assert np.array_equal(m[:P, :P], np.tril(np.ones((P, P), dtype=np.uint8)))
+    assert np.all(m[:P, P:] == 0) and np.all(m[P:, :P] == 1)
+    for k in range(40):
+        anc, a = set(), k
+        while a >= 0:
+            anc.add(a)
+            a = parent[a]
+        assert set(np.flatnonzero(m[P + k, P:]).tolist()) == anc
+
+
+def test_row_runs_rebuild_the_tile_list_and_are_maximal():
+    rng = np.random.default_rng(4)
+    m = W.random_mask(rng, 2, 600, 700, density=0.3, empty_rows=2)
+    t = tiles.tile_list(m)
+    run_ptr, runs = tiles.row_runs(t)
+    col, kind = [], []
+    for r in range(len(run_ptr) - 1):
+        prev = None
+        for kt0, n, kd, e0 in runs[run_ptr[r]:run_ptr[r + 1]]:
+            assert n >= 1 and e0 == len(col)
+            if prev is not None:  # maximal: the next run is not a continuation
+                assert not (kt0 == prev[0] + prev[1] and kd == prev[2])
+            col.extend(range(kt0, kt0 + n))
+            kind.extend([kd] * n)
+            prev = (kt0, n, kd)
+        assert len(col) == t["row_ptr"][r + 1]
+    assert np.array_equal(np.array(col), t["col_idx"]) and np.array_equal(np.array(kind), t["kind"])
+    # a padded batch: full rows are one FULL run and at most one PARTIAL tail
+    tl = tiles.tile_list_from_lengths([300], 300)
+    rp, rr = tiles.row_runs(tl)
+    assert rr.tolist()[:2] == [[0, 2, 1, 0], [2, 1, 2, 2]]
