@@ -59,6 +59,13 @@ def workload_name(w: W.Workload, epi: int) -> str:
     return f"{desc}, {W.EPILOGUE_NAMES[epi]}, seed {w.seed}"
 
 
+def bench_workload(args, epi: int) -> W.Workload:
+    """The workload of --config, or of --mask (the other block-mask families)."""
+    if args.mask:
+        return W.mask_family(args.mask, epilogue=epi)
+    return W.config(args.config, epilogue=epi)
+
+
 def fwd_flops(w: W.Workload) -> float:
     return 4.0 * w.d * w.H * w.pairs()
 
@@ -151,7 +158,7 @@ def run_reference(args, rank: int, world: int):
     if rank != 0:
         return None
     epi = EPI_BY_NAME[args.epilogue]
-    w = W.config(args.config, epilogue=epi)
+    w = bench_workload(args, epi)
     w.backward = True
     t = W.tensors(w, with_grad=True)
     order = [(b, h) for h in range(w.H) for b in range(w.B)]
@@ -184,7 +191,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     epi = EPI_BY_NAME[args.epilogue]
-    w = W.config(args.config, epilogue=epi)
+    w = bench_workload(args, epi)
     w.backward = True
     w.seed = replica_seed(w.seed, rank)
     t = W.tensors(w, with_grad=True)
@@ -192,20 +199,31 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     d = {k: v.to(dev) for k, v in t.items()}
     counts = torch.from_numpy(np.ascontiguousarray(w.counts, dtype=np.int32)).to(dev)
 
+    # the planner's input, resident on the device before its timing starts
+    plan_in = (torch.from_numpy(w.lengths.astype(np.int32)).to(dev) if w.lengths is not None
+               else torch.from_numpy(w.mask).to(dev))
+
     def build_plan():
         if w.lengths is not None:
-            return Bd.Plan.from_lengths(torch.from_numpy(w.lengths.astype(np.int32)).to(dev), w.Nq)
-        return Bd.Plan.from_mask(torch.from_numpy(w.mask).to(dev))
+            return Bd.Plan.from_lengths(plan_in, w.Nq)
+        return Bd.Plan.from_mask(plan_in)
 
-    # plan build time (reported, not part of the step)
-    build_plan().close()
+    # plan build time (reported, not part of the step): median of a few builds, each
+    # bracketed by events on the stream (the build synchronises once inside)
+    for _ in range(2):
+        build_plan().close()
     torch.cuda.synchronize()
-    pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    pe0.record(stream)
+    plan_times = []
+    for _ in range(5):
+        pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pe0.record(stream)
+        p_ = build_plan()
+        pe1.record(stream)
+        torch.cuda.synchronize()
+        plan_times.append(pe0.elapsed_time(pe1))
+        p_.close()
+    plan_ms = statistics.median(plan_times)
     plan = build_plan()
-    pe1.record(stream)
-    torch.cuda.synchronize()
-    plan_ms = pe0.elapsed_time(pe1)
     sizes = plan.sizes()
 
     bias = Bd.bias_from_counts(counts) if epi == W.SIGMOID else None
@@ -215,13 +233,25 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # 256 MB > L2
 
-    parts = [
-        lambda: Bd.fwd(plan, d["q"], d["k"], d["v"], bias, epi, out=o, lse=lse),
-        lambda: Bd.bwd(plan, d["q"], d["k"], d["v"], o, d["do"], bias, epi, lse=lse, workspace=ws,
-                       dq=dq, dk=dk, dv=dv, parts=Bd.BWD_PREP | Bd.BWD_DKDV),
-        lambda: Bd.bwd(plan, d["q"], d["k"], d["v"], o, d["do"], bias, epi, lse=lse, workspace=ws,
-                       dq=dq, dk=dk, dv=dv, parts=Bd.BWD_DQ),
-    ]
+    fused = args.bwd == "fused" or (args.bwd == "auto" and w.d == 64)
+    fwd_part = lambda: Bd.fwd(plan, d["q"], d["k"], d["v"], bias, epi, out=o, lse=lse)
+    if fused:
+        fws = torch.empty((Bd.bwd_fused_workspace_bytes(plan, w.H, w.d, epi) + 3) // 4,
+                          dtype=torch.float32, device=dev)
+        parts = [fwd_part,
+                 lambda: Bd.bwd_fused(plan, d["q"], d["k"], d["v"], o, d["do"], bias, epi, lse=lse,
+                                      workspace=fws, dq=dq, dk=dk, dv=dv)]
+        part_names = ["fwd", "bwd_fused"]
+        # forward; [D preprocess,] accumulator zeroing, fused kernel, dQ conversion
+        launches_per_step = 1 + 3 + (1 if epi != W.SIGMOID else 0)
+    else:
+        parts = [fwd_part,
+                 lambda: Bd.bwd(plan, d["q"], d["k"], d["v"], o, d["do"], bias, epi, lse=lse,
+                                workspace=ws, dq=dq, dk=dk, dv=dv, parts=Bd.BWD_PREP | Bd.BWD_DKDV),
+                 lambda: Bd.bwd(plan, d["q"], d["k"], d["v"], o, d["do"], bias, epi, lse=lse,
+                                workspace=ws, dq=dq, dk=dk, dv=dv, parts=Bd.BWD_DQ)]
+        part_names = ["fwd", "bwd_dkdv", "bwd_dq"]
+        launches_per_step = 3 + (1 if epi != W.SIGMOID else 0)
     if not args.no_graph:
         # One CUDA graph per part: the host only replays, so no launch preparation (tensor
         # maps, argument checks, Python) sits between the device events.
@@ -243,9 +273,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 ev[k_].record(stream)
             fn()
         if ev:
-            ev[3].record(stream)
+            ev[len(parts)].record(stream)
 
-    launches_per_step = 3 + (1 if epi != W.SIGMOID else 0)
     sampler = ClockSampler(local_rank if os.environ.get("CUDA_VISIBLE_DEVICES") is None else 0)
     sampler.start()
     t_warm = time.perf_counter()
@@ -259,7 +288,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+           for _ in range(args.steps)]
     for i in range(args.steps):
         step(evs[i])
         flush.zero_()  # L2 flush between timed steps (outside the events)
@@ -268,10 +298,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         torch.distributed.barrier()
     clocks = sampler.stop()
     assert Bd.get_status() == 0, "device status reports a timed-out wait"
-    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
-    dkdv_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
-    dq_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
-    total_ms = max_over_ranks(fwd_ms + dkdv_ms + dq_ms, dev)
+    part_ms = [sum(e[k_].elapsed_time(e[k_ + 1]) for e in evs) for k_ in range(len(parts))]
+    total_ms = max_over_ranks(sum(part_ms), dev)
 
     ff = fwd_flops(w)
     step_flops = 3.5 * ff
@@ -279,12 +307,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     peaks, peak_src = load_peaks()
     peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     K = args.steps
-    kernels = {
-        "fwd": {"ms": fwd_ms / K, "flops": ff, "tflops": ff / (fwd_ms / K / 1e3) / 1e12},
-        "bwd_dkdv": {"ms": dkdv_ms / K, "flops": 2.0 * ff,
-                     "tflops": 2.0 * ff / (dkdv_ms / K / 1e3) / 1e12},
-        "bwd_dq": {"ms": dq_ms / K, "flops": 0.5 * ff, "tflops": 0.5 * ff / (dq_ms / K / 1e3) / 1e12},
-    }
+    # algorithmic FLOPs of each part: forward 4 d per pair; backward 10 d per pair, of
+    # which dK / dV 8 d and dQ 2 d in the split form
+    part_flops = {"fwd": ff, "bwd_fused": 2.5 * ff, "bwd_dkdv": 2.0 * ff, "bwd_dq": 0.5 * ff}
+    kernels = {}
+    for name, ms in zip(part_names, part_ms):
+        kernels[name] = {"ms": ms / K, "flops": part_flops[name],
+                         "tflops": part_flops[name] / (ms / K / 1e3) / 1e12}
+    bwd_ms = sum(part_ms[1:])
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
@@ -307,9 +337,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "launch": "API calls each step" if args.no_graph else "CUDA graph replay per part",
                    "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
         "fwd_tflops": kernels["fwd"]["tflops"], "fwd_frac": kernels["fwd"]["tflops"] / peak_tf,
-        "bwd_tflops": 2.5 * ff / ((dkdv_ms + dq_ms) / K / 1e3) / 1e12,
-        "bwd_frac": 2.5 * ff / ((dkdv_ms + dq_ms) / K / 1e3) / 1e12 / peak_tf,
+        "bwd_tflops": 2.5 * ff / (bwd_ms / K / 1e3) / 1e12,
+        "bwd_frac": 2.5 * ff / (bwd_ms / K / 1e3) / 1e12 / peak_tf,
+        "bwd_algo": "fused (one kernel, dQ by TMA reduce-add)" if fused else "split (dK/dV + dQ)",
         "kernels": kernels, "plan_ms": plan_ms,
+        "plan": plan_report(w, plan_ms, peaks, peak_src),
         "tiles": {"nonempty": sizes["nonempty"], "full": sizes["full"], "partial": sizes["partial"],
                   "grid_total": sizes["grid_total"],
                   "skipped_frac": 1.0 - sizes["nonempty"] / max(1, sizes["grid_total"])},
@@ -319,7 +351,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     }
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timing
-    out["e2e"] = run_e2e(Bd, w, t, epi, dev, stream, args, world)
+    out["e2e"] = run_e2e(Bd, w, t, epi, dev, stream, args, world, fused)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         order = [(b, h) for h in range(w.H) for b in range(w.B)]
         f, s, n = oracle_sample(w, epi, t, order, args.cpu_seconds)
@@ -331,7 +363,19 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     return out
 
 
-def run_e2e(Bd, w, t, epi, dev, stream, args, world):
+def plan_report(w, plan_ms, peaks, peak_src):
+    """The planner's rate: an element mask is read once (1 byte per element; the PARTIAL
+    blocks' bytes a second time for their bitmasks), a lengths plan reads B ints."""
+    if w.mask is not None:
+        nbytes = int(w.mask.size)
+        gbs = nbytes / (plan_ms * 1e-3) / 1e9
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        return {"input": "element mask", "bytes": nbytes, "ms": plan_ms, "gb_per_s": gbs,
+                "hbm_frac": gbs / hbm, "hbm_peak_gbs": hbm, "peak_source": f"{peak_src} copy"}
+    return {"input": "lengths", "bytes": int(w.lengths.size * 4), "ms": plan_ms}
+
+
+def run_e2e(Bd, w, t, epi, dev, stream, args, world, fused):
     """Same metric through the user's call with HOST buffers: every step copies Q, K, V, dO,
     the lengths (or mask) and the bias counts in from pinned memory, builds the plan, runs
     forward + backward, and copies O, dQ, dK, dV back out."""
@@ -355,7 +399,8 @@ def run_e2e(Bd, w, t, epi, dev, stream, args, world):
             plan = Bd.Plan.from_mask(host_mask.to(dev, non_blocking=True))
         bias = Bd.bias_from_counts(counts) if epi == W.SIGMOID else None
         o, lse = Bd.fwd(plan, d["q"], d["k"], d["v"], bias, epi)
-        dq, dk, dv = Bd.bwd(plan, d["q"], d["k"], d["v"], o, d["do"], bias, epi, lse=lse)
+        bwd = Bd.bwd_fused if fused else Bd.bwd
+        dq, dk, dv = bwd(plan, d["q"], d["k"], d["v"], o, d["do"], bias, epi, lse=lse)
         for name, x in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
             outs[name].copy_(x, non_blocking=True)
         return plan
@@ -388,8 +433,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--epilogue", default="sigmoid", choices=list(EPI_BY_NAME))
+    ap.add_argument("--mask", default=None, choices=["longformer", "tree", "packed"],
+                    help="run a block-mask family (B=4, H=16, d=128) instead of --config")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bwd", default="auto", choices=["auto", "fused", "split"],
+                    help="backward form: fused (d = 64 only) or the two-kernel split; auto = "
+                         "fused where supported")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every part through the API each step instead of replaying CUDA graphs")
     args = ap.parse_args()

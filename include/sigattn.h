@@ -135,6 +135,20 @@ SIGATTN_API int sigattn_plan_export(const sigattn_plan* plan, int32_t* row_ptr, 
  */
 SIGATTN_API int sigattn_plan_export_work(const sigattn_plan* plan, int32_t* row_work, int32_t* col_work);
 
+/*
+ * Copies the runs of the tile list to HOST buffers (any may be NULL); synchronises.  A run
+ * is a maximal range of consecutive k-tiles of one kind within a q-tile row: the kernels
+ * walk a run without a per-tile list lookup ("Binary Block Masking for FlashAttention",
+ * section "Comment ça marche ?": consecutive non-zero blocks skip the redundant checks and
+ * reads).  The entries of a run are consecutive in the CSR list, and so are the bitmask
+ * numbers of a PARTIAL run.
+ *   run_ptr int32 [B*QT + 1]     runs of row r: runs[run_ptr[r] .. run_ptr[r+1])
+ *   runs    int32 [nruns * 4]    {first k-tile, number of tiles, kind (1 / 2), first CSR entry}
+ *   nruns   int64, one value     number of runs
+ */
+SIGATTN_API int sigattn_plan_export_runs(const sigattn_plan* plan, int32_t* run_ptr, int32_t* runs,
+                                         int64_t* nruns);
+
 /* Releases the plan's device memory.  Safe on NULL.  The caller must ensure no
  * kernel that uses the plan is still running. */
 SIGATTN_API void sigattn_plan_destroy(sigattn_plan* plan);
@@ -212,6 +226,39 @@ SIGATTN_API int sigattn_bwd_ex(const sigattn_plan* plan, int epilogue, int H, in
                                int parts, sigattn_stream stream);
 
 /*
+ * Fused backward (d = 64 only): the same dQ, dK, dV as sigattn_bwd from ONE walk over the
+ * k-tile columns of the plan, so the attention weights and dP of each tile are computed
+ * once instead of once per kernel.  Each tile's dQ contribution (dS K, tensor cores) is
+ * added into an fp32 accumulator in `workspace` with TMA bulk reduce-adds; a small kernel
+ * zeroes the accumulator rows of listed q-tiles first and one converts them to bf16 dQ
+ * (times scale; rows of q-tiles with no tile get 0) at the end.  This is the variant the
+ * two-kernel split of "Better Models, Faster Training", section 2C, avoids (there the
+ * accumulation would need atomics); here the TMA unit does the additions.
+ *
+ * workspace: device memory of at least sigattn_bwd_fused_workspace_size() bytes, 16-byte
+ * aligned, owned by the caller; its contents on entry do not matter and are undefined after.
+ * Layout: fp32 dQ accumulator [B, Nq, H, 64], then (softmax modes) D [B, H, Nq].  Calls
+ * sharing a workspace must not overlap on the GPU.  The order of the fp32 additions varies
+ * from run to run, so dQ can differ in the last bits between runs; dK and dV are
+ * deterministic.  Other arguments, results and errors as sigattn_bwd; d != 64 gives
+ * UNSUPPORTED, a missing or too small workspace INVALID.
+ */
+SIGATTN_API int sigattn_bwd_fused_workspace_size(const sigattn_plan* plan, int epilogue, int H,
+                                                 int d, size_t* bytes);
+SIGATTN_API int sigattn_bwd_fused(const sigattn_plan* plan, int epilogue, int H, int d,
+                                  float scale, const void* q, const int64_t q_strides[3],
+                                  const void* k, const int64_t k_strides[3],
+                                  const void* v, const int64_t v_strides[3],
+                                  const void* o, const int64_t o_strides[3],
+                                  const void* dout, const int64_t do_strides[3],
+                                  const float* bias, int64_t bias_stride_b, const float* lse,
+                                  void* workspace, size_t workspace_bytes,
+                                  void* dq, const int64_t dq_strides[3],
+                                  void* dk, const int64_t dk_strides[3],
+                                  void* dv, const int64_t dv_strides[3],
+                                  sigattn_stream stream);
+
+/*
  * Backward that allocates nothing, for callers that cannot call cudaMalloc: code running
  * under a memory manager that owns all device memory (a framework's caching allocator, or a
  * fixed budget set by a host application that loads this library as a plug-in), and step
@@ -224,8 +271,9 @@ SIGATTN_API int sigattn_bwd_ex(const sigattn_plan* plan, int epilogue, int H, in
  * by every GPU that loads the library until the process exits).  B * H * Nq above
  * SIGATTN_NOALLOC_MAX_ROWS gives SIGATTN_ERR_UNSUPPORTED for SOFTMAX / SOFTMAX1 (SIGMOID uses
  * no scratch and has no limit).  The first call on a device looks up the array's device
- * address (once per device, with that device current); make that first call before any
- * stream capture.  All calls share the one array and it keeps the last call's contents;
+ * address (once per device, with that device current) and keeps it for the life of the
+ * process, so a cudaDeviceReset after that is not supported; make that first call before
+ * any stream capture.  All calls share the one array and it keeps the last call's contents;
  * every value a call reads is written by that same call first, so nothing has to be cleared,
  * but calls whose kernels overlap on the GPU (other streams, other threads) race on it.
  */

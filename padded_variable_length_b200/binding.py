@@ -63,6 +63,7 @@ _sig("sigattn_plan_from_mask", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, cty
 _sig("sigattn_plan_get_sizes", ctypes.c_int, _p, ctypes.POINTER(PlanSizes))
 _sig("sigattn_plan_export", ctypes.c_int, _p, _p, _p, _p, _p, _p, _p, _p, _p)
 _sig("sigattn_plan_export_work", ctypes.c_int, _p, _p, _p)
+_sig("sigattn_plan_export_runs", ctypes.c_int, _p, _p, _p, ctypes.POINTER(_i64))
 _sig("sigattn_plan_destroy", None, _p)
 _sig("sigattn_bias_from_counts", ctypes.c_int, _p, _i64, _p, _p)
 _sig("sigattn_fwd", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
@@ -75,6 +76,11 @@ _sig("sigattn_bwd_ex", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_in
      _p, _I64x3, _p, _I64x3, _p, _I64x3, ctypes.c_int, _p)
 _sig("sigattn_bwd_noalloc", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
      _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _i64, _p,
+     _p, _I64x3, _p, _I64x3, _p, _I64x3, _p)
+_sig("sigattn_bwd_fused_workspace_size", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+     ctypes.POINTER(ctypes.c_size_t))
+_sig("sigattn_bwd_fused", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+     _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _i64, _p, _p, ctypes.c_size_t,
      _p, _I64x3, _p, _I64x3, _p, _I64x3, _p)
 _sig("sigattn_get_status", ctypes.c_int, _p)
 _sig("sigattn_set_wait_limit_ns", ctypes.c_int, _u64)
@@ -159,6 +165,19 @@ class Plan:
         _check(_lib.sigattn_plan_export_work(self._h, rw.ctypes.data, cw.ctypes.data), "plan_export_work")
         return rw, cw
 
+    def export_runs(self):
+        """(run_ptr int32 [B*QT + 1], runs int32 [nruns, 4]): each q-tile row's maximal
+        ranges of consecutive k-tiles of one kind, {first k-tile, count, kind, first entry}."""
+        z = self.sizes()
+        n = _i64()
+        _check(_lib.sigattn_plan_export_runs(self._h, None, None, ctypes.byref(n)), "plan_export_runs")
+        run_ptr = np.zeros(z["B"] * z["QT"] + 1, np.int32)
+        runs = np.zeros((n.value, 4), np.int32)
+        _check(_lib.sigattn_plan_export_runs(self._h, run_ptr.ctypes.data,
+                                             runs.ctypes.data if runs.size else None,
+                                             ctypes.byref(n)), "plan_export_runs")
+        return run_ptr, runs
+
     def close(self):
         if self._h is not None and self._h.value:
             _lib.sigattn_plan_destroy(self._h)
@@ -233,6 +252,41 @@ def bwd(plan: Plan, q, k, v, o, do, bias=None, epilogue: int = SIGMOID, lse=None
                                workspace.data_ptr() if workspace is not None else None,
                                dq.data_ptr(), _strides(dq), dk.data_ptr(), _strides(dk),
                                dv.data_ptr(), _strides(dv), int(parts), _stream(stream)), "bwd")
+    return dq, dk, dv
+
+
+def bwd_fused_workspace_bytes(plan: Plan, H: int, d: int, epilogue: int = SIGMOID) -> int:
+    n = ctypes.c_size_t()
+    _check(_lib.sigattn_bwd_fused_workspace_size(plan.handle, epilogue, H, d, ctypes.byref(n)),
+           "bwd_fused_workspace_size")
+    return n.value
+
+
+def bwd_fused(plan: Plan, q, k, v, o, do, bias=None, epilogue: int = SIGMOID, lse=None,
+              scale: Optional[float] = None, workspace=None, dq=None, dk=None, dv=None, stream=None):
+    """dQ, dK, dV of L = sum(dO * O) in one walk over the k-tile columns (d = 64): dQ is
+    accumulated in fp32 in ``workspace`` (a 16-byte aligned CUDA buffer of at least
+    bwd_fused_workspace_bytes bytes; allocated here if None) and converted at the end."""
+    B, Nq, H, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_fused_workspace_bytes(plan, H, d, epilogue)
+    if workspace is None:
+        workspace = torch.empty((need + 3) // 4, dtype=torch.float32, device=q.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    bp, bs = _bias_args(bias)
+    o_ptr = o.data_ptr() if o is not None else None
+    o_str = _strides(o) if o is not None else _I64x3(0, 0, 0)
+    _check(_lib.sigattn_bwd_fused(plan.handle, epilogue, H, d, float(scale),
+                                  q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
+                                  v.data_ptr(), _strides(v), o_ptr, o_str, do.data_ptr(), _strides(do),
+                                  bp, bs, lse.data_ptr() if lse is not None else None,
+                                  workspace.data_ptr(), nbytes,
+                                  dq.data_ptr(), _strides(dq), dk.data_ptr(), _strides(dk),
+                                  dv.data_ptr(), _strides(dv), _stream(stream)), "bwd_fused")
     return dq, dk, dv
 
 

@@ -28,6 +28,14 @@ int launch_bwd_impl(const sigattn_plan* plan, int epilogue, int H, int d, float 
                     const TensorDesc& dq, const TensorDesc& dk, const TensorDesc& dv,
                     int parts, int* status, unsigned long long wait_ns, cudaStream_t stream);
 
+int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float scale,
+                          const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, const CUtensorMap& tdq, const TensorDesc& o,
+                          const TensorDesc& dout, const float* bias, int64_t bias_sb,
+                          const float* lse, float* Dws, float* dqacc, const TensorDesc& dq,
+                          const TensorDesc& dk, const TensorDesc& dv, int* status,
+                          unsigned long long wait_ns, cudaStream_t stream);
+
 std::atomic<int> g_last_cuda_error{0};
 
 int cuda_status(cudaError_t e) {
@@ -41,28 +49,14 @@ namespace {
 
 std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-int* g_status_ptr[kMaxDevices] = {nullptr};
+SymbolAddressCache g_status_addr;
 
-// Device address of this device's status word (host code cannot name the symbol's
-// address directly).
+// Device address of this device's status word.
 int status_ptr(int** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
-    cudaGetLastError();
-    return SIGATTN_ERR_NO_DEVICE;
-  }
-  if (dev < 0 || dev >= kMaxDevices) return SIGATTN_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_status_ptr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_status_word);
-    if (e != cudaSuccess) return cuda_status(e);
-    g_status_ptr[dev] = static_cast<int*>(p);
-  }
-  *out = g_status_ptr[dev];
-  return SIGATTN_OK;
+  void* p = nullptr;
+  const int rc = g_status_addr.get(g_status_word, &p);
+  *out = static_cast<int*>(p);
+  return rc;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -154,6 +148,21 @@ int make_tmap_bf16(CUtensorMap* map, const TensorDesc& t, int B, int H, int d) {
   return r == CUDA_SUCCESS ? SIGATTN_OK : SIGATTN_ERR_ALIGNMENT;
 }
 
+int make_tmap_f32_acc(CUtensorMap* map, float* base, int B, int N, int H, int d) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return SIGATTN_ERR_CUDA;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  const cuuint64_t row = static_cast<cuuint64_t>(d) * 4;  // bytes of one (token, head) row
+  const cuuint64_t st[3] = {row * H, row, row * H * N};   // token, head, batch strides
+  const cuuint32_t box[4] = {32, 16, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, st, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SIGATTN_OK : SIGATTN_ERR_ALIGNMENT;
+}
+
 }  // namespace sigattn
 
 using namespace sigattn;
@@ -228,6 +237,67 @@ extern "C" int sigattn_bwd_ex(const sigattn_plan* plan, int epilogue, int H, int
   return launch_bwd_impl(plan, epilogue, H, d, scale, mq, mk, mv, mdo, to, tdo, bias,
                          bias_stride_b, lse, workspace, tdq, tdk, tdv, parts, status,
                          g_wait_limit_ns.load(), static_cast<cudaStream_t>(s));
+}
+
+extern "C" int sigattn_bwd_fused_workspace_size(const sigattn_plan* plan, int epilogue, int H,
+                                                int d, size_t* bytes) {
+  if (!plan || !bytes || H < 1 || epilogue < 0 || epilogue > 2) return SIGATTN_ERR_INVALID;
+  if (d != 64) return SIGATTN_ERR_UNSUPPORTED;
+  const size_t rows = static_cast<size_t>(plan->B) * plan->Nq * H;
+  *bytes = rows * d * sizeof(float) + (epilogue != SIGATTN_SIGMOID ? rows * sizeof(float) : 0);
+  return SIGATTN_OK;
+}
+
+extern "C" int sigattn_bwd_fused(const sigattn_plan* plan, int epilogue, int H, int d, float scale,
+                                 const void* q, const int64_t q_strides[3], const void* k,
+                                 const int64_t k_strides[3], const void* v,
+                                 const int64_t v_strides[3], const void* o,
+                                 const int64_t o_strides[3], const void* dout,
+                                 const int64_t do_strides[3], const float* bias,
+                                 int64_t bias_stride_b, const float* lse, void* workspace,
+                                 size_t workspace_bytes, void* dq, const int64_t dq_strides[3],
+                                 void* dk, const int64_t dk_strides[3], void* dv,
+                                 const int64_t dv_strides[3], sigattn_stream s) {
+  if (!plan || H < 1 || !std::isfinite(scale)) return SIGATTN_ERR_INVALID;
+  if (epilogue < 0 || epilogue > 2) return SIGATTN_ERR_INVALID;
+  if (d != 64) return SIGATTN_ERR_UNSUPPORTED;
+  if (epilogue != SIGATTN_SIGMOID && (!lse || !o)) return SIGATTN_ERR_INVALID;
+  if (bias && bias_stride_b < 0) return SIGATTN_ERR_INVALID;
+  size_t need = 0;
+  int rc = sigattn_bwd_fused_workspace_size(plan, epilogue, H, d, &need);
+  if (rc != SIGATTN_OK) return rc;
+  if (!workspace || workspace_bytes < need) return SIGATTN_ERR_INVALID;
+  if (!aligned16(workspace)) return SIGATTN_ERR_ALIGNMENT;
+  if (static_cast<int64_t>(plan->B) * (plan->QT > plan->KT ? plan->QT : plan->KT) * H >
+      0x7FFFFFFF)
+    return SIGATTN_ERR_UNSUPPORTED;
+  TensorDesc tq, tk, tv, to{}, tdo, tdq, tdk, tdv;
+  if ((rc = check_tensor(q, q_strides, plan->Nq, &tq)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(k, k_strides, plan->Nk, &tk)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(v, v_strides, plan->Nk, &tv)) != SIGATTN_OK) return rc;
+  if (epilogue != SIGATTN_SIGMOID &&
+      (rc = check_tensor(o, o_strides, plan->Nq, &to)) != SIGATTN_OK)
+    return rc;
+  if ((rc = check_tensor(dout, do_strides, plan->Nq, &tdo)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(dq, dq_strides, plan->Nq, &tdq)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(dk, dk_strides, plan->Nk, &tdk)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(dv, dv_strides, plan->Nk, &tdv)) != SIGATTN_OK) return rc;
+  if ((rc = check_plan_device(plan)) != SIGATTN_OK) return rc;
+  int* status = nullptr;
+  if ((rc = status_ptr(&status)) != SIGATTN_OK) return rc;
+  float* dqacc = static_cast<float*>(workspace);
+  float* Dws = epilogue != SIGATTN_SIGMOID
+                   ? dqacc + static_cast<size_t>(plan->B) * plan->Nq * H * d
+                   : nullptr;
+  CUtensorMap mq, mk, mv, mdo, macc;
+  if ((rc = make_tmap_bf16(&mq, tq, plan->B, H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mk, tk, plan->B, H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mv, tv, plan->B, H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mdo, tdo, plan->B, H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_f32_acc(&macc, dqacc, plan->B, plan->Nq, H, d)) != SIGATTN_OK) return rc;
+  return launch_bwd_fused_impl(plan, epilogue, H, scale, mq, mk, mv, mdo, macc, to, tdo, bias,
+                               bias_stride_b, lse, Dws, dqacc, tdq, tdk, tdv, status,
+                               g_wait_limit_ns.load(), static_cast<cudaStream_t>(s));
 }
 
 extern "C" int sigattn_bwd(const sigattn_plan* plan, int epilogue, int H, int d, float scale,

@@ -60,14 +60,14 @@ struct BwdParams {
   unsigned long long wait_ns;
 };
 
-// Offset of one query row in the weight's argument, with c1 the matching slope:
-// SIGMOID  p = 0.5 + 0.5 tanh(c1 s + off),  c1 = scale / 2,  off = bias / 2;
-// softmax  p = 2^(c1 s + off),               c1 = scale log2 e,  off = (bias - lse) log2 e.
+// Offset of one query row in the weight's argument t = c1 s + off, c1 = scale log2 e:
+// SIGMOID  p = sigma(t ln 2),  off = bias log2 e  (sigmoid_grad2);
+// softmax  p = 2^t,            off = (bias - lse) log2 e.
 template <int EPI>
 __device__ __forceinline__ float row_offset(const BwdParams& p, int b, int h, int qg) {
   if (qg >= p.Nq) return 0.0f;
   const float bias = p.bias ? p.bias[b * p.bias_sb + qg] : 0.0f;
-  if (EPI == 0) return 0.5f * bias;
+  if (EPI == 0) return bias * kLog2e;
   return (bias - p.lse[(static_cast<int64_t>(b) * p.H + h) * p.Nq + qg]) * kLog2e;
 }
 
@@ -78,20 +78,18 @@ __device__ __forceinline__ float row_D(const BwdParams& p, int b, int h, int qg)
 }
 
 // p and ds of two neighbouring elements (packed fp32 pairs); k0 / k1 are the mask bits.
-// SIGMOID: th = tanh(c1 s + off), p = (1 + th) / 2, p (1 - p) = (1 - th^2) / 4, so
-//   ds = dp (1/4 - th^2 / 4); a masked element takes th = -1, which gives p = ds = 0.
-// softmax: p = 2^(c1 s + off), ds = p (dp - D); a masked element takes p = 0.
+// SIGMOID: p = sigma(x), ds = dp sigma'(x) with sigma' = sigma (1 - sigma) from the same
+//   exp2 (sigmoid_grad2); a masked element takes t = -inf, which gives p = ds = 0.
+// softmax: p = 2^t, ds = p (dp - D); a masked element takes p = 0.
 template <int EPI>
 __device__ __forceinline__ void weight_grad2(float2 s, float2 dp, float2 c1, float2 off, float2 Dv,
                                              bool k0, bool k1, float2& pw, float2& ds) {
-  const float2 x = fma2(s, c1, off);
+  float2 x = fma2(s, c1, off);
   if (EPI == 0) {
-    float2 th = make_float2(tanh_approx(x.x), tanh_approx(x.y));
-    th.x = k0 ? th.x : -1.0f;
-    th.y = k1 ? th.y : -1.0f;
-    pw = fma2(th, make_float2(0.5f, 0.5f), make_float2(0.5f, 0.5f));
-    const float2 m = mul2(th, make_float2(-0.25f, -0.25f));
-    const float2 w = fma2(m, th, make_float2(0.25f, 0.25f));
+    x.x = k0 ? x.x : -INFINITY;
+    x.y = k1 ? x.y : -INFINITY;
+    float2 w;
+    sigmoid_grad2(x, pw, w);
     ds = mul2(w, dp);
   } else {
     pw = make_float2(k0 ? ex2_approx(x.x) : 0.0f, k1 ? ex2_approx(x.y) : 0.0f);
@@ -392,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (lane == 0 && *abort_flag) {
-      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
       for (int u = max(0, ii - KVB); u < ii; ++u) mbar_wait(kv_full + u % KVB, (u / KVB) & 1, drain);
       for (int u = max(0, qc - S); u < qc; ++u) mbar_wait(q_full + u % S, (u / S) & 1, drain);
     }
@@ -479,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // every MMA complete before the TMEM is released (also after an abort)
     mma_commit_w(done);
     {
-      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
       mbar_wait_w(done, 0, drain);
     }
   } else if (warp == 1) {
@@ -560,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // every MMA complete before the TMEM is released (also after an abort)
     mma_commit_w(done);
     {
-      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
       mbar_wait_w(done, 0, drain);
     }
   } else if (warp >= kEpiWarp0 && L::kUnits) {
@@ -569,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;
     const int row = wq * 32 + lane;  // key row of the tile
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const float c1s = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
+    const float c1s = p.scale * kLog2e;
     const float2 c1 = make_float2(c1s, c1s);
     constexpr int kOc = D / 2;  // dV / dK columns written by this warpgroup
     bool ok = true;
@@ -689,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;
     const int row = wq * 32 + lane;  // key row of the tile
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const float c1s = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
+    const float c1s = p.scale * kLog2e;
     const float2 c1 = make_float2(c1s, c1s);
     bool ok = true;
     int qc = 0, ii = 0;
@@ -956,7 +954,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (lane == 0 && *abort_flag) {
-      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
       for (int u = max(0, ii - QB); u < ii; ++u) mbar_wait(qd_full + u % QB, (u / QB) & 1, drain);
       for (int u = max(0, tk_ - S); u < tk_; ++u) mbar_wait(kv_full + u % S, (u / S) & 1, drain);
     }
@@ -1039,7 +1037,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // every MMA complete before the TMEM is released (also after an abort)
     mma_commit_w(done);
     {
-      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
       mbar_wait_w(done, 0, drain);
     }
   } else if (warp == 1) {
@@ -1111,7 +1109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // every MMA complete before the TMEM is released (also after an abort)
     mma_commit_w(done);
     {
-      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
       mbar_wait_w(done, 0, drain);
     }
   } else if (warp >= kEpiWarp0 && L::kUnits) {
@@ -1120,7 +1118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const float c1s = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
+    const float c1s = p.scale * kLog2e;
     const float2 c1 = make_float2(c1s, c1s);
     constexpr int kOc = D / 2;  // dQ columns written by this warpgroup
     bool ok = true;
@@ -1237,7 +1235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const float c1s = EPI == 0 ? 0.5f * p.scale : p.scale * kLog2e;
+    const float c1s = p.scale * kLog2e;
     const float2 c1 = make_float2(c1s, c1s);
     bool ok = true;
     int tk_ = 0, ii = 0;
@@ -1345,6 +1343,539 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, 512);
   }
 }
+// ---------------------------------------------------------------------------------------
+// Fused backward (d = 64): dK, dV and dQ in one walk over the k-tile columns of the plan.
+//
+// Per q-tile t of a column (thread = key row in the epilogue, as in the dK / dV kernel):
+//   S^T = K Q^T,  dP^T = V dO^T                  (full-width N = 128 MMAs)
+//   P^T, dS^T from the epilogue                  (TMEM, bf16, A operands of the next two)
+//   dV += P^T dO,  dK += dS^T Q                   (accumulated over the column in TMEM)
+//   dQ_t = dS K                                   (dS from shared memory, M = queries)
+// and dQ_t is added into an fp32 accumulator in global memory with TMA bulk reduce-adds, so
+// S and dP are computed once per tile instead of once per kernel of the two-kernel split
+// ("Better Models, Faster Training", section 2C, names that split; this is the variant it
+// avoids, with the reductions done by the TMA unit instead of atomics).  A zeroing kernel
+// before and a conversion kernel after (dQ = bf16(scale dQacc), pad rows 0) complete it.
+//
+// TMEM columns: X0 [0,128), X1 [128,256): S^T of tile t in X[t % 2]; the epilogue overwrites
+// it with P^T and dS^T (bf16, interleaved per 16 queries: P at 16j + [0,8), dS at
+// 16j + [8,16)); after the dV / dK MMAs have read them, dQ_t (fp32, 64 columns) is
+// accumulated in X[t % 2] [0,64) and drained by the epilogue.  Y [256,384): dP^T of tile t.
+// dV [384,448), dK [448,512).  The tensor pipe runs MMAs in issue order, so an MMA that
+// writes columns an earlier one reads needs no barrier between them.
+//
+// MMA issue order: S^T / dP^T of tile t, then dV / dK / dQ of tile t - 1 -- so the next
+// tile's scores are computed while the epilogue still works on the current one.
+// Barriers: sdp_full (S^T, dP^T of t ready), y_free (epilogue read dP^T of t), p_full (P /
+// dS of t in TMEM and dS in shared memory), dq_full (dQ_t done: its TMEM columns hold the
+// result and the shared dS buffer is free), x_free (dQ_t drained, X[t % 2] free).
+// ---------------------------------------------------------------------------------------
+struct FusedLayout {
+  static constexpr int kStages = 3;  // Q / dO ring
+  static constexpr int kKVBufs = 2;  // K / V of consecutive items
+  static constexpr int kTileBytes = 128 * 128;  // 128 rows x 64 bf16
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kKVBufs * kTileBytes;
+  static constexpr int kQ = kV + kKVBufs * kTileBytes;
+  static constexpr int kDO = kQ + kStages * kTileBytes;
+  static constexpr int kDS = kDO + kStages * kTileBytes;       // dS, two 64-query boxes
+  static constexpr int kStg = kDS + 2 * kTileBytes;            // dQ staging, 2 KB per warp
+  static constexpr int kVec = kStg + 8 * 2048;                 // float [S][2][128]
+  static constexpr int kMetaBits = kVec + kStages * 2 * 128 * 4;
+  static constexpr int kMetaKind = kMetaBits + kStages * 2048;
+  static constexpr int kBar = kMetaKind + 16;
+  // kv_full[2] kv_empty[2] q_full[S] q_empty[S] sdp_full[2] p_full[2] dq_full[2] x_free[2]
+  // y_free acc_full acc_empty done
+  static constexpr int kNumBars = 4 + 2 * kStages + 8 + 4;
+  static constexpr int kMisc = kBar + 8 * kNumBars;
+  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kStages * 4 <= 16, "meta kinds");
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    fused_bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                     const __grid_constant__ CUtensorMap tdq, const BwdParams p) {
+  using L = FusedLayout;
+  constexpr int D = 64;
+  constexpr int S = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int warp = warp_id(), lane = lane_id();
+  const int nitems = p.B * p.KT * p.H;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + 2;
+  uint64_t* q_full = bars + 4;
+  uint64_t* q_empty = q_full + S;
+  uint64_t* sdp_full = q_empty + S;  // [2]
+  uint64_t* p_full = sdp_full + 2;   // [2]
+  uint64_t* dq_full = p_full + 2;    // [2]
+  uint64_t* x_free = dq_full + 2;    // [2]
+  uint64_t* y_free = x_free + 2;
+  uint64_t* acc_full = y_free + 1;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* done = acc_empty + 1;
+  float* vec = reinterpret_cast<float*>(smem + L::kVec);
+  uint32_t* meta_bits = reinterpret_cast<uint32_t*>(smem + L::kMetaBits);
+  int* meta_kind = reinterpret_cast<int*>(smem + L::kMetaKind);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* drain_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
+  const WaitCtx wctx{p.status, p.wait_ns, abort_flag};
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(kv_full + i, 1);
+      mbar_init(kv_empty + i, 1);
+      mbar_init(sdp_full + i, 1);
+      mbar_init(p_full + i, 8);
+      mbar_init(dq_full + i, 1);
+      mbar_init(x_free + i, 8);
+    }
+    for (int i = 0; i < S; ++i) {
+      mbar_init(q_full + i, 2);  // TMA bytes + the producer's column vectors
+      mbar_init(q_empty + i, 1);
+    }
+    mbar_init(y_free, 8);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 8);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    *drain_flag = 0;
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  constexpr uint32_t kY = 256, kDV = 384, kDK = 448;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    // As in the dK / dV kernel: lane 0 waits and issues the copies; all lanes fetch the
+    // list entries of the next 32 q-tiles at once and the column vectors one tile ahead.
+    if (lane == 0) {
+      tma_prefetch_desc(&tq);
+      tma_prefetch_desc(&tk);
+      tma_prefetch_desc(&tv);
+      tma_prefetch_desc(&tdo);
+    }
+    int qc = 0, ii = 0;
+    bool ok = true;
+    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
+      if (it.n == 0) continue;
+      const int kb = ii & 1;
+      if (lane == 0 && ii >= 2) ok = mbar_wait(kv_empty + kb, ((ii >> 1) - 1) & 1, wctx);
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(kv_full + kb, 2 * L::kTileBytes);
+        tma_load_4d(smem + L::kK + kb * L::kTileBytes, &tk, kv_full + kb, 0, it.t * kTile, it.h, it.b);
+        tma_load_4d(smem + L::kV + kb * L::kTileBytes, &tv, kv_full + kb, 0, it.t * kTile, it.h, it.b);
+      }
+      ++ii;
+      auto fetch_vec = [&](int qt, float (&v0)[4], float (&v1)[4]) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int qg = qt * kTile + lane + 32 * k;
+          v0[k] = row_offset<EPI>(p, it.b, it.h, qg);
+          v1[k] = row_D<EPI>(p, it.b, it.h, qg);
+        }
+      };
+      float cur0[4], cur1[4], nx0[4], nx1[4];
+      fetch_vec(p.rowT_idx[it.e0], cur0, cur1);
+      for (int i0 = 0; ok && i0 < it.n; i0 += 32) {
+        const int il = i0 + lane;
+        int qt_l = 0, kd_l = 0, pi_l = 0;
+        if (il < it.n) {
+          qt_l = p.rowT_idx[it.e0 + il];
+          const int e = p.csc_map[it.e0 + il];
+          kd_l = p.kind[e];
+          if (kd_l == 2) pi_l = p.pidx[e];
+        }
+        const int jn = min(32, it.n - i0);
+        for (int u = 0; u < jn; ++u, ++qc) {
+          const int qt = __shfl_sync(0xFFFFFFFFu, qt_l, u);
+          const int kd = __shfl_sync(0xFFFFFFFFu, kd_l, u);
+          const int pi = __shfl_sync(0xFFFFFFFFu, pi_l, u);
+          const int i = i0 + u;
+          if (i + 1 < it.n) {
+            const int qn = (u + 1 < jn) ? __shfl_sync(0xFFFFFFFFu, qt_l, u + 1)
+                                        : p.rowT_idx[it.e0 + i + 1];
+            fetch_vec(qn, nx0, nx1);
+          }
+          const int s = qc % S;
+          if (lane == 0 && qc >= S) ok = mbar_wait(q_empty + s, ((qc / S) - 1) & 1, wctx);
+          ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          if (lane == 0) {
+            meta_kind[s] = kd;
+            mbar_arrive_expect_tx(q_full + s, 2 * L::kTileBytes + (kd == 2 ? 2048 : 0));
+            tma_load_4d(smem + L::kQ + s * L::kTileBytes, &tq, q_full + s, 0, qt * kTile, it.h, it.b);
+            tma_load_4d(smem + L::kDO + s * L::kTileBytes, &tdo, q_full + s, 0, qt * kTile, it.h,
+                        it.b);
+            if (kd == 2)
+              bulk_load(meta_bits + s * 512, p.bitsT + static_cast<int64_t>(pi) * 512, 2048,
+                        q_full + s);
+          }
+          float* vs = vec + s * 256;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            vs[lane + 32 * k] = cur0[k];
+            vs[128 + lane + 32 * k] = cur1[k];
+            cur0[k] = nx0[k];
+            cur1[k] = nx1[k];
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(q_full + s);
+        }
+      }
+    }
+    if (lane == 0 && *abort_flag) {
+      // Let the copies still in flight land before the CTA's shared memory goes away.
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
+      for (int u = max(0, ii - 2); u < ii; ++u) mbar_wait(kv_full + (u & 1), (u >> 1) & 1, drain);
+      for (int u = max(0, qc - S); u < qc; ++u) mbar_wait(q_full + u % S, (u / S) & 1, drain);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    constexpr uint32_t kHi = sw128_desc_hi(1024);
+    constexpr uint32_t idesc_sdp = idesc_bf16_f32(128, 128, false);       // S^T, dP^T
+    constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);          // dV, dK
+    constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, true, true);     // dQ (A = dS, MN-major)
+    constexpr uint32_t kT = L::kTileBytes >> 4;
+    const uint32_t k_lo0 = sw128_desc_lo(smem_u32(smem + L::kK), 16);
+    const uint32_t v_lo0 = sw128_desc_lo(smem_u32(smem + L::kV), 16);
+    const uint32_t q_lo0 = sw128_desc_lo(smem_u32(smem + L::kQ), 16);
+    const uint32_t do_lo0 = sw128_desc_lo(smem_u32(smem + L::kDO), 16);
+    const uint32_t q_mn0 = sw128_desc_lo(smem_u32(smem + L::kQ), L::kTileBytes);
+    const uint32_t do_mn0 = sw128_desc_lo(smem_u32(smem + L::kDO), L::kTileBytes);
+    const uint32_t k_mn0 = sw128_desc_lo(smem_u32(smem + L::kK), L::kTileBytes);
+    const uint32_t ds_mn = sw128_desc_lo(smem_u32(smem + L::kDS), L::kTileBytes);
+    bool ok = true;
+    // the tile whose dV / dK / dQ are still to issue: stage | kv buffer << 2 |
+    // first of item << 3 | last of item << 4 | item << 5
+    int pend = -1;
+    // dV += P^T dO, dK += dS^T Q, dQ_x = dS K for tile x, once its epilogue is done
+    auto acc = [&](int x, int info) -> bool {
+      const int s = info & 3, kb = (info >> 2) & 1, item = info >> 5;
+      const bool first = ((info >> 3) & 1) != 0, last = ((info >> 4) & 1) != 0;
+      if (!mbar_wait_w(p_full + (x & 1), (x >> 1) & 1, wctx)) return false;
+      if (first && item >= 1 && !mbar_wait_w(acc_empty, (item - 1) & 1, wctx)) return false;
+      tc_fence_after();
+      const uint32_t xb = tmem + (x & 1) * 128;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        // P^T of queries 16kk.. at columns [16kk, 16kk+8), dS^T at [16kk+8, 16kk+16)
+        const uint32_t a = (first && kk == 0) ? 0u : 1u;
+        mma_ts_lh_w(tmem + kDV, xb + 16 * kk, do_mn0 + s * kT + kk * 128, kHi, idesc_acc, a);
+        mma_ts_lh_w(tmem + kDK, xb + 16 * kk + 8, q_mn0 + s * kT + kk * 128, kHi, idesc_acc, a);
+      }
+      // dQ_x = dS K: keys 16kk.. are rows 16kk.. of the dS boxes and of the K tile
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ss_lh_w(xb, ds_mn + kk * 128, k_mn0 + kb * kT + kk * 128, kHi, idesc_dq,
+                    kk > 0 ? 1u : 0u);
+      mma_commit_w(q_empty + s);
+      mma_commit_w(dq_full + (x & 1));
+      if (last) {
+        mma_commit_w(acc_full);
+        mma_commit_w(kv_empty + kb);
+      }
+      return true;
+    };
+    int t = 0, ii = 0;
+    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
+      if (it.n == 0) continue;
+      const int kb = ii & 1;
+      if (!(ok = mbar_wait_w(kv_full + kb, (ii >> 1) & 1, wctx))) break;
+      const uint32_t k_lo = k_lo0 + kb * kT, v_lo = v_lo0 + kb * kT;
+      for (int i = 0; i < it.n; ++i, ++t) {
+        const int s = t % S;
+        if (!(ok = mbar_wait_w(q_full + s, (t / S) & 1, wctx))) break;
+        if (t >= 2 && !(ok = mbar_wait_w(x_free + (t & 1), ((t - 2) >> 1) & 1, wctx))) break;
+        if (t >= 1 && !(ok = mbar_wait_w(y_free, (t - 1) & 1, wctx))) break;
+        tc_fence_after();
+        const uint32_t xb = tmem + (t & 1) * 128;
+        const uint32_t q_lo = q_lo0 + s * kT, do_lo = do_lo0 + s * kT;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss_lh_w(xb, k_lo + kk * 2, q_lo + kk * 2, kHi, idesc_sdp, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss_lh_w(tmem + kY, v_lo + kk * 2, do_lo + kk * 2, kHi, idesc_sdp, kk > 0 ? 1u : 0u);
+        mma_commit_w(sdp_full + (t & 1));
+        if (pend >= 0 && !(ok = acc(t - 1, pend))) break;
+        pend = s | (kb << 2) | (i == 0 ? 8 : 0) | (i == it.n - 1 ? 16 : 0) | (ii << 5);
+      }
+      if (!ok) break;
+      ++ii;
+    }
+    if (ok && pend >= 0) ok = acc(t - 1, pend);
+    // every MMA complete before the TMEM is released (also after an abort)
+    mma_commit_w(done);
+    {
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
+      mbar_wait_w(done, 0, drain);
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ---------------------------------------------------------------- epilogue
+    // Warpgroup g owns queries [64g, 64g+64) of every tile; thread = key row (TMEM lane).
+    const int g = (warp - kEpiWarp0) >> 2;
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float c1s = p.scale * kLog2e;
+    const float2 c1 = make_float2(c1s, c1s);
+    uint8_t* ds_box = smem + L::kDS + g * L::kTileBytes;          // this warpgroup's queries
+    uint8_t* stg = smem + L::kStg + (warp - kEpiWarp0) * 2048;   // this warp's dQ staging
+    bool ok = true;
+    // previous tile (its dQ is drained one tile late) and previous item (its dV / dK are
+    // read out at the first tile of the next item)
+    int prev_b = 0, prev_h = 0, prev_qt = 0;
+    WorkRef pit{};
+    bool have_item = false;
+    int t = 0, ii = 0;
+    // dQ of tile x (TMEM X[x % 2], columns [32g, 32g+32) of query row `row`) into the fp32
+    // accumulator: TMEM -> registers -> this warp's staging (16 rows at a time, 128-byte
+    // swizzle) -> TMA reduce-add
+    auto drain_dq = [&](int x, int b, int h, int qt, bool release) {
+      ok = ok && mbar_wait(dq_full + (x & 1), (x >> 1) & 1, wctx);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) return;
+      tc_fence_after();
+      uint32_t r[32];
+      tmem_ld32(t_lane + (x & 1) * 128 + 32 * g, r);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (release && lane == 0) mbar_arrive(x_free + (x & 1));
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        if ((lane >> 4) == half) {
+          const int rr = lane & 15;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(stg + rr * 128 + ((j ^ (rr & 7)) << 4)) =
+                make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_4d(&tdq, stg, 32 * g, qt * kTile + 32 * wq + 16 * half, h, b);
+          bulk_commit_group();
+          bulk_wait_read();
+        }
+        __syncwarp();
+      }
+    };
+    // dV / dK of item `x` (number ix) from TMEM to global memory, bf16
+    auto read_acc = [&](const WorkRef& x, int ix) {
+      ok = ok && mbar_wait(acc_full, ix & 1, wctx);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) return;
+      tc_fence_after();
+      uint32_t av[32], ak[32];
+      tmem_ld32(t_lane + kDV + 32 * g, av);
+      tmem_ld32(t_lane + kDK + 32 * g, ak);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      const int kg = x.t * kTile + row;
+      if (kg < p.Nk) {
+        uint4* dvp = reinterpret_cast<uint4*>(p.dv + x.b * p.dv_sb + static_cast<int64_t>(kg) * p.dv_sn +
+                                              x.h * p.dv_sh + 32 * g);
+        uint4* dkp = reinterpret_cast<uint4*>(p.dk + x.b * p.dk_sb + static_cast<int64_t>(kg) * p.dk_sn +
+                                              x.h * p.dk_sh + 32 * g);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t w0[4], w1[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = 8 * c + 2 * e;
+            w0[e] = pack_bf16x2(__uint_as_float(av[k]), __uint_as_float(av[k + 1]));
+            w1[e] = pack_bf16x2(__uint_as_float(ak[k]) * p.scale, __uint_as_float(ak[k + 1]) * p.scale);
+          }
+          dvp[c] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+          dkp[c] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+        }
+      }
+    };
+    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
+      if (it.n == 0) {
+        // No query attends to this k-tile: dK = dV = 0 on its rows.
+        const int rows = min(kTile, p.Nk - it.t * kTile);
+        const int tid = threadIdx.x - kEpiWarp0 * 32;
+        zero_rows<D>(p.dk + it.b * p.dk_sb + static_cast<int64_t>(it.t * kTile) * p.dk_sn +
+                         it.h * p.dk_sh, p.dk_sn, rows, tid, 256);
+        zero_rows<D>(p.dv + it.b * p.dv_sb + static_cast<int64_t>(it.t * kTile) * p.dv_sn +
+                         it.h * p.dv_sh, p.dv_sn, rows, tid, 256);
+        continue;
+      }
+      for (int i = 0; i < it.n; ++i, ++t) {
+        const int s = t % S;
+        // q_full of the stage also publishes the kind, bitmask and column vectors
+        if (ok) ok = mbar_wait(q_full + s, (t / S) & 1, wctx);
+        if (ok) ok = mbar_wait(sdp_full + (t & 1), (t >> 1) & 1, wctx);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+        if (meta_kind[s] == 2)
+          mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * g);
+        const float* vs = vec + s * 256 + 64 * g;
+        const int qt_cur = p.rowT_idx[it.e0 + i];
+        const uint32_t xb = t_lane + (t & 1) * 128 + 64 * g;
+        const uint32_t yb = t_lane + kY + 64 * g;
+        // four chunks of 16 queries; the TMEM loads of chunk c + 1 overlap the math of
+        // chunk c.  P and dS of chunk c overwrite its own S^T columns [16c, 16c+16): P in
+        // the first 8, dS in the last 8.
+        uint32_t sr[2][16], dpr[2][16];
+        tmem_ld16(xb, sr[0]);
+        tmem_ld16(yb, dpr[0]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c < 3) {
+            tmem_ld16(xb + 16 * (c + 1), sr[(c + 1) & 1]);
+            tmem_ld16(yb + 16 * (c + 1), dpr[(c + 1) & 1]);
+          }
+          const uint32_t mw = (c < 2 ? mb.x : mb.y) >> (16 * (c & 1));
+          uint32_t pk[8], dk[8];
+#pragma unroll
+          for (int cc = 0; cc < 16; cc += 2) {
+            float2 pw, ds;
+            const float2 off2 = *reinterpret_cast<const float2*>(vs + 16 * c + cc);
+            const float2 D2 = EPI == 0 ? make_float2(0.0f, 0.0f)
+                                       : *reinterpret_cast<const float2*>(vs + 128 + 16 * c + cc);
+            weight_grad2<EPI>(
+                make_float2(__uint_as_float(sr[c & 1][cc]), __uint_as_float(sr[c & 1][cc + 1])),
+                make_float2(__uint_as_float(dpr[c & 1][cc]), __uint_as_float(dpr[c & 1][cc + 1])),
+                c1, off2, D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
+            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
+            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+          }
+          tmem_st8(xb + 16 * c, pk);
+          tmem_st8(xb + 16 * c + 8, dk);
+          if (c < 3) tmem_wait_ld();
+          if (c == 2) {
+            // every dP^T column read: the next tile's dP^T may go into Y
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(y_free);
+          }
+        }
+        // dS into shared memory for the dQ MMA, once dQ of the previous tile has read it:
+        // row = key, 64 queries of this warpgroup, 128-byte swizzled (16-byte chunk j of row
+        // k at position j ^ (k % 8)).  The values are read back from TMEM rather than kept
+        // in registers across the wait.
+        if (t >= 1) ok = mbar_wait(dq_full + ((t - 1) & 1), ((t - 1) >> 1) & 1, wctx);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        {
+          uint32_t dsr[4][8];
+          tmem_wait_st();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld8(xb + 16 * c + 8, dsr[c]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t* w = &dsr[j >> 1][4 * (j & 1)];
+            *reinterpret_cast<uint4*>(ds_box + row * 128 + ((j ^ (row & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+        // dV / dK of the previous item leave TMEM before this tile's dV / dK MMAs may
+        // start a new accumulation
+        if (i == 0 && have_item) read_acc(pit, ii - 1);
+        if (!ok) break;
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + (t & 1));
+        // the previous tile's dQ (its MMA completed above): drain it, freeing X[(t-1) % 2]
+        if (t >= 1) drain_dq(t - 1, prev_b, prev_h, prev_qt, true);
+        prev_b = it.b;
+        prev_h = it.h;
+        prev_qt = qt_cur;
+      }
+      if (!ok) break;
+      pit = it;
+      have_item = true;
+      ++ii;
+    }
+    if (ok && t >= 1) drain_dq(t - 1, prev_b, prev_h, prev_qt, false);
+    if (ok && have_item) read_acc(pit, ii - 1);
+    if (lane == 0) bulk_wait_all();
+  }
+  // Single-lane roles (MMA issue, copy issue) end at different times than the rest of
+  // their warp: reconverge every warp before the CTA-wide barrier, which counts warps.
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Zeroes the fp32 dQ accumulator rows of every q-tile that has tiles (the others are never
+// read): rows qt*128 .. of batch entry b for each listed row r = b*QT + qt.
+__global__ void dq_zero_kernel(const int4* __restrict__ row_desc, int rows_nonempty, int QT, int Nq,
+                               int H, float* __restrict__ dqacc) {
+  constexpr int kVec = 64 / 4;  // float4 per (row, head), d = 64
+  const int64_t per_tile = static_cast<int64_t>(kTile) * H * kVec;
+  const int64_t total = per_tile * rows_nonempty;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int r = row_desc[i / per_tile].x;
+    const int64_t w = i % per_tile;
+    const int rr = static_cast<int>(w / (H * kVec));
+    const int b = r / QT, qt = r % QT;
+    const int q = qt * kTile + rr;
+    if (q >= Nq) continue;
+    const int64_t off = ((static_cast<int64_t>(b) * Nq + q) * H) * 64 + (w % (H * kVec)) * 4;
+    *reinterpret_cast<float4*>(dqacc + off) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  }
+}
+
+// dQ = bf16(scale * dQacc) on rows of q-tiles with tiles, 0 on every other row.  One thread
+// per 8 elements (16 bytes of dQ).
+__global__ void dq_convert_kernel(const int32_t* __restrict__ row_ptr, const float* __restrict__ dqacc,
+                                  int B, int QT, int Nq, int H, float scale,
+                                  __nv_bfloat16* __restrict__ dq, int64_t sb, int64_t sn, int64_t sh) {
+  constexpr int kChunks = 64 / 8;
+  const int64_t total = static_cast<int64_t>(B) * Nq * H * kChunks;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(i % kChunks);
+    const int h = static_cast<int>((i / kChunks) % H);
+    const int64_t bq = i / (static_cast<int64_t>(kChunks) * H);
+    const int q = static_cast<int>(bq % Nq), b = static_cast<int>(bq / Nq);
+    const int r = b * QT + q / kTile;
+    uint4 out = make_uint4(0u, 0u, 0u, 0u);
+    if (row_ptr[r + 1] > row_ptr[r]) {
+      const float4* src = reinterpret_cast<const float4*>(dqacc + (bq * H + h) * 64 + c * 8);
+      const float4 a = src[0], e = src[1];
+      out = make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
+                       pack_bf16x2(e.x * scale, e.y * scale), pack_bf16x2(e.z * scale, e.w * scale));
+    }
+    *reinterpret_cast<uint4*>(dq + b * sb + static_cast<int64_t>(q) * sn + h * sh + c * 8) = out;
+  }
+}
+
 int num_sms() {
   static int sms = 0;
   static std::once_flag once;
@@ -1435,6 +1966,83 @@ int launch_bwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
 
 }  // namespace
 
+int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float scale,
+                          const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, const CUtensorMap& tdq, const TensorDesc& o,
+                          const TensorDesc& dout, const float* bias, int64_t bias_sb,
+                          const float* lse, float* Dws, float* dqacc, const TensorDesc& dq,
+                          const TensorDesc& dk, const TensorDesc& dv, int* status,
+                          unsigned long long wait_ns, cudaStream_t stream) {
+  constexpr int D = 64;
+  BwdParams p{};
+  p.rowT_idx = plan->rowT_idx;
+  p.csc_map = plan->csc_map;
+  p.kind = plan->kind;
+  p.pidx = plan->pidx;
+  p.bitsT = plan->bitsT;
+  p.col_desc = plan->col_desc;
+  p.row_desc = plan->row_desc;
+  p.B = plan->B;
+  p.QT = plan->QT;
+  p.KT = plan->KT;
+  p.Nq = plan->Nq;
+  p.Nk = plan->Nk;
+  p.H = H;
+  p.scale = scale;
+  p.bias = bias;
+  p.bias_sb = bias_sb;
+  p.lse = lse;
+  p.Dws = Dws;
+  p.dk = static_cast<__nv_bfloat16*>(const_cast<void*>(dk.ptr));
+  p.dk_sb = dk.sb;
+  p.dk_sn = dk.sn;
+  p.dk_sh = dk.sh;
+  p.dv = static_cast<__nv_bfloat16*>(const_cast<void*>(dv.ptr));
+  p.dv_sb = dv.sb;
+  p.dv_sn = dv.sn;
+  p.dv_sh = dv.sh;
+  p.status = status;
+  p.wait_ns = wait_ns;
+  cudaError_t e;
+  if (epilogue != 0) {
+    const int64_t threads = static_cast<int64_t>(plan->B) * plan->Nq * H * (D / 8);
+    d_preprocess_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o.ptr), o.sb, o.sn, o.sh,
+        static_cast<const __nv_bfloat16*>(dout.ptr), dout.sb, dout.sn, dout.sh, plan->B, plan->Nq,
+        H, Dws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  }
+  const int sms = num_sms();
+  if (plan->rows_nonempty > 0) {
+    const int64_t work = static_cast<int64_t>(plan->rows_nonempty) * kTile * H * (D / 4);
+    const int blocks = static_cast<int>(std::min<int64_t>((work + 255) / 256, sms * 8));
+    dq_zero_kernel<<<blocks, 256, 0, stream>>>(plan->row_desc, plan->rows_nonempty, plan->QT,
+                                                plan->Nq, H, dqacc);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  }
+  static_assert(FusedLayout::kAlloc <= 227 * 1024, "shared memory");
+  {
+    auto kern = epilogue == 0 ? fused_bwd_kernel<0>
+                              : (epilogue == 1 ? fused_bwd_kernel<1> : fused_bwd_kernel<2>);
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  FusedLayout::kAlloc)) != cudaSuccess)
+      return cuda_status(e);
+    const int items = plan->B * plan->KT * H;
+    kern<<<std::min(items, sms), kThreads, FusedLayout::kAlloc, stream>>>(tq, tk, tv, tdo, tdq, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  }
+  {
+    const int64_t work = static_cast<int64_t>(plan->B) * plan->Nq * H * (D / 8);
+    const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, sms * 8)));
+    dq_convert_kernel<<<blocks, 256, 0, stream>>>(plan->row_ptr, dqacc, plan->B, plan->QT, plan->Nq,
+                                                   H, scale,
+                                                   static_cast<__nv_bfloat16*>(const_cast<void*>(dq.ptr)),
+                                                   dq.sb, dq.sn, dq.sh);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  }
+  return SIGATTN_OK;
+}
+
 int launch_bwd_impl(const sigattn_plan* plan, int epilogue, int H, int d, float scale,
                     const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     const CUtensorMap& tdo, const TensorDesc& o, const TensorDesc& dout,
@@ -1466,29 +2074,15 @@ static __device__ __align__(256) float g_noalloc_scratch[SIGATTN_NOALLOC_MAX_ROW
 
 namespace {
 
-constexpr int kNoAllocMaxDevices = 64;
-std::mutex g_noalloc_mu;
-float* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
+sigattn::SymbolAddressCache g_noalloc_addr;
 
-// Device address of g_noalloc_scratch on the current device.  In host code the array's
-// name is only a host-side stand-in, so the address is looked up once per device, with that
-// device current, and reused.
+// Device address of g_noalloc_scratch on the current device (looked up once per device,
+// with that device current; see SymbolAddressCache).
 int noalloc_scratch(float** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
-    cudaGetLastError();
-    return SIGATTN_ERR_NO_DEVICE;
-  }
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return SIGATTN_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    float* ptr = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_noalloc_scratch);
-    if (e != cudaSuccess) return sigattn::cuda_status(e);
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
-  return SIGATTN_OK;
+  void* p = nullptr;
+  const int rc = g_noalloc_addr.get(g_noalloc_scratch, &p);
+  *out = static_cast<float*>(p);
+  return rc;
 }
 
 }  // namespace

@@ -4,11 +4,14 @@
 // Method: "Better Models, Faster Training: Sigmoid Attention for single-cell Foundation
 // Models", section 2A: O = sigma(Q K^T / sqrt(d) + b) V, each weight computed on its own
 // with no row normalisation; section 2C: one fused kernel that skips every tile that is
-// padding on the query or the key side, with the sigmoid on the hardware tanh
-// approximation.  softmax and softmax_1 (the QuietAttention page, section "Proposition :
-// softmax_1 et QuietAttention") run through the same kernel with the online max / sum
-// recombination of the FlashAttention article (section on the mathematics of blockwise
-// softmax); softmax_1 starts from a zero logit whose value row is zero (m = 0, l = 1).
+// padding on the query or the key side.  The sigmoid is evaluated as in sm100.cuh
+// (sigmoid2: hardware exp2 plus a polynomial reciprocal, accurate in relative terms for
+// the tiny weights that b = -log n gives long sequences) instead of the page's hardware
+// tanh, which loses them.  softmax and softmax_1 (the QuietAttention page, section
+// "Proposition : softmax_1 et QuietAttention") run through the same kernel with the online
+// max / sum recombination of the FlashAttention article (section on the mathematics of
+// blockwise softmax); softmax_1 starts from a zero logit whose value row is zero (m = 0,
+// l = 1).
 //
 // Persistent: one CTA per SM walks the plan's longest-first list of (q-tile row, head)
 // work items in snake order (even rounds forward, odd rounds backward over the grid).
@@ -240,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0 && *abort_flag) {
       // Let the copies still in flight land before the CTA's shared memory goes away.
-      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
       for (int u = max(0, i - 2); u < i; ++u) mbar_wait(q_full + (u & 1), (u >> 1) & 1, drain);
       for (int u = max(0, t - S); u < t; ++u) {
         mbar_wait(k_full + u % S, (u / S) & 1, drain);
@@ -690,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0 && *abort_flag) {
       // Let the copies still in flight land before the CTA's shared memory goes away.
-      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
       if (role == 0)
         for (int u = max(0, i - 2); u < i; ++u) mbar_wait(q_full + (u & 1), (u >> 1) & 1, drain);
       for (int u = max(0, t - NR); u < t; ++u) mbar_wait(full + u % NR, (u / NR) & 1, drain);
@@ -780,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every MMA complete before the TMEM is released
       mma_commit_w(done);
-      const WaitCtx drain{p.status, p.wait_ns, drain_flag};
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
       mbar_wait_w(done, 0, drain);
     }
   } else if (warp >= kEpiWarp0) {
@@ -795,8 +798,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = wq * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     constexpr int kOc = D / 2;  // O columns written by this warpgroup
-    const float2 c1 = make_float2(0.5f * p.scale, 0.5f * p.scale);
-    const float2 half2 = make_float2(0.5f, 0.5f);
+    // t = x log2(e) = (scale s + bias) log2(e), the argument of sigmoid2
+    const float2 c1 = make_float2(p.scale * kLog2e, p.scale * kLog2e);
     bool ok = true;
     auto row_bias = [&](const Item& x) {
       const int r = x.qt * kTile + row;
@@ -859,7 +862,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         continue;
       }
-      const float2 c0 = make_float2(0.5f * bias_r, 0.5f * bias_r);
+      const float2 c0 = make_float2(bias_r * kLog2e, bias_r * kLog2e);
       const int t_end = t + it.n;
       for (int tt = t + ((t & 1) != g ? 1 : 0); tt < t_end; tt += 2) {
         const int ms = tt % SM;
@@ -884,15 +887,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int cc = 0; cc < 32; cc += 2) {
-            const float2 x = fma2(make_float2(__uint_as_float(buf[c & 1][cc]),
-                                              __uint_as_float(buf[c & 1][cc + 1])),
-                                  c1, c0);
-            float2 th = make_float2(tanh_approx(x.x), tanh_approx(x.y));
+            float2 x = fma2(make_float2(__uint_as_float(buf[c & 1][cc]),
+                                        __uint_as_float(buf[c & 1][cc + 1])),
+                            c1, c0);
             if (masked) {
-              th.x = ((mw >> cc) & 1u) ? th.x : -1.0f;
-              th.y = ((mw >> (cc + 1)) & 1u) ? th.y : -1.0f;
+              x.x = ((mw >> cc) & 1u) ? x.x : -INFINITY;
+              x.y = ((mw >> (cc + 1)) & 1u) ? x.y : -INFINITY;
             }
-            const float2 pw = fma2(th, half2, half2);
+            const float2 pw = sigmoid2(x);
             pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
           }
           tmem_st16(sp + (c >> 1) * 64 + (c & 1) * 16, pk);

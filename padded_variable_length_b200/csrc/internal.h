@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "sigattn.h"
 
 // Device buffers of a tile plan.  Layouts are those of sigattn_plan_export; in addition
@@ -14,6 +16,7 @@
 //   col_work[B*KT]  every (b, k-tile) column, columns with no tile last
 struct sigattn_plan {
   int device;
+  void* arena[2];  // the two device allocations every buffer below is carved from
   int B, Nq, Nk, QT, KT;
   int64_t nonempty, full, partial;
   int32_t rows_nonempty, cols_nonempty;
@@ -32,6 +35,11 @@ struct sigattn_plan {
   // number of entries, 0}, so that a kernel decodes a work item with one independent load
   int4* row_desc;
   int4* col_desc;
+  // runs of each q-tile row: maximal ranges of consecutive k-tiles of one kind, one 16-byte
+  // record each {first k-tile, number of tiles, kind, first CSR entry}; row r's runs are
+  // run[run_ptr[r] .. run_ptr[r+1])
+  int32_t* run_ptr;
+  int4* run;
 };
 
 namespace sigattn {
@@ -49,6 +57,43 @@ struct TensorDesc {
 // 64 (d) x 128 (tokens) x 1 x 1 and 128-byte swizzle.
 int make_tmap_bf16(CUtensorMap* map, const TensorDesc& t, int B, int H, int d);
 
+// 4-D TMA descriptor over a contiguous fp32 [B, N, H, d] tensor with a box of 32 (d) x 16
+// (tokens) x 1 x 1 and 128-byte swizzle (the fused backward's dQ accumulator).
+int make_tmap_f32_acc(CUtensorMap* map, float* base, int B, int N, int H, int d);
+
 int cuda_status(cudaError_t e);
+
+// Per-device cache of the device address of one file-scope __device__ variable.  In host
+// code such a variable's name is only a host-side stand-in, so its address is looked up with
+// cudaGetSymbolAddress once per device, with that device current, and reused.  The cache
+// lives as long as the process: a cudaDeviceReset invalidates the addresses it holds (this
+// library does not support resetting a device it has been used on).
+constexpr int kMaxDevices = 64;
+
+struct SymbolAddressCache {
+  std::mutex mu;
+  void* addr[kMaxDevices] = {nullptr};
+
+  // *out = the symbol's address on the current device.  Errors: NO_DEVICE, UNSUPPORTED
+  // (device ordinal past kMaxDevices), CUDA.
+  template <class T>
+  int get(const T& symbol, void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+      cudaGetLastError();
+      return SIGATTN_ERR_NO_DEVICE;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return SIGATTN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+      void* p = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&p, symbol);
+      if (e != cudaSuccess) return cuda_status(e);
+      addr[dev] = p;
+    }
+    *out = addr[dev];
+    return SIGATTN_OK;
+  }
+};
 
 }  // namespace sigattn

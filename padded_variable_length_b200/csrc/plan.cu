@@ -112,157 +112,197 @@ __global__ void __launch_bounds__(256) k_kinds_from_mask(const uint8_t* __restri
   if (threadIdx.x == 0) kinds[blk] = all_b ? 1 : (any_b ? 2 : 0);
 }
 
-// One warp per q-tile row: number of listed blocks and of PARTIAL blocks.
-__global__ void k_count_rows(const uint8_t* __restrict__ kinds, int rows, int KT,
-                             int32_t* __restrict__ cnt, int32_t* __restrict__ pcnt) {
+// One warp per q-tile row r < rows (number of listed blocks and of PARTIAL blocks), then
+// one warp per k-tile column c = b*KT + kt (number of listed blocks).
+__global__ void k_count(const uint8_t* __restrict__ kinds, int B, int QT, int KT,
+                        int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_pcnt,
+                        int32_t* __restrict__ col_cnt) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= rows) return;
-  const uint8_t* k = kinds + static_cast<int64_t>(warp) * KT;
-  int c = 0, p = 0;
-  for (int kt = lane; kt < KT; kt += 32) {
-    const uint8_t v = k[kt];
-    c += v != 0;
-    p += v == 2;
-  }
+  const int rows = B * QT;
+  if (warp < rows) {
+    const uint8_t* k = kinds + static_cast<int64_t>(warp) * KT;
+    int c = 0, p = 0;
+    for (int kt = lane; kt < KT; kt += 32) {
+      const uint8_t v = k[kt];
+      c += v != 0;
+      p += v == 2;
+    }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
-    p += __shfl_xor_sync(0xFFFFFFFFu, p, o);
+    for (int o = 16; o > 0; o >>= 1) {
+      c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+      p += __shfl_xor_sync(0xFFFFFFFFu, p, o);
+    }
+    if (lane == 0) {
+      row_cnt[warp] = c;
+      row_pcnt[warp] = p;
+    }
+    return;
   }
-  if (lane == 0) {
-    cnt[warp] = c;
-    pcnt[warp] = p;
-  }
-}
-
-// One warp per k-tile column c = b*KT + kt.
-__global__ void k_count_cols(const uint8_t* __restrict__ kinds, int B, int QT, int KT,
-                             int32_t* __restrict__ cnt) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= B * KT) return;
-  const int b = warp / KT, kt = warp % KT;
+  const int col = warp - rows;
+  if (col >= B * KT) return;
+  const int b = col / KT, kt = col % KT;
   int c = 0;
   for (int qt = lane; qt < QT; qt += 32) c += kinds[(static_cast<int64_t>(b) * QT + qt) * KT + kt] != 0;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
-  if (lane == 0) cnt[warp] = c;
+  if (lane == 0) col_cnt[col] = c;
 }
 
-// Exclusive scan of in[0..n) into out[0..n]; out[n] is the total, also stored to *total.
-// One CTA of 1024 threads walking the input in chunks.
-__global__ void __launch_bounds__(1024) k_scan(const int32_t* __restrict__ in, int n,
-                                               int32_t* __restrict__ out, int64_t* total) {
-  __shared__ int32_t warp_sums[32];
-  __shared__ int32_t carry;
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
+// Inclusive scan over the 1024 threads of a CTA (every thread must call it).
+__device__ __forceinline__ int block_inclusive_scan(int x, int32_t* warp_sums) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int base = 0; base < n; base += 1024) {
-    const int i = base + threadIdx.x;
-    const int x = i < n ? in[i] : 0;
-    int incl = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) warp_sums[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      int s = warp_sums[lane];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xFFFFFFFFu, s, o);
-        if (lane >= o) s += y;
-      }
-      warp_sums[lane] = s;  // inclusive over warps
-    }
-    __syncthreads();
-    const int before = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + incl - x;
-    if (i < n) out[i] = before;
-    __syncthreads();
-    if (threadIdx.x == 0) carry += warp_sums[31];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
-    out[n] = carry;
-    if (total) *total = carry;
-  }
-}
-
-// Stable counting sort of indices 0..n-1 by cnt[i] descending (counts past 4094 share a
-// bucket).  One warp.  Also stores the number of nonzero counts to *nonzero.
-__global__ void __launch_bounds__(32) k_sort_longest_first(const int32_t* __restrict__ cnt, int n,
-                                                           int32_t* __restrict__ out,
-                                                           int64_t* nonzero) {
-  __shared__ int32_t start[kSortBuckets];
-  const int lane = threadIdx.x;
-  for (int i = lane; i < kSortBuckets; i += 32) start[i] = 0;
-  __syncwarp();
-  int nz = 0;
-  // key = kSortBuckets - 1 - min(cnt, kSortBuckets - 1): ascending key = descending count
-  for (int i = lane; i < n; i += 32) {
-    const int c = cnt[i];
-    nz += c > 0;
-    atomicAdd(&start[kSortBuckets - 1 - min(c, kSortBuckets - 1)], 1);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) nz += __shfl_xor_sync(0xFFFFFFFFu, nz, o);
-  __syncwarp();
-  // exclusive scan over the buckets: lane l owns buckets [l*128, l*128+128)
-  constexpr int per = kSortBuckets / 32;
-  int sum = 0;
-  for (int j = 0; j < per; ++j) sum += start[lane * per + j];
-  int incl = sum;
+  int incl = x;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
     if (lane >= o) incl += y;
   }
-  int run = incl - sum;
-  __syncwarp();
-  for (int j = 0; j < per; ++j) {
-    const int c = start[lane * per + j];
-    start[lane * per + j] = run;
-    run += c;
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int s = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, s, o);
+      if (lane >= o) s += y;
+    }
+    warp_sums[lane] = s;  // inclusive over warps
   }
-  __syncwarp();
-  for (int base = 0; base < n; base += 32) {
-    const int i = base + lane;
-    const bool act = i < n;
-    const int key = act ? kSortBuckets - 1 - min(cnt[i], kSortBuckets - 1) : -1 - lane;
+  __syncthreads();
+  const int r = incl + (warp > 0 ? warp_sums[warp - 1] : 0);
+  __syncthreads();  // warp_sums is reused by the next call
+  return r;
+}
+
+// Exclusive scan of in[0..n) into out[0..n]; out[n] is the total, also stored to *total.
+struct ScanJob {
+  const int32_t* in;
+  int n;
+  int32_t* out;
+  int64_t* total;
+};
+
+// One CTA of 1024 threads per job (blockIdx.x picks one of three), walking its input in
+// chunks of 1024.
+__global__ void __launch_bounds__(1024) k_scan3(ScanJob j0, ScanJob j1, ScanJob j2) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t chunk_total;
+  const ScanJob j = blockIdx.x == 0 ? j0 : (blockIdx.x == 1 ? j1 : j2);
+  int carry = 0;
+  for (int base = 0; base < j.n; base += 1024) {
+    const int i = base + threadIdx.x;
+    const int x = i < j.n ? j.in[i] : 0;
+    const int incl = block_inclusive_scan(x, warp_sums);
+    if (i < j.n) j.out[i] = carry + incl - x;
+    if (threadIdx.x == 1023) chunk_total = incl;
+    __syncthreads();
+    carry += chunk_total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    j.out[j.n] = carry;
+    if (j.total) *j.total = carry;
+  }
+}
+
+// Stable counting sort of indices 0..n-1 by cnt[i] descending (counts past 4094 share a
+// bucket); also stores the number of nonzero counts to *nonzero.
+struct SortJob {
+  const int32_t* cnt;
+  int n;
+  int32_t* out;
+  int64_t* nonzero;
+};
+
+__device__ __forceinline__ int sort_key(int c) {
+  return kSortBuckets - 1 - min(c, kSortBuckets - 1);  // ascending key = descending count
+}
+
+// One CTA of 1024 threads per job (blockIdx.x picks one of two).  Histogram and bucket
+// offsets in shared memory; then the indices are placed in chunks of 1024 in index order:
+// equal keys within a warp are ranked by lane (match), and the 32 warps of a chunk claim
+// their slots one after another, so that the order of equal keys is the index order.
+__global__ void __launch_bounds__(1024) k_sort_longest_first(SortJob j0, SortJob j1) {
+  __shared__ int32_t start[kSortBuckets];
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t nz_total;
+  const SortJob j = blockIdx.x == 0 ? j0 : j1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < kSortBuckets; i += 1024) start[i] = 0;
+  if (tid == 0) nz_total = 0;
+  __syncthreads();
+  int nz = 0;
+  for (int i = tid; i < j.n; i += 1024) {
+    const int c = j.cnt[i];
+    nz += c > 0;
+    atomicAdd(&start[sort_key(c)], 1);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) nz += __shfl_xor_sync(0xFFFFFFFFu, nz, o);
+  if (lane == 0) atomicAdd(&nz_total, nz);
+  __syncthreads();
+  // exclusive scan over the buckets: thread t owns buckets [4t, 4t + 4)
+  static_assert(kSortBuckets == 4 * 1024, "four buckets per thread");
+  int v[4], sum = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    v[k] = start[4 * tid + k];
+    sum += v[k];
+  }
+  int run = block_inclusive_scan(sum, warp_sums) - sum;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    start[4 * tid + k] = run;
+    run += v[k];
+  }
+  __syncthreads();
+  for (int base = 0; base < j.n; base += 1024) {
+    const int i = base + tid;
+    const bool act = i < j.n;
+    const int key = act ? sort_key(j.cnt[i]) : -1 - lane;
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
     const int rank = __popc(peers & ((1u << lane) - 1u));
-    int pos = 0;
-    if (act) pos = start[key] + rank;
-    __syncwarp();
-    if (act) {
-      out[pos] = i;
-      if (rank == 0) start[key] += __popc(peers);
+    const int leader = __ffs(peers) - 1;
+    int first = 0;
+    for (int w = 0; w < 32; ++w) {
+      if (warp == w && act && rank == 0) {
+        first = start[key];
+        start[key] = first + __popc(peers);
+      }
+      __syncthreads();
     }
-    __syncwarp();
+    const int pos = __shfl_sync(0xFFFFFFFFu, first, leader) + rank;
+    if (act) j.out[pos] = i;
   }
-  if (lane == 0 && nonzero) *nonzero = nz;
+  if (tid == 0 && j.nonzero) *j.nonzero = nz_total;
 }
 
 // One warp per q-tile row: CSR entries in ascending kt, the PARTIAL numbering, the dense
 // entry index of every listed block and the block of every PARTIAL number.
+// A listed block starts a run iff the block before it in the row is not listed or of the
+// other kind (runs: maximal ranges of consecutive k-tiles of one kind).  Also counts the
+// runs of every row into run_cnt.
 __global__ void k_fill_csr(const uint8_t* __restrict__ kinds, int rows, int KT,
                            const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ row_poff,
                            int32_t* __restrict__ col_idx, uint8_t* __restrict__ kind,
                            int32_t* __restrict__ pidx, int32_t* __restrict__ eidx,
-                           int64_t* __restrict__ ptile) {
+                           int64_t* __restrict__ ptile, int32_t* __restrict__ run_cnt) {
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
   int e = row_ptr[r];
   int p = row_poff[r];
+  int runs = 0;
+  uint8_t carry = 0;  // kind of the block before this chunk
   const uint8_t* k = kinds + static_cast<int64_t>(r) * KT;
   for (int base = 0; base < KT; base += 32) {
     const int kt = base + lane;
     const uint8_t v = kt < KT ? k[kt] : 0;
+    const uint8_t before = static_cast<uint8_t>(__shfl_up_sync(0xFFFFFFFFu, v, 1));
+    const uint8_t prev = lane == 0 ? carry : before;
+    carry = static_cast<uint8_t>(__shfl_sync(0xFFFFFFFFu, v, 31));
+    runs += __popc(__ballot_sync(0xFFFFFFFFu, v != 0 && v != prev));
     const unsigned nzm = __ballot_sync(0xFFFFFFFFu, v != 0);
     const unsigned pm = __ballot_sync(0xFFFFFFFFu, v == 2);
     const unsigned lt = (1u << lane) - 1u;
@@ -281,6 +321,40 @@ __global__ void k_fill_csr(const uint8_t* __restrict__ kinds, int rows, int KT,
     }
     e += __popc(nzm);
     p += __popc(pm);
+  }
+  if (lane == 0) run_cnt[r] = runs;
+}
+
+// One warp per q-tile row: its runs {first k-tile, number of tiles, kind, first CSR entry}
+// in ascending order, at run[run_ptr[r] ..).
+__global__ void k_fill_runs(const uint8_t* __restrict__ kinds, const int32_t* __restrict__ eidx,
+                            int rows, int KT, const int32_t* __restrict__ row_ptr,
+                            const int32_t* __restrict__ run_ptr, int4* __restrict__ run) {
+  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  int pos = run_ptr[r];
+  uint8_t carry = 0;
+  const uint8_t* k = kinds + static_cast<int64_t>(r) * KT;
+  for (int base = 0; base < KT; base += 32) {
+    const int kt = base + lane;
+    const uint8_t v = kt < KT ? k[kt] : 0;
+    const uint8_t before = static_cast<uint8_t>(__shfl_up_sync(0xFFFFFFFFu, v, 1));
+    const uint8_t prev = lane == 0 ? carry : before;
+    carry = static_cast<uint8_t>(__shfl_sync(0xFFFFFFFFu, v, 31));
+    const bool start = v != 0 && v != prev;
+    const unsigned sm = __ballot_sync(0xFFFFFFFFu, start);
+    if (start)
+      run[pos + __popc(sm & ((1u << lane) - 1u))] =
+          make_int4(kt, 0, v, eidx[static_cast<int64_t>(r) * KT + kt]);
+    pos += __popc(sm);
+  }
+  __syncwarp();
+  // length = first entry of the next run (or the row's end) minus the run's first entry
+  const int a = run_ptr[r], b = run_ptr[r + 1], end = row_ptr[r + 1];
+  for (int j = a + lane; j < b; j += 32) {
+    const int next = j + 1 < b ? run[j + 1].w : end;
+    run[j].y = next - run[j].w;
   }
 }
 
@@ -346,13 +420,20 @@ __global__ void __launch_bounds__(128) k_bits_from_lengths(const int32_t* __rest
   reinterpret_cast<uint4*>(bits + static_cast<int64_t>(blockIdx.x) * 512)[q] = w;
 }
 
-// desc[k] = {work[k], ptr[work[k]], ptr[work[k] + 1] - ptr[work[k]], 0}
-__global__ void k_work_desc(const int32_t* __restrict__ work, const int32_t* __restrict__ ptr, int n,
-                            int4* __restrict__ desc) {
-  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) {
-    const int r = work[k];
+// desc[k] = {work[k], ptr[work[k]], ptr[work[k] + 1] - ptr[work[k]], 0} for the row list
+// (k < rows) and then the column list.
+__global__ void k_work_desc(const int32_t* __restrict__ row_work, const int32_t* __restrict__ row_ptr,
+                            int rows, int4* __restrict__ row_desc,
+                            const int32_t* __restrict__ col_work,
+                            const int32_t* __restrict__ col_ptr, int cols,
+                            int4* __restrict__ col_desc) {
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < rows + cols; k += gridDim.x * blockDim.x) {
+    const bool is_row = k < rows;
+    const int kk = is_row ? k : k - rows;
+    const int r = (is_row ? row_work : col_work)[kk];
+    const int32_t* ptr = is_row ? row_ptr : col_ptr;
     const int a = ptr[r];
-    desc[k] = make_int4(r, a, ptr[r + 1] - a, 0);
+    (is_row ? row_desc : col_desc)[kk] = make_int4(r, a, ptr[r + 1] - a, 0);
   }
 }
 
@@ -370,33 +451,43 @@ __global__ void __launch_bounds__(128) k_transpose_bits(const uint32_t* __restri
       make_uint4(out[0], out[1], out[2], out[3]);
 }
 
-template <class T>
-int dev_alloc(T** p, size_t count) {
-  *p = nullptr;
-  if (count == 0) return SIGATTN_OK;
-  const cudaError_t e = cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T));
-  if (e != cudaSuccess) {
-    *p = nullptr;
-    cudaGetLastError();
-    return e == cudaErrorMemoryAllocation ? SIGATTN_ERR_NOMEM : SIGATTN_ERR_CUDA;
+// Buffers are carved out of a few large allocations: a byte count laid out first (every
+// buffer 256-byte aligned), then one allocation, then the pointers.
+struct Carve {
+  size_t bytes = 0;
+  template <class T>
+  size_t add(size_t count) {
+    bytes = (bytes + 255) & ~size_t(255);
+    const size_t at = bytes;
+    bytes += count * sizeof(T);
+    return at;
   }
-  return SIGATTN_OK;
+  template <class T>
+  static T* at(void* base, size_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
+  }
+};
+
+int alloc_status(cudaError_t e) {
+  if (e == cudaSuccess) return SIGATTN_OK;
+  cudaGetLastError();
+  return e == cudaErrorMemoryAllocation ? SIGATTN_ERR_NOMEM : SIGATTN_ERR_CUDA;
 }
 
-template <class T>
-int scratch_alloc(T** p, size_t count, cudaStream_t s) {
+// Plan memory (owned by the plan until sigattn_plan_destroy): cudaMalloc.
+int plan_alloc(void** p, size_t bytes) {
   *p = nullptr;
-  if (count == 0) count = 1;
-  const cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(p), count * sizeof(T), s);
-  if (e != cudaSuccess) {
-    *p = nullptr;
-    cudaGetLastError();
-    return e == cudaErrorMemoryAllocation ? SIGATTN_ERR_NOMEM : SIGATTN_ERR_CUDA;
-  }
-  return SIGATTN_OK;
+  return alloc_status(cudaMalloc(p, bytes > 0 ? bytes : 256));
+}
+
+// Scratch of one plan build: stream-ordered, released on the stream at the end.
+int scratch_alloc(void** p, size_t bytes, cudaStream_t s) {
+  *p = nullptr;
+  return alloc_status(cudaMallocAsync(p, bytes > 0 ? bytes : 256, s));
 }
 
 struct Scratch {
+  void* block[2] = {nullptr, nullptr};
   uint8_t* kinds = nullptr;
   int32_t* eidx = nullptr;
   int32_t* row_cnt = nullptr;
@@ -404,20 +495,21 @@ struct Scratch {
   int32_t* row_poff = nullptr;
   int32_t* col_cnt = nullptr;
   int64_t* totals = nullptr;
+  int32_t* run_cnt = nullptr;
   int64_t* ptile = nullptr;
   void release(cudaStream_t s) {
-    void* ps[] = {kinds, eidx, row_cnt, row_pcnt, row_poff, col_cnt, totals, ptile};
-    for (void* p : ps)
+    for (void*& p : block) {
       if (p) cudaFreeAsync(p, s);
+      p = nullptr;
+    }
   }
 };
 
 void plan_free_buffers(sigattn_plan* p) {
-  void* ps[] = {p->row_ptr, p->col_idx, p->kind,     p->pidx,     p->colT_ptr, p->rowT_idx,
-                p->csc_map, p->bits,    p->bitsT,    p->row_work, p->col_work, p->row_desc,
-                p->col_desc};
-  for (void* q : ps)
-    if (q) cudaFree(q);
+  for (void*& a : p->arena) {
+    if (a) cudaFree(a);
+    a = nullptr;
+  }
 }
 
 #define SIGATTN_TRY(x)            \
@@ -438,39 +530,63 @@ int grid_for(int64_t work, int per_block) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(g, 1 << 30)));
 }
 
-// Shared tail of both planners: kinds are in sc.kinds; `bits_kernel` fills bitmasks.
-template <class BitsFn>
-int finish_plan(sigattn_plan* plan, Scratch& sc, cudaStream_t stream, BitsFn bits_kernel,
-                sigattn_plan** out) {
+// Both planners: `classify` writes every block's kind into sc.kinds, `bits_kernel` the
+// bitmasks of the PARTIAL blocks.  Two plan allocations (one sized by the grid, one by the
+// number of listed tiles, known after the one synchronisation), two scratch allocations.
+template <class ClassifyFn, class BitsFn>
+int build_plan(sigattn_plan* plan, cudaStream_t stream, ClassifyFn classify, BitsFn bits_kernel,
+               sigattn_plan** out) {
+  Scratch sc;
   const int B = plan->B, QT = plan->QT, KT = plan->KT;
   const int rows = B * QT, cols = B * KT;
-  SIGATTN_TRY(dev_alloc(&plan->row_ptr, rows + 1));
-  SIGATTN_TRY(dev_alloc(&plan->colT_ptr, cols + 1));
-  SIGATTN_TRY(dev_alloc(&plan->row_work, rows));
-  SIGATTN_TRY(dev_alloc(&plan->col_work, cols));
-  SIGATTN_TRY(dev_alloc(&plan->row_desc, rows));
-  SIGATTN_TRY(dev_alloc(&plan->col_desc, cols));
-  SIGATTN_TRY(scratch_alloc(&sc.row_cnt, rows, stream));
-  SIGATTN_TRY(scratch_alloc(&sc.row_pcnt, rows, stream));
-  SIGATTN_TRY(scratch_alloc(&sc.row_poff, rows + 1, stream));
-  SIGATTN_TRY(scratch_alloc(&sc.col_cnt, cols, stream));
-  SIGATTN_TRY(scratch_alloc(&sc.totals, 8, stream));
-  k_count_rows<<<grid_for(static_cast<int64_t>(rows) * 32, 256), 256, 0, stream>>>(
-      sc.kinds, rows, KT, sc.row_cnt, sc.row_pcnt);
-  k_count_cols<<<grid_for(static_cast<int64_t>(cols) * 32, 256), 256, 0, stream>>>(
-      sc.kinds, B, QT, KT, sc.col_cnt);
-  k_scan<<<1, 1024, 0, stream>>>(sc.row_cnt, rows, plan->row_ptr, sc.totals + 0);
-  k_scan<<<1, 1024, 0, stream>>>(sc.row_pcnt, rows, sc.row_poff, sc.totals + 1);
-  k_scan<<<1, 1024, 0, stream>>>(sc.col_cnt, cols, plan->colT_ptr, nullptr);
-  k_sort_longest_first<<<1, 32, 0, stream>>>(sc.row_cnt, rows, plan->row_work, sc.totals + 2);
-  k_sort_longest_first<<<1, 32, 0, stream>>>(sc.col_cnt, cols, plan->col_work, sc.totals + 3);
-  k_work_desc<<<grid_for(rows, 256), 256, 0, stream>>>(plan->row_work, plan->row_ptr, rows,
-                                                        plan->row_desc);
-  k_work_desc<<<grid_for(cols, 256), 256, 0, stream>>>(plan->col_work, plan->colT_ptr, cols,
-                                                        plan->col_desc);
+  const int64_t grid_total = static_cast<int64_t>(rows) * KT;
+  {
+    Carve c;
+    const size_t o_kinds = c.add<uint8_t>(grid_total), o_eidx = c.add<int32_t>(grid_total),
+                 o_rc = c.add<int32_t>(rows), o_rp = c.add<int32_t>(rows),
+                 o_ro = c.add<int32_t>(rows + 1), o_cc = c.add<int32_t>(cols),
+                 o_tot = c.add<int64_t>(8), o_run = c.add<int32_t>(rows);
+    SIGATTN_TRY(scratch_alloc(&sc.block[0], c.bytes, stream));
+    void* m = sc.block[0];
+    sc.kinds = Carve::at<uint8_t>(m, o_kinds);
+    sc.eidx = Carve::at<int32_t>(m, o_eidx);
+    sc.row_cnt = Carve::at<int32_t>(m, o_rc);
+    sc.row_pcnt = Carve::at<int32_t>(m, o_rp);
+    sc.row_poff = Carve::at<int32_t>(m, o_ro);
+    sc.col_cnt = Carve::at<int32_t>(m, o_cc);
+    sc.totals = Carve::at<int64_t>(m, o_tot);
+    sc.run_cnt = Carve::at<int32_t>(m, o_run);
+  }
+  {
+    Carve c;
+    const size_t o_rptr = c.add<int32_t>(rows + 1), o_cptr = c.add<int32_t>(cols + 1),
+                 o_rw = c.add<int32_t>(rows), o_cw = c.add<int32_t>(cols),
+                 o_rd = c.add<int4>(rows), o_cd = c.add<int4>(cols),
+                 o_rp = c.add<int32_t>(rows + 1);
+    SIGATTN_TRY(plan_alloc(&plan->arena[0], c.bytes));
+    void* m = plan->arena[0];
+    plan->row_ptr = Carve::at<int32_t>(m, o_rptr);
+    plan->colT_ptr = Carve::at<int32_t>(m, o_cptr);
+    plan->row_work = Carve::at<int32_t>(m, o_rw);
+    plan->col_work = Carve::at<int32_t>(m, o_cw);
+    plan->row_desc = Carve::at<int4>(m, o_rd);
+    plan->col_desc = Carve::at<int4>(m, o_cd);
+    plan->run_ptr = Carve::at<int32_t>(m, o_rp);
+  }
+  classify(sc.kinds);
+  k_count<<<grid_for(static_cast<int64_t>(rows + cols) * 32, 256), 256, 0, stream>>>(
+      sc.kinds, B, QT, KT, sc.row_cnt, sc.row_pcnt, sc.col_cnt);
+  k_scan3<<<3, 1024, 0, stream>>>(ScanJob{sc.row_cnt, rows, plan->row_ptr, sc.totals + 0},
+                                  ScanJob{sc.row_pcnt, rows, sc.row_poff, sc.totals + 1},
+                                  ScanJob{sc.col_cnt, cols, plan->colT_ptr, nullptr});
+  k_sort_longest_first<<<2, 1024, 0, stream>>>(SortJob{sc.row_cnt, rows, plan->row_work, sc.totals + 2},
+                                               SortJob{sc.col_cnt, cols, plan->col_work, sc.totals + 3});
+  k_work_desc<<<grid_for(rows + cols, 256), 256, 0, stream>>>(
+      plan->row_work, plan->row_ptr, rows, plan->row_desc, plan->col_work, plan->colT_ptr, cols,
+      plan->col_desc);
   SIGATTN_TRY_CUDA(cudaGetLastError());
-  int64_t totals[8] = {0};
-  SIGATTN_TRY_CUDA(cudaMemcpyAsync(totals, sc.totals, 4 * sizeof(int64_t), cudaMemcpyDeviceToHost,
+  int64_t totals[4] = {0, 0, 0, 0};
+  SIGATTN_TRY_CUDA(cudaMemcpyAsync(totals, sc.totals, sizeof(totals), cudaMemcpyDeviceToHost,
                                    stream));
   SIGATTN_TRY_CUDA(cudaStreamSynchronize(stream));
   plan->nonempty = totals[0];
@@ -478,21 +594,38 @@ int finish_plan(sigattn_plan* plan, Scratch& sc, cudaStream_t stream, BitsFn bit
   plan->full = totals[0] - totals[1];
   plan->rows_nonempty = static_cast<int32_t>(totals[2]);
   plan->cols_nonempty = static_cast<int32_t>(totals[3]);
-  SIGATTN_TRY(dev_alloc(&plan->col_idx, plan->nonempty));
-  SIGATTN_TRY(dev_alloc(&plan->kind, plan->nonempty));
-  SIGATTN_TRY(dev_alloc(&plan->pidx, plan->nonempty));
-  SIGATTN_TRY(dev_alloc(&plan->rowT_idx, plan->nonempty));
-  SIGATTN_TRY(dev_alloc(&plan->csc_map, plan->nonempty));
-  SIGATTN_TRY(dev_alloc(&plan->bits, static_cast<size_t>(plan->partial) * 512));
-  SIGATTN_TRY(dev_alloc(&plan->bitsT, static_cast<size_t>(plan->partial) * 512));
-  SIGATTN_TRY(scratch_alloc(&sc.eidx, static_cast<size_t>(rows) * KT, stream));
-  SIGATTN_TRY(scratch_alloc(&sc.ptile, static_cast<size_t>(plan->partial), stream));
+  const size_t nz = static_cast<size_t>(plan->nonempty), np = static_cast<size_t>(plan->partial);
+  {
+    Carve c;
+    const size_t o_ci = c.add<int32_t>(nz), o_k = c.add<uint8_t>(nz), o_pi = c.add<int32_t>(nz),
+                 o_ri = c.add<int32_t>(nz), o_cm = c.add<int32_t>(nz),
+                 o_b = c.add<uint32_t>(np * 512), o_bt = c.add<uint32_t>(np * 512),
+                 o_run = c.add<int4>(nz);  // at most one run per listed tile
+    SIGATTN_TRY(plan_alloc(&plan->arena[1], c.bytes));
+    void* m = plan->arena[1];
+    plan->col_idx = Carve::at<int32_t>(m, o_ci);
+    plan->kind = Carve::at<uint8_t>(m, o_k);
+    plan->pidx = Carve::at<int32_t>(m, o_pi);
+    plan->rowT_idx = Carve::at<int32_t>(m, o_ri);
+    plan->csc_map = Carve::at<int32_t>(m, o_cm);
+    plan->bits = Carve::at<uint32_t>(m, o_b);
+    plan->bitsT = Carve::at<uint32_t>(m, o_bt);
+    plan->run = Carve::at<int4>(m, o_run);
+  }
+  SIGATTN_TRY(scratch_alloc(&sc.block[1], np * sizeof(int64_t), stream));
+  sc.ptile = static_cast<int64_t*>(sc.block[1]);
   if (plan->nonempty > 0) {
     k_fill_csr<<<grid_for(static_cast<int64_t>(rows) * 32, 256), 256, 0, stream>>>(
         sc.kinds, rows, KT, plan->row_ptr, sc.row_poff, plan->col_idx, plan->kind, plan->pidx,
-        sc.eidx, sc.ptile);
+        sc.eidx, sc.ptile, sc.run_cnt);
     k_fill_csc<<<grid_for(static_cast<int64_t>(cols) * 32, 256), 256, 0, stream>>>(
         sc.kinds, sc.eidx, B, QT, KT, plan->colT_ptr, plan->rowT_idx, plan->csc_map);
+    const ScanJob runs{sc.run_cnt, rows, plan->run_ptr, nullptr};
+    k_scan3<<<1, 1024, 0, stream>>>(runs, runs, runs);
+    k_fill_runs<<<grid_for(static_cast<int64_t>(rows) * 32, 256), 256, 0, stream>>>(
+        sc.kinds, sc.eidx, rows, KT, plan->row_ptr, plan->run_ptr, plan->run);
+  } else {
+    SIGATTN_TRY_CUDA(cudaMemsetAsync(plan->run_ptr, 0, (rows + 1) * sizeof(int32_t), stream));
   }
   if (plan->partial > 0) {
     bits_kernel(sc.ptile, plan->bits, static_cast<int>(plan->partial));
@@ -536,13 +669,14 @@ extern "C" int sigattn_plan_from_lengths(const int32_t* d_lengths, int B, int Np
   plan->Nq = plan->Nk = Npad;
   plan->QT = plan->KT = QT;
   const int64_t grid_total = static_cast<int64_t>(B) * QT * QT;
-  SIGATTN_TRY(scratch_alloc(&sc.kinds, static_cast<size_t>(grid_total), stream));
-  k_kinds_from_lengths<<<grid_for(grid_total, 256), 256, 0, stream>>>(d_lengths, B, Npad, QT, QT,
-                                                                        sc.kinds);
+  auto classify = [&](uint8_t* kinds) {
+    k_kinds_from_lengths<<<grid_for(grid_total, 256), 256, 0, stream>>>(d_lengths, B, Npad, QT,
+                                                                          QT, kinds);
+  };
   auto bits = [&](const int64_t* ptile, uint32_t* dst, int np) {
     k_bits_from_lengths<<<np, 128, 0, stream>>>(d_lengths, Npad, QT, QT, ptile, dst);
   };
-  return finish_plan(plan, sc, stream, bits, out);
+  return build_plan(plan, stream, classify, bits, out);
 }
 
 extern "C" int sigattn_plan_from_mask(const uint8_t* d_mask, int B, int Nq, int Nk,
@@ -565,14 +699,15 @@ extern "C" int sigattn_plan_from_mask(const uint8_t* d_mask, int B, int Nq, int 
   plan->QT = QT;
   plan->KT = KT;
   const int64_t grid_total = static_cast<int64_t>(B) * QT * KT;
-  SIGATTN_TRY(scratch_alloc(&sc.kinds, static_cast<size_t>(grid_total), stream));
-  k_kinds_from_mask<<<static_cast<unsigned>(grid_total), 256, 0, stream>>>(
-      d_mask, B, Nq, Nk, stride_b, stride_q, QT, KT, sc.kinds);
+  auto classify = [&](uint8_t* kinds) {
+    k_kinds_from_mask<<<static_cast<unsigned>(grid_total), 256, 0, stream>>>(
+        d_mask, B, Nq, Nk, stride_b, stride_q, QT, KT, kinds);
+  };
   auto bits = [&](const int64_t* ptile, uint32_t* dst, int np) {
     k_bits_from_mask<<<np, 256, 0, stream>>>(d_mask, Nq, Nk, stride_b, stride_q, QT, KT, ptile,
                                              dst);
   };
-  return finish_plan(plan, sc, stream, bits, out);
+  return build_plan(plan, stream, classify, bits, out);
 }
 
 extern "C" int sigattn_plan_get_sizes(const sigattn_plan* plan, sigattn_plan_sizes* sz) {
@@ -640,6 +775,33 @@ extern "C" int sigattn_plan_export_work(const sigattn_plan* plan, int32_t* row_w
     return SIGATTN_ERR_CUDA;
   }
   if (col_work && cudaMemcpy(col_work, plan->col_work, cols * 4, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return SIGATTN_ERR_CUDA;
+  }
+  return SIGATTN_OK;
+}
+
+extern "C" int sigattn_plan_export_runs(const sigattn_plan* plan, int32_t* run_ptr, int32_t* runs,
+                                        int64_t* nruns) {
+  if (!plan) return SIGATTN_ERR_INVALID;
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return SIGATTN_ERR_CUDA;
+  }
+  const size_t rows = static_cast<size_t>(plan->B) * plan->QT;
+  int32_t total = 0;
+  if (cudaMemcpy(&total, plan->run_ptr + rows, sizeof(int32_t), cudaMemcpyDeviceToHost) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return SIGATTN_ERR_CUDA;
+  }
+  if (nruns) *nruns = total;
+  if (run_ptr && cudaMemcpy(run_ptr, plan->run_ptr, (rows + 1) * 4, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return SIGATTN_ERR_CUDA;
+  }
+  if (runs && total > 0 &&
+      cudaMemcpy(runs, plan->run, static_cast<size_t>(total) * 16, cudaMemcpyDeviceToHost) != cudaSuccess) {
     cudaGetLastError();
     return SIGATTN_ERR_CUDA;
   }

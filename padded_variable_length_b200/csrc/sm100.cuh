@@ -11,6 +11,11 @@ namespace sigattn {
 
 constexpr int kStatusTimeout = 1;
 
+// Limit of the waits that end a kernel after another wait gave up: the copies a CTA issued
+// and the MMAs it committed always complete, so these waits never depend on the caller's
+// limit (which a test may set very short) and give up only if the hardware is gone.
+constexpr unsigned long long kDrainWaitNs = 4000000000ull;
+
 // What a bounded wait needs: the device status word to record a timeout in, the
 // limit in nanoseconds, and a CTA-wide abort flag in shared memory that lets the other
 // roles of the CTA stop waiting once one of them gave up.
@@ -122,6 +127,39 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// 4-D tiled reduce-add shared -> global (element type and box from the tensor map; box
+// rows past the tensor's extent are not written).  Tracked as a bulk async-group of the
+// issuing thread: bulk_commit_group() after it, then bulk_wait_read() before the shared
+// source is rewritten and bulk_wait_all() before the kernel ends.
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* smem_src,
+                                                  int x, int y, int z, int w) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%1, %2, %3, %4}], [%5];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(smem_src))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until every committed bulk group of this thread has finished reading its source.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Waits until every committed bulk group of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Makes this thread's generic-proxy writes to shared memory visible to the async proxy
+// (tensor-core operands, bulk copies) once a later barrier orders them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Untiled bulk copy global -> shared, completing on `bar` (both addresses 16-byte
 // aligned, `bytes` a multiple of 16).
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
@@ -211,6 +249,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : SIGATTN_R8(0)
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+                   taddr),
+               SIGATTN_W8(0)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -296,9 +347,11 @@ __device__ __forceinline__ void mma_ts_lh_w(uint32_t d_tmem, uint32_t a_tmem, ui
 // Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, dense.
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format (1 = bf16),
 //   bit 15 A major (0 = K), bit 16 B major (1 = MN), bits 17-22 N >> 3, bits 24-28 M >> 4.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major,
+                                                      bool a_mn_major = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // ------------------------------------------------------------------------------------
@@ -335,21 +388,6 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ float tanh_approx(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// sigma(x) for x = a * s + c given as (s, a/2, c/2): 0.5 + 0.5 tanh(x / 2) on the hardware
-// tanh approximation (one MUFU op per element, the form the sigmoid-attention page's kernel
-// uses).  Measured on B200 over x in [-40, 20]: absolute error <= 4e-6, far below the
-// bf16 rounding of the weights fed to the MMA (that is why absolute, not relative, error is
-// the figure of merit here).
-__device__ __forceinline__ float sigmoid_tanh(float s, float half_a, float half_c) {
-  return fmaf(0.5f, tanh_approx(fmaf(s, half_a, half_c)), 0.5f);
-}
-
 // Packed fp32 pairs (sm_100): one instruction for two lanes of math, same per-element
 // throughput as scalar FFMA but half the issue slots.
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
@@ -377,6 +415,50 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// ------------------------------------------------------------------------------------
+// Sigmoid with small relative error over the whole range, at one MUFU op per element.
+//
+// With t = x log2(e), e = 2^(-|t|) = exp(-|x|) in (0, 1] and g = 1 / (1 + e) in [1/2, 1):
+//   sigma(x) = g for x >= 0,   sigma(x) = e g for x < 0,   sigma'(x) = sigma (1 - sigma) = e g^2
+// (for x < 0: 1 - sigma(x) = sigma(-x) = g; for x >= 0: 1 - sigma = e g).  No cancellation
+// anywhere, so the relative error of sigma is that of g plus that of exp2 -- unlike
+// 0.5 + 0.5 tanh(x / 2), whose hardware tanh loses every digit of a weight like 1/n for
+// long sequences (x = -log n well below -8).  e is the hardware exp2 (MUFU); g is the
+// degree-4 polynomial below on the FMA pipe, fitted for minimal maximum relative error on
+// [0, 1] (fit_sigmoid_poly.py): relative error 3.0e-4 = 2^-11.7 in float32, far below the
+// bf16 rounding (2^-9) of the weights fed to the MMAs.
+// A masked element takes t = -inf: e = 0, so sigma = sigma' = 0 there.
+// ------------------------------------------------------------------------------------
+constexpr float kSigG0 = 0.999702513f;
+constexpr float kSigG1 = -0.984833419f;
+constexpr float kSigG2 = 0.865889132f;
+constexpr float kSigG3 = -0.532853127f;
+constexpr float kSigG4 = 0.152243674f;
+
+// e = 2^(-|t|) and g = 1 / (1 + e) for two elements.
+__device__ __forceinline__ void sigmoid_parts2(float2 t, float2& e, float2& g) {
+  e = make_float2(ex2_approx(-fabsf(t.x)), ex2_approx(-fabsf(t.y)));
+  float2 a = fma2(make_float2(kSigG4, kSigG4), e, make_float2(kSigG3, kSigG3));
+  a = fma2(a, e, make_float2(kSigG2, kSigG2));
+  a = fma2(a, e, make_float2(kSigG1, kSigG1));
+  g = fma2(a, e, make_float2(kSigG0, kSigG0));
+}
+
+// sigma(x) for two elements given t = x log2(e) (t = -inf for a masked element: 0).
+__device__ __forceinline__ float2 sigmoid2(float2 t) {
+  float2 e, g;
+  sigmoid_parts2(t, e, g);
+  return mul2(make_float2(t.x < 0.0f ? e.x : 1.0f, t.y < 0.0f ? e.y : 1.0f), g);
+}
+
+// sigma(x) and sigma'(x) = sigma (1 - sigma) for two elements, t as in sigmoid2.
+__device__ __forceinline__ void sigmoid_grad2(float2 t, float2& p, float2& dp) {
+  float2 e, g;
+  sigmoid_parts2(t, e, g);
+  p = mul2(make_float2(t.x < 0.0f ? e.x : 1.0f, t.y < 0.0f ? e.y : 1.0f), g);
+  dp = mul2(mul2(e, g), g);
 }
 
 }  // namespace sigattn

@@ -64,5 +64,10 @@ def test_full_size_sampled(cfg):
         ref["dk"].append(dk_ref)
         ref["dv"].append(dv_ref)
     for name in got:
-        Hn.check_close(np.concatenate(got[name]), np.concatenate(ref[name]),
-                       f"{w.name} {name} (sampled)")
+        g, r = np.concatenate(got[name]), np.concatenate(ref[name])
+        Hn.check_close(g, r, f"{w.name} {name} (sampled)")
+        # relative to the largest reference value, with no absolute floor: the floor of the
+        # parity tolerance would hide a systematic error of the small sigmoid weights
+        ratio = float(np.max(np.abs(g - r)) / np.max(np.abs(r)))
+        print(f"{w.name} {name}: max|err| / max|ref| = {ratio:.3e}")
+        assert ratio <= 1e-2, f"{w.name} {name}: max|err| / max|ref| = {ratio:.3e}"

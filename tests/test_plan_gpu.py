@@ -98,3 +98,43 @@ def test_plan_packed_documents():
     z = plan.sizes()
     pop = int(np.unpackbits(ref["bits"].view(np.uint8)).sum())
     assert pop + 16384 * z["full"] == w.pairs()
+
+
+def test_plan_with_more_rows_than_one_sort_chunk():
+    """More than 1024 q-tile rows and k-tile columns (the work lists are sorted in chunks
+    of 1024): still bit-exact, longest-first and stable."""
+    from padded_variable_length_b200 import binding as Bd
+    rng = np.random.default_rng(77)
+    npad = 7000
+    lengths = rng.integers(0, npad + 1, 24).astype(np.int32)
+    lengths[0] = npad
+    plan = Bd.Plan.from_lengths(torch.from_numpy(lengths).cuda(), npad)
+    assert plan.sizes()["B"] * plan.sizes()["QT"] > 1024
+    _compare(plan, OT.tile_list_from_lengths(lengths, npad))
+
+
+RUN_CASES = ["lengths", "mask", "packed", "tree", "longformer"]
+
+
+@pytest.mark.parametrize("case", RUN_CASES)
+def test_plan_runs_bit_exact(case):
+    """The run-length rows of the plan equal the oracle's, walked entry by entry."""
+    from padded_variable_length_b200 import binding as Bd
+    rng = np.random.default_rng(9)
+    if case == "lengths":
+        lengths = np.array([0, 1, 640, 129, 1000], dtype=np.int32)
+        plan = Bd.Plan.from_lengths(torch.from_numpy(lengths).cuda(), 1000)
+        ref = OT.tile_list_from_lengths(lengths, 1000)
+    else:
+        if case == "mask":
+            m = W.random_mask(rng, 3, 700, 900, density=0.3, empty_rows=4)
+        elif case == "packed":
+            m = W.config(4).mask[:2]
+        else:
+            m = W.mask_family(case).mask[:2]
+        plan = Bd.Plan.from_mask(torch.from_numpy(m).cuda())
+        ref = OT.tile_list(m)
+    run_ptr, runs = plan.export_runs()
+    ref_ptr, ref_runs = OT.row_runs(ref)
+    assert np.array_equal(run_ptr, ref_ptr)
+    assert np.array_equal(runs, ref_runs)
