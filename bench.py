@@ -60,10 +60,19 @@ def workload_name(w: W.Workload, epi: int) -> str:
 
 
 def bench_workload(args, epi: int) -> W.Workload:
-    """The workload of --config, or of --mask (the other block-mask families)."""
-    if args.mask:
-        return W.mask_family(args.mask, epilogue=epi)
-    return W.config(args.config, epilogue=epi)
+    """The workload of --config, or of --mask (the other block-mask families); --batch keeps
+    only its first batch entries (a smaller case of the same shapes, for profiler captures)."""
+    w = W.mask_family(args.mask, epilogue=epi) if args.mask else W.config(args.config, epilogue=epi)
+    if args.batch and args.batch < w.B:
+        nb = args.batch
+        if w.lengths is not None:
+            w = W.padded_workload(w.name, w.lengths[:nb], H=w.H, d=w.d, epilogue=epi, backward=True,
+                                  seed=w.seed, npad=w.Nq)
+        else:
+            w = W.masked_workload(w.name, w.mask[:nb], w.counts[:nb], H=w.H, d=w.d, epilogue=epi,
+                                  backward=True, seed=w.seed,
+                                  doc_lengths=w.doc_lengths[:nb] if w.doc_lengths else None)
+    return w
 
 
 def fwd_flops(w: W.Workload) -> float:
@@ -267,13 +276,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         torch.cuda.synchronize()
         parts = [g.replay for g in graphs]
 
+    L_ = args.layers  # layers per step, all on the one plan (built once per batch)
+
     def step(ev=None):
-        for k_, fn in enumerate(parts):
-            if ev:
-                ev[k_].record(stream)
-            fn()
+        for layer in range(L_):
+            for k_, fn in enumerate(parts):
+                if ev:
+                    ev[layer * len(parts) + k_].record(stream)
+                fn()
         if ev:
-            ev[len(parts)].record(stream)
+            ev[L_ * len(parts)].record(stream)
 
     sampler = ClockSampler(local_rank if os.environ.get("CUDA_VISIBLE_DEVICES") is None else 0)
     sampler.start()
@@ -288,7 +300,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(L_ * len(parts) + 1)]
            for _ in range(args.steps)]
     for i in range(args.steps):
         step(evs[i])
@@ -298,11 +310,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         torch.distributed.barrier()
     clocks = sampler.stop()
     assert Bd.get_status() == 0, "device status reports a timed-out wait"
-    part_ms = [sum(e[k_].elapsed_time(e[k_ + 1]) for e in evs) for k_ in range(len(parts))]
-    total_ms = max_over_ranks(sum(part_ms), dev)
+    # per part, summed over steps and layers; the per-launch figures below divide by both
+    part_ms = [sum(e[layer * len(parts) + k_].elapsed_time(e[layer * len(parts) + k_ + 1])
+                   for e in evs for layer in range(L_)) / L_ for k_ in range(len(parts))]
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[-1]) for e in evs), dev)
 
     ff = fwd_flops(w)
-    step_flops = 3.5 * ff
+    step_flops = 3.5 * ff * L_
     value = job_throughput(world, step_flops, args.steps, total_ms)
     peaks, peak_src = load_peaks()
     peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -334,13 +348,15 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "data": "synthetic",
         "config": {"workload": workload_name(w, epi), "l2": "flushed (256 MB write) between steps",
                    "plan": "built once per batch, outside the step",
+                   "layers_per_step": L_,
                    "launch": "API calls each step" if args.no_graph else "CUDA graph replay per part",
                    "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
         "fwd_tflops": kernels["fwd"]["tflops"], "fwd_frac": kernels["fwd"]["tflops"] / peak_tf,
         "bwd_tflops": 2.5 * ff / (bwd_ms / K / 1e3) / 1e12,
         "bwd_frac": 2.5 * ff / (bwd_ms / K / 1e3) / 1e12 / peak_tf,
         "bwd_algo": "fused (one kernel, dQ by TMA reduce-add)" if fused else "split (dK/dV + dQ)",
-        "kernels": kernels, "plan_ms": plan_ms,
+        "kernels": kernels, "plan_ms": plan_ms, "layers": L_,
+        "plan_share": plan_ms / (plan_ms + total_ms / K),
         "plan": plan_report(w, plan_ms, peaks, peak_src),
         "tiles": {"nonempty": sizes["nonempty"], "full": sizes["full"], "partial": sizes["partial"],
                   "grid_total": sizes["grid_total"],
@@ -440,6 +456,10 @@ def main():
     ap.add_argument("--bwd", default="auto", choices=["auto", "fused", "split"],
                     help="backward form: fused (d = 64 only) or the two-kernel split; auto = "
                          "fused where supported")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="keep only the first B batch entries of the workload (profiling)")
+    ap.add_argument("--layers", type=int, default=1,
+                    help="attention layers per step, all reusing the one plan of the batch")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every part through the API each step instead of replaying CUDA graphs")
     args = ap.parse_args()

@@ -109,6 +109,22 @@ SIGATTN_API int sigattn_plan_from_lengths(const int32_t* d_lengths, int B, int N
 SIGATTN_API int sigattn_plan_from_mask(const uint8_t* d_mask, int B, int Nq, int Nk, int64_t stride_b,
                            int64_t stride_q, sigattn_stream stream, sigattn_plan** out);
 
+/*
+ * Plan for a PACKED batch (no padding): sequence b occupies rows cu[b] .. cu[b+1] of
+ * tensors laid out [T, H, d] (T = cu[B]); d_cu: device int32 [B + 1], non-decreasing, each
+ * length cu[b+1] - cu[b] in [0, max_seqlen].  The tile list is that of the padded batch
+ * with these lengths and Npad = max_seqlen ("Better Models, Faster Training", section 1:
+ * ragged cells; here without the padding), so the kernels skip the same tiles; they address
+ * row r of sequence b at packed row cu[b] + r and write only the sequence's own rows.  With
+ * such a plan, every tensor argument of the attention calls is [T, H, d]: pass strides
+ * {any, token, head} (the batch stride is ignored), bias is fp32 [T] (bias_stride_b
+ * ignored), and lse / the softmax workspace keep their [B, H, max_seqlen] layout.  The plan
+ * keeps a copy of cu.  Synchronises `stream` once.  Errors: INVALID (null, B < 1,
+ * max_seqlen < 1, a length outside [0, max_seqlen], T < 1), UNSUPPORTED, CUDA, NOMEM.
+ */
+SIGATTN_API int sigattn_plan_from_cu_seqlens(const int32_t* d_cu, int B, int max_seqlen,
+                                             sigattn_stream stream, sigattn_plan** out);
+
 /* Fills *sizes (host struct).  No device work. */
 SIGATTN_API int sigattn_plan_get_sizes(const sigattn_plan* plan, sigattn_plan_sizes* sizes);
 

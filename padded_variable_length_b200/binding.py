@@ -60,6 +60,7 @@ def _sig(name, res, *args):
 _sig("sigattn_plan_from_lengths", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, _p, ctypes.POINTER(_p))
 _sig("sigattn_plan_from_mask", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _i64, _i64,
      _p, ctypes.POINTER(_p))
+_sig("sigattn_plan_from_cu_seqlens", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, _p, ctypes.POINTER(_p))
 _sig("sigattn_plan_get_sizes", ctypes.c_int, _p, ctypes.POINTER(PlanSizes))
 _sig("sigattn_plan_export", ctypes.c_int, _p, _p, _p, _p, _p, _p, _p, _p, _p)
 _sig("sigattn_plan_export_work", ctypes.c_int, _p, _p, _p)
@@ -104,8 +105,12 @@ def _stream(stream) -> Optional[int]:
 
 
 def _strides(t: torch.Tensor) -> ctypes.Array:
-    if t.dim() != 4 or t.dtype != torch.bfloat16 or t.stride(3) != 1:
-        raise ValueError("expected a bf16 [B, N, H, d] tensor with d contiguous")
+    """(batch, token, head) element strides of a padded [B, N, H, d] tensor, or of a packed
+    [T, H, d] tensor (batch stride 0: ignored by the library for packed plans)."""
+    if t.dtype != torch.bfloat16 or t.stride(-1) != 1 or t.dim() not in (3, 4):
+        raise ValueError("expected a bf16 [B, N, H, d] or packed [T, H, d] tensor, d contiguous")
+    if t.dim() == 3:
+        return _I64x3(0, t.stride(0), t.stride(1))
     return _I64x3(t.stride(0), t.stride(1), t.stride(2))
 
 
@@ -122,6 +127,16 @@ class Plan:
         h = ctypes.c_void_p()
         _check(_lib.sigattn_plan_from_lengths(lengths.data_ptr(), lengths.numel(), int(npad),
                                               _stream(stream), ctypes.byref(h)), "plan_from_lengths")
+        return cls(h.value)
+
+    @classmethod
+    def from_cu_seqlens(cls, cu: torch.Tensor, max_seqlen: int, stream=None) -> "Plan":
+        """Plan of a packed batch: sequence b is rows cu[b] .. cu[b+1] of [T, H, d] tensors."""
+        if cu.dtype != torch.int32 or not cu.is_cuda or not cu.is_contiguous() or cu.dim() != 1:
+            raise ValueError("cu must be a contiguous int32 CUDA tensor [B + 1]")
+        h = ctypes.c_void_p()
+        _check(_lib.sigattn_plan_from_cu_seqlens(cu.data_ptr(), cu.numel() - 1, int(max_seqlen),
+                                                 _stream(stream), ctypes.byref(h)), "plan_from_cu_seqlens")
         return cls(h.value)
 
     @classmethod
@@ -204,15 +219,23 @@ def bias_from_counts(counts: torch.Tensor, out: Optional[torch.Tensor] = None, s
 def _bias_args(bias):
     if bias is None:
         return None, 0
-    if bias.dtype != torch.float32 or bias.dim() != 2 or bias.stride(1) != 1:
-        raise ValueError("bias must be fp32 [B, Nq] with unit row stride")
-    return bias.data_ptr(), bias.stride(0)
+    if bias.dtype != torch.float32 or bias.stride(-1) != 1 or bias.dim() not in (1, 2):
+        raise ValueError("bias must be fp32 [B, Nq] (or [T] for a packed plan) with unit row stride")
+    return bias.data_ptr(), (bias.stride(0) if bias.dim() == 2 else 0)
+
+
+def _shape(plan: "Plan", q: torch.Tensor):
+    """(B, Nq, H, d): from a padded Q, or from the plan for a packed [T, H, d] Q."""
+    if q.dim() == 4:
+        return tuple(q.shape)
+    z = plan.sizes()
+    return z["B"], z["Nq"], q.shape[1], q.shape[2]
 
 
 def fwd(plan: Plan, q, k, v, bias=None, epilogue: int = SIGMOID, scale: Optional[float] = None,
         out=None, lse=None, stream=None):
     """O (and the row log-normaliser for the softmax modes) of the planned attention."""
-    B, Nq, H, d = q.shape
+    B, Nq, H, d = _shape(plan, q)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
@@ -234,7 +257,7 @@ def bwd(plan: Plan, q, k, v, o, do, bias=None, epilogue: int = SIGMOID, lse=None
         scale: Optional[float] = None, workspace=None, dq=None, dk=None, dv=None, stream=None,
         parts: int = BWD_ALL):
     """dQ, dK, dV of L = sum(dO * O) (``parts`` selects PREP / DKDV / DQ)."""
-    B, Nq, H, d = q.shape
+    B, Nq, H, d = _shape(plan, q)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq
@@ -267,7 +290,7 @@ def bwd_fused(plan: Plan, q, k, v, o, do, bias=None, epilogue: int = SIGMOID, ls
     """dQ, dK, dV of L = sum(dO * O) in one walk over the k-tile columns (d = 64): dQ is
     accumulated in fp32 in ``workspace`` (a 16-byte aligned CUDA buffer of at least
     bwd_fused_workspace_bytes bytes; allocated here if None) and converted at the end."""
-    B, Nq, H, d = q.shape
+    B, Nq, H, d = _shape(plan, q)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq

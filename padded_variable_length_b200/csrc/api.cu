@@ -76,7 +76,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int check_tensor(const void* ptr, const int64_t* strides, int N, TensorDesc* t) {
+int check_tensor(const void* ptr, const int64_t* strides, int64_t N, TensorDesc* t) {
+  if (N < 1 || N > 0x7FFFFFFF) return SIGATTN_ERR_UNSUPPORTED;
   if (!ptr || !strides) return SIGATTN_ERR_INVALID;
   for (int i = 0; i < 3; ++i)
     if (strides[i] < 0) return SIGATTN_ERR_INVALID;
@@ -87,9 +88,15 @@ int check_tensor(const void* ptr, const int64_t* strides, int N, TensorDesc* t) 
   t->sb = strides[0];
   t->sn = strides[1];
   t->sh = strides[2];
-  t->N = N;
+  t->N = static_cast<int>(N);
   return SIGATTN_OK;
 }
+
+// Rows of the Q-side / K-side tensors and the batch extent of their TMA maps: padded batches
+// are [B, N, H, d]; a packed batch is one [T, H, d] tensor (T = the plan's last offset).
+int64_t rows_q(const sigattn_plan* plan) { return plan->cu ? plan->T : plan->Nq; }
+int64_t rows_k(const sigattn_plan* plan) { return plan->cu ? plan->T : plan->Nk; }
+int tma_batches(const sigattn_plan* plan) { return plan->cu ? 1 : plan->B; }
 
 int check_plan_device(const sigattn_plan* plan) {
   int dev = -1;
@@ -180,17 +187,17 @@ extern "C" int sigattn_fwd(const sigattn_plan* plan, int epilogue, int H, int d,
   if (static_cast<int64_t>(plan->B) * plan->QT * H > 0x7FFFFFFF) return SIGATTN_ERR_UNSUPPORTED;
   TensorDesc tq, tk, tv, to;
   int rc;
-  if ((rc = check_tensor(q, q_strides, plan->Nq, &tq)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(k, k_strides, plan->Nk, &tk)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(v, v_strides, plan->Nk, &tv)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(o, o_strides, plan->Nq, &to)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(q, q_strides, rows_q(plan), &tq)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(k, k_strides, rows_k(plan), &tk)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(v, v_strides, rows_k(plan), &tv)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(o, o_strides, rows_q(plan), &to)) != SIGATTN_OK) return rc;
   if ((rc = check_plan_device(plan)) != SIGATTN_OK) return rc;
   int* status = nullptr;
   if ((rc = status_ptr(&status)) != SIGATTN_OK) return rc;
   CUtensorMap mq, mk, mv;
-  if ((rc = make_tmap_bf16(&mq, tq, plan->B, H, d)) != SIGATTN_OK) return rc;
-  if ((rc = make_tmap_bf16(&mk, tk, plan->B, H, d)) != SIGATTN_OK) return rc;
-  if ((rc = make_tmap_bf16(&mv, tv, plan->B, H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mq, tq, tma_batches(plan), H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mk, tk, tma_batches(plan), H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mv, tv, tma_batches(plan), H, d)) != SIGATTN_OK) return rc;
   return launch_fwd_impl(plan, epilogue, H, d, scale, mq, mk, mv, bias, bias_stride_b, to, lse,
                          status, g_wait_limit_ns.load(), static_cast<cudaStream_t>(s));
 }
@@ -216,24 +223,24 @@ extern "C" int sigattn_bwd_ex(const sigattn_plan* plan, int epilogue, int H, int
     return SIGATTN_ERR_UNSUPPORTED;
   TensorDesc tq, tk, tv, to{}, tdo, tdq, tdk, tdv;
   int rc;
-  if ((rc = check_tensor(q, q_strides, plan->Nq, &tq)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(k, k_strides, plan->Nk, &tk)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(v, v_strides, plan->Nk, &tv)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(q, q_strides, rows_q(plan), &tq)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(k, k_strides, rows_k(plan), &tk)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(v, v_strides, rows_k(plan), &tv)) != SIGATTN_OK) return rc;
   if (epilogue != SIGATTN_SIGMOID &&
-      (rc = check_tensor(o, o_strides, plan->Nq, &to)) != SIGATTN_OK)
+      (rc = check_tensor(o, o_strides, rows_q(plan), &to)) != SIGATTN_OK)
     return rc;
-  if ((rc = check_tensor(dout, do_strides, plan->Nq, &tdo)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(dq, dq_strides, plan->Nq, &tdq)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(dk, dk_strides, plan->Nk, &tdk)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(dv, dv_strides, plan->Nk, &tdv)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(dout, do_strides, rows_q(plan), &tdo)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(dq, dq_strides, rows_q(plan), &tdq)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(dk, dk_strides, rows_k(plan), &tdk)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(dv, dv_strides, rows_k(plan), &tdv)) != SIGATTN_OK) return rc;
   if ((rc = check_plan_device(plan)) != SIGATTN_OK) return rc;
   int* status = nullptr;
   if ((rc = status_ptr(&status)) != SIGATTN_OK) return rc;
   CUtensorMap mq, mk, mv, mdo;
-  if ((rc = make_tmap_bf16(&mq, tq, plan->B, H, d)) != SIGATTN_OK) return rc;
-  if ((rc = make_tmap_bf16(&mk, tk, plan->B, H, d)) != SIGATTN_OK) return rc;
-  if ((rc = make_tmap_bf16(&mv, tv, plan->B, H, d)) != SIGATTN_OK) return rc;
-  if ((rc = make_tmap_bf16(&mdo, tdo, plan->B, H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mq, tq, tma_batches(plan), H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mk, tk, tma_batches(plan), H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mv, tv, tma_batches(plan), H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mdo, tdo, tma_batches(plan), H, d)) != SIGATTN_OK) return rc;
   return launch_bwd_impl(plan, epilogue, H, d, scale, mq, mk, mv, mdo, to, tdo, bias,
                          bias_stride_b, lse, workspace, tdq, tdk, tdv, parts, status,
                          g_wait_limit_ns.load(), static_cast<cudaStream_t>(s));
@@ -272,16 +279,16 @@ extern "C" int sigattn_bwd_fused(const sigattn_plan* plan, int epilogue, int H, 
       0x7FFFFFFF)
     return SIGATTN_ERR_UNSUPPORTED;
   TensorDesc tq, tk, tv, to{}, tdo, tdq, tdk, tdv;
-  if ((rc = check_tensor(q, q_strides, plan->Nq, &tq)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(k, k_strides, plan->Nk, &tk)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(v, v_strides, plan->Nk, &tv)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(q, q_strides, rows_q(plan), &tq)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(k, k_strides, rows_k(plan), &tk)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(v, v_strides, rows_k(plan), &tv)) != SIGATTN_OK) return rc;
   if (epilogue != SIGATTN_SIGMOID &&
-      (rc = check_tensor(o, o_strides, plan->Nq, &to)) != SIGATTN_OK)
+      (rc = check_tensor(o, o_strides, rows_q(plan), &to)) != SIGATTN_OK)
     return rc;
-  if ((rc = check_tensor(dout, do_strides, plan->Nq, &tdo)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(dq, dq_strides, plan->Nq, &tdq)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(dk, dk_strides, plan->Nk, &tdk)) != SIGATTN_OK) return rc;
-  if ((rc = check_tensor(dv, dv_strides, plan->Nk, &tdv)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(dout, do_strides, rows_q(plan), &tdo)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(dq, dq_strides, rows_q(plan), &tdq)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(dk, dk_strides, rows_k(plan), &tdk)) != SIGATTN_OK) return rc;
+  if ((rc = check_tensor(dv, dv_strides, rows_k(plan), &tdv)) != SIGATTN_OK) return rc;
   if ((rc = check_plan_device(plan)) != SIGATTN_OK) return rc;
   int* status = nullptr;
   if ((rc = status_ptr(&status)) != SIGATTN_OK) return rc;
@@ -290,10 +297,10 @@ extern "C" int sigattn_bwd_fused(const sigattn_plan* plan, int epilogue, int H, 
                    ? dqacc + static_cast<size_t>(plan->B) * plan->Nq * H * d
                    : nullptr;
   CUtensorMap mq, mk, mv, mdo, macc;
-  if ((rc = make_tmap_bf16(&mq, tq, plan->B, H, d)) != SIGATTN_OK) return rc;
-  if ((rc = make_tmap_bf16(&mk, tk, plan->B, H, d)) != SIGATTN_OK) return rc;
-  if ((rc = make_tmap_bf16(&mv, tv, plan->B, H, d)) != SIGATTN_OK) return rc;
-  if ((rc = make_tmap_bf16(&mdo, tdo, plan->B, H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mq, tq, tma_batches(plan), H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mk, tk, tma_batches(plan), H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mv, tv, tma_batches(plan), H, d)) != SIGATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&mdo, tdo, tma_batches(plan), H, d)) != SIGATTN_OK) return rc;
   if ((rc = make_tmap_f32_acc(&macc, dqacc, plan->B, plan->Nq, H, d)) != SIGATTN_OK) return rc;
   return launch_bwd_fused_impl(plan, epilogue, H, scale, mq, mk, mv, mdo, macc, to, tdo, bias,
                                bias_stride_b, lse, Dws, dqacc, tdq, tdk, tdv, status,

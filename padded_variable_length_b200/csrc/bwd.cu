@@ -44,6 +44,7 @@ struct BwdParams {
   const int32_t* csc_map;
   const int4* row_desc;
   const int4* col_desc;
+  const int32_t* cu;  // packed batches: cumulative row offsets [B + 1]; nullptr when padded
   int B, QT, KT, Nq, Nk, H;
   float scale;
   const float* bias;
@@ -64,9 +65,12 @@ struct BwdParams {
 // SIGMOID  p = sigma(t ln 2),  off = bias log2 e  (sigmoid_grad2);
 // softmax  p = 2^t,            off = (bias - lse) log2 e.
 template <int EPI>
-__device__ __forceinline__ float row_offset(const BwdParams& p, int b, int h, int qg) {
+__device__ __forceinline__ float row_offset(const BwdParams& p, const SeqRows& sq, int b, int h,
+                                           int qg) {
   if (qg >= p.Nq) return 0.0f;
-  const float bias = p.bias ? p.bias[b * p.bias_sb + qg] : 0.0f;
+  const float bias =
+      (p.bias && qg < sq.limit) ? p.bias[static_cast<int64_t>(sq.tma_b) * p.bias_sb + sq.row0 + qg]
+                                : 0.0f;
   if (EPI == 0) return bias * kLog2e;
   return (bias - p.lse[(static_cast<int64_t>(b) * p.H + h) * p.Nq + qg]) * kLog2e;
 }
@@ -115,7 +119,7 @@ template <int D>
 __global__ void d_preprocess_kernel(const __nv_bfloat16* __restrict__ o, int64_t o_sb, int64_t o_sn,
                                     int64_t o_sh, const __nv_bfloat16* __restrict__ dout,
                                     int64_t do_sb, int64_t do_sn, int64_t do_sh, int B, int Nq,
-                                    int H, float* __restrict__ Dws) {
+                                    int H, const int32_t* __restrict__ cu, float* __restrict__ Dws) {
   constexpr int kLanes = D / 8;
   const int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   const int64_t row = t / kLanes;
@@ -127,8 +131,11 @@ __global__ void d_preprocess_kernel(const __nv_bfloat16* __restrict__ o, int64_t
     h = static_cast<int>(row % H);
     i = static_cast<int>((row / H) % Nq);
     b = static_cast<int>(row / (static_cast<int64_t>(H) * Nq));
-    const uint4 ov = *reinterpret_cast<const uint4*>(o + b * o_sb + i * o_sn + h * o_sh + chunk * 8);
-    const uint4 dv = *reinterpret_cast<const uint4*>(dout + b * do_sb + i * do_sn + h * do_sh + chunk * 8);
+  }
+  const SeqRows sq = seq_rows(cu, b, Nq);
+  if (act && i < sq.limit) {
+    const uint4 ov = *reinterpret_cast<const uint4*>(o + seq_row_offset(sq, o_sb, o_sn, i) + h * o_sh + chunk * 8);
+    const uint4 dv = *reinterpret_cast<const uint4*>(dout + seq_row_offset(sq, do_sb, do_sn, i) + h * do_sh + chunk * 8);
     const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
     const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
 #pragma unroll
@@ -156,6 +163,7 @@ __global__ void d_preprocess_kernel(const __nv_bfloat16* __restrict__ o, int64_t
 // ---------------------------------------------------------------------------------------
 struct WorkRef {
   int b, t, h, e0, n;  // batch, tile index on the item's own axis, head, list range
+  SeqRows sq;          // where the rows of sequence b live (padded or packed)
 };
 
 // dK/dV: item w -> (k-tile column, head); dQ: item w -> (q-tile row, head).
@@ -167,6 +175,7 @@ __device__ __forceinline__ WorkRef decode_col(const BwdParams& p, int w) {
   r.t = d.x % p.KT;
   r.e0 = d.y;
   r.n = d.z;
+  r.sq = seq_rows(p.cu, r.b, p.Nk);
   return r;
 }
 
@@ -178,6 +187,7 @@ __device__ __forceinline__ WorkRef decode_row(const BwdParams& p, int w) {
   r.t = d.x % p.QT;
   r.e0 = d.y;
   r.n = d.z;
+  r.sq = seq_rows(p.cu, r.b, p.Nq);
   return r;
 }
 
@@ -322,9 +332,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(kv_full + kb, 2 * L::kTileBytes);
         for (int x = 0; x < L::kBoxes; ++x) {
           tma_load_4d(smem + L::kK + kb * L::kTileBytes + x * L::kBoxBytes, &tk, kv_full + kb,
-                      x * 64, it.t * kTile, it.h, it.b);
+                      x * 64, it.sq.row0 + it.t * kTile, it.h, it.sq.tma_b);
           tma_load_4d(smem + L::kV + kb * L::kTileBytes + x * L::kBoxBytes, &tv, kv_full + kb,
-                      x * 64, it.t * kTile, it.h, it.b);
+                      x * 64, it.sq.row0 + it.t * kTile, it.h, it.sq.tma_b);
         }
       }
       ++ii;
@@ -333,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int qg = qt * kTile + lane + 32 * k;
-          v0[k] = row_offset<EPI>(p, it.b, it.h, qg);
+          v0[k] = row_offset<EPI>(p, it.sq, it.b, it.h, qg);
           v1[k] = row_D<EPI>(p, it.b, it.h, qg);
         }
       };
@@ -368,9 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(q_full + s, 2 * L::kTileBytes + (kd == 2 ? 2048 : 0));
             for (int x = 0; x < L::kBoxes; ++x) {
               tma_load_4d(smem + L::kQ + s * L::kTileBytes + x * L::kBoxBytes, &tq, q_full + s,
-                          x * 64, qt * kTile, it.h, it.b);
+                          x * 64, it.sq.row0 + qt * kTile, it.h, it.sq.tma_b);
               tma_load_4d(smem + L::kDO + s * L::kTileBytes + x * L::kBoxBytes, &tdo, q_full + s,
-                          x * 64, qt * kTile, it.h, it.b);
+                          x * 64, it.sq.row0 + qt * kTile, it.h, it.sq.tma_b);
             }
             if (kd == 2)
               bulk_load(meta_bits + s * 512, p.bitsT + static_cast<int64_t>(pi) * 512, 2048,
@@ -600,13 +610,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
       const int kg = pit.t * kTile + row;
-      if (kg < p.Nk) {
-        uint4* dvp = reinterpret_cast<uint4*>(p.dv + pit.b * p.dv_sb +
-                                              static_cast<int64_t>(kg) * p.dv_sn + pit.h * p.dv_sh +
-                                              h * kOc);
-        uint4* dkp = reinterpret_cast<uint4*>(p.dk + pit.b * p.dk_sb +
-                                              static_cast<int64_t>(kg) * p.dk_sn + pit.h * p.dk_sh +
-                                              h * kOc);
+      if (kg < pit.sq.limit) {
+        uint4* dvp = reinterpret_cast<uint4*>(p.dv + seq_row_offset(pit.sq, p.dv_sb, p.dv_sn, kg) +
+                                              pit.h * p.dv_sh + h * kOc);
+        uint4* dkp = reinterpret_cast<uint4*>(p.dk + seq_row_offset(pit.sq, p.dk_sb, p.dk_sn, kg) +
+                                              pit.h * p.dk_sh + h * kOc);
 #pragma unroll
         for (int c = 0; c < kOc / 8; ++c) {
           dvp[c] = make_uint4(pv[4 * c], pv[4 * c + 1], pv[4 * c + 2], pv[4 * c + 3]);
@@ -620,11 +628,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (it.n == 0) {
         // No query attends to this k-tile: dK = dV = 0 on its rows.
         if (pend) flush();
-        const int rows = min(kTile, p.Nk - it.t * kTile);
+        const int rows = min(kTile, it.sq.limit - it.t * kTile);
         const int tid = threadIdx.x - kEpiWarp0 * 32;
-        zero_rows<D>(p.dk + it.b * p.dk_sb + static_cast<int64_t>(it.t * kTile) * p.dk_sn +
+        zero_rows<D>(p.dk + seq_row_offset(it.sq, p.dk_sb, p.dk_sn, it.t * kTile) +
                          it.h * p.dk_sh, p.dk_sn, rows, tid, 256);
-        zero_rows<D>(p.dv + it.b * p.dv_sb + static_cast<int64_t>(it.t * kTile) * p.dv_sn +
+        zero_rows<D>(p.dv + seq_row_offset(it.sq, p.dv_sb, p.dv_sn, it.t * kTile) +
                          it.h * p.dv_sh, p.dv_sn, rows, tid, 256);
         continue;
       }
@@ -695,11 +703,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WorkRef it = iter.cur;
       if (it.n == 0) {
         // No query attends to this k-tile: dK = dV = 0 on its rows.
-        const int rows = min(kTile, p.Nk - it.t * kTile);
+        const int rows = min(kTile, it.sq.limit - it.t * kTile);
         const int tid = threadIdx.x - kEpiWarp0 * 32;
-        zero_rows<D>(p.dk + it.b * p.dk_sb + static_cast<int64_t>(it.t * kTile) * p.dk_sn +
+        zero_rows<D>(p.dk + seq_row_offset(it.sq, p.dk_sb, p.dk_sn, it.t * kTile) +
                          it.h * p.dk_sh, p.dk_sn, rows, tid, 256);
-        zero_rows<D>(p.dv + it.b * p.dv_sb + static_cast<int64_t>(it.t * kTile) * p.dv_sn +
+        zero_rows<D>(p.dv + seq_row_offset(it.sq, p.dv_sb, p.dv_sn, it.t * kTile) +
                          it.h * p.dv_sh, p.dv_sn, rows, tid, 256);
         continue;
       }
@@ -775,10 +783,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty + ab);
       const int kg = it.t * kTile + row;
-      if (kg < p.Nk) {
-        uint4* dvp = reinterpret_cast<uint4*>(p.dv + it.b * p.dv_sb + static_cast<int64_t>(kg) * p.dv_sn +
+      if (kg < it.sq.limit) {
+        uint4* dvp = reinterpret_cast<uint4*>(p.dv + seq_row_offset(it.sq, p.dv_sb, p.dv_sn, kg) +
                                               it.h * p.dv_sh + h * kOc);
-        uint4* dkp = reinterpret_cast<uint4*>(p.dk + it.b * p.dk_sb + static_cast<int64_t>(kg) * p.dk_sn +
+        uint4* dkp = reinterpret_cast<uint4*>(p.dk + seq_row_offset(it.sq, p.dk_sb, p.dk_sn, kg) +
                                               it.h * p.dk_sh + h * kOc);
 #pragma unroll
         for (int c = 0; c < kOc / 8; ++c) {
@@ -909,9 +917,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(qd_full + qb, 2 * L::kTileBytes);
           for (int x = 0; x < L::kBoxes; ++x) {
             tma_load_4d(smem + L::kQ + qb * L::kTileBytes + x * L::kBoxBytes, &tq, qd_full + qb,
-                        x * 64, it.t * kTile, it.h, it.b);
+                        x * 64, it.sq.row0 + it.t * kTile, it.h, it.sq.tma_b);
             tma_load_4d(smem + L::kDO + qb * L::kTileBytes + x * L::kBoxBytes, &tdo, qd_full + qb,
-                        x * 64, it.t * kTile, it.h, it.b);
+                        x * 64, it.sq.row0 + it.t * kTile, it.h, it.sq.tma_b);
           }
         }
       }
@@ -939,9 +947,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_expect_tx(kv_full + s, 2 * L::kTileBytes + (kd == 2 ? 2048 : 0));
               for (int x = 0; x < L::kBoxes; ++x) {
                 tma_load_4d(smem + L::kK + s * L::kTileBytes + x * L::kBoxBytes, &tk, kv_full + s,
-                            x * 64, kt * kTile, it.h, it.b);
+                            x * 64, it.sq.row0 + kt * kTile, it.h, it.sq.tma_b);
                 tma_load_4d(smem + L::kV + s * L::kTileBytes + x * L::kBoxBytes, &tv, kv_full + s,
-                            x * 64, kt * kTile, it.h, it.b);
+                            x * 64, it.sq.row0 + kt * kTile, it.h, it.sq.tma_b);
               }
               if (kd == 2)
                 bulk_load(meta_bits + s * 512, p.bits + static_cast<int64_t>(pi) * 512, 2048,
@@ -1147,10 +1155,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty + ab);
       const int qg = pit.t * kTile + row;
-      if (qg < p.Nq) {
-        uint4* dqp = reinterpret_cast<uint4*>(p.dq + pit.b * p.dq_sb +
-                                              static_cast<int64_t>(qg) * p.dq_sn + pit.h * p.dq_sh +
-                                              h * kOc);
+      if (qg < pit.sq.limit) {
+        uint4* dqp = reinterpret_cast<uint4*>(p.dq + seq_row_offset(pit.sq, p.dq_sb, p.dq_sn, qg) +
+                                              pit.h * p.dq_sh + h * kOc);
 #pragma unroll
         for (int c = 0; c < kOc / 8; ++c)
           dqp[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
@@ -1160,7 +1167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     WorkIter<false> iter(p, nitems);
     float off_cur = 0.0f, D_cur = 0.0f;
     if (iter.valid()) {
-      off_cur = row_offset<EPI>(p, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
+      off_cur = row_offset<EPI>(p, iter.cur.sq, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
       D_cur = row_D<EPI>(p, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
     }
     for (; ok && iter.valid(); iter.advance()) {
@@ -1168,7 +1175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the next item's row values, in flight while this one is processed
       float off_nxt = 0.0f, D_nxt = 0.0f;
       if (iter.wn < nitems && iter.nxt.n > 0) {
-        off_nxt = row_offset<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
+        off_nxt = row_offset<EPI>(p, iter.nxt.sq, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
         D_nxt = row_D<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
       }
       const float off = off_cur, Drow = D_cur;
@@ -1176,8 +1183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       D_cur = D_nxt;
       if (it.n == 0) {
         if (pend) flush();
-        const int rows = min(kTile, p.Nq - it.t * kTile);
-        zero_rows<D>(p.dq + it.b * p.dq_sb + static_cast<int64_t>(it.t * kTile) * p.dq_sn +
+        const int rows = min(kTile, it.sq.limit - it.t * kTile);
+        zero_rows<D>(p.dq + seq_row_offset(it.sq, p.dq_sb, p.dq_sn, it.t * kTile) +
                          it.h * p.dq_sh, p.dq_sn, rows, threadIdx.x - kEpiWarp0 * 32, 256);
         continue;
       }
@@ -1242,7 +1249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     WorkIter<false> iter(p, nitems);
     float off_cur = 0.0f, D_cur = 0.0f;
     if (iter.valid()) {
-      off_cur = row_offset<EPI>(p, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
+      off_cur = row_offset<EPI>(p, iter.cur.sq, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
       D_cur = row_D<EPI>(p, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
     }
     for (; iter.valid(); iter.advance()) {
@@ -1250,15 +1257,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the next item's row values, in flight while this one is processed
       float off_nxt = 0.0f, D_nxt = 0.0f;
       if (iter.wn < nitems && iter.nxt.n > 0) {
-        off_nxt = row_offset<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
+        off_nxt = row_offset<EPI>(p, iter.nxt.sq, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
         D_nxt = row_D<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
       }
       const float off = off_cur, Drow = D_cur;
       off_cur = off_nxt;
       D_cur = D_nxt;
       if (it.n == 0) {
-        const int rows = min(kTile, p.Nq - it.t * kTile);
-        zero_rows<D>(p.dq + it.b * p.dq_sb + static_cast<int64_t>(it.t * kTile) * p.dq_sn +
+        const int rows = min(kTile, it.sq.limit - it.t * kTile);
+        zero_rows<D>(p.dq + seq_row_offset(it.sq, p.dq_sb, p.dq_sn, it.t * kTile) +
                          it.h * p.dq_sh, p.dq_sn, rows, threadIdx.x - kEpiWarp0 * 32, 256);
         continue;
       }
@@ -1323,8 +1330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty + ab);
-      if (qg < p.Nq) {
-        uint4* dqp = reinterpret_cast<uint4*>(p.dq + it.b * p.dq_sb + static_cast<int64_t>(qg) * p.dq_sn +
+      if (qg < it.sq.limit) {
+        uint4* dqp = reinterpret_cast<uint4*>(p.dq + seq_row_offset(it.sq, p.dq_sb, p.dq_sn, qg) +
                                               it.h * p.dq_sh + h * kOc);
 #pragma unroll
         for (int c = 0; c < kOc / 8; ++c)
@@ -1478,15 +1485,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(kv_full + kb, 2 * L::kTileBytes);
-        tma_load_4d(smem + L::kK + kb * L::kTileBytes, &tk, kv_full + kb, 0, it.t * kTile, it.h, it.b);
-        tma_load_4d(smem + L::kV + kb * L::kTileBytes, &tv, kv_full + kb, 0, it.t * kTile, it.h, it.b);
+        tma_load_4d(smem + L::kK + kb * L::kTileBytes, &tk, kv_full + kb, 0, it.sq.row0 + it.t * kTile, it.h, it.sq.tma_b);
+        tma_load_4d(smem + L::kV + kb * L::kTileBytes, &tv, kv_full + kb, 0, it.sq.row0 + it.t * kTile, it.h, it.sq.tma_b);
       }
       ++ii;
       auto fetch_vec = [&](int qt, float (&v0)[4], float (&v1)[4]) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int qg = qt * kTile + lane + 32 * k;
-          v0[k] = row_offset<EPI>(p, it.b, it.h, qg);
+          v0[k] = row_offset<EPI>(p, it.sq, it.b, it.h, qg);
           v1[k] = row_D<EPI>(p, it.b, it.h, qg);
         }
       };
@@ -1519,9 +1526,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             meta_kind[s] = kd;
             mbar_arrive_expect_tx(q_full + s, 2 * L::kTileBytes + (kd == 2 ? 2048 : 0));
-            tma_load_4d(smem + L::kQ + s * L::kTileBytes, &tq, q_full + s, 0, qt * kTile, it.h, it.b);
-            tma_load_4d(smem + L::kDO + s * L::kTileBytes, &tdo, q_full + s, 0, qt * kTile, it.h,
-                        it.b);
+            tma_load_4d(smem + L::kQ + s * L::kTileBytes, &tq, q_full + s, 0, it.sq.row0 + qt * kTile, it.h,
+                        it.sq.tma_b);
+            tma_load_4d(smem + L::kDO + s * L::kTileBytes, &tdo, q_full + s, 0,
+                        it.sq.row0 + qt * kTile, it.h, it.sq.tma_b);
             if (kd == 2)
               bulk_load(meta_bits + s * 512, p.bitsT + static_cast<int64_t>(pi) * 512, 2048,
                         q_full + s);
@@ -1692,10 +1700,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
       const int kg = x.t * kTile + row;
-      if (kg < p.Nk) {
-        uint4* dvp = reinterpret_cast<uint4*>(p.dv + x.b * p.dv_sb + static_cast<int64_t>(kg) * p.dv_sn +
+      if (kg < x.sq.limit) {
+        uint4* dvp = reinterpret_cast<uint4*>(p.dv + seq_row_offset(x.sq, p.dv_sb, p.dv_sn, kg) +
                                               x.h * p.dv_sh + 32 * g);
-        uint4* dkp = reinterpret_cast<uint4*>(p.dk + x.b * p.dk_sb + static_cast<int64_t>(kg) * p.dk_sn +
+        uint4* dkp = reinterpret_cast<uint4*>(p.dk + seq_row_offset(x.sq, p.dk_sb, p.dk_sn, kg) +
                                               x.h * p.dk_sh + 32 * g);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -1715,11 +1723,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WorkRef it = iter.cur;
       if (it.n == 0) {
         // No query attends to this k-tile: dK = dV = 0 on its rows.
-        const int rows = min(kTile, p.Nk - it.t * kTile);
+        const int rows = min(kTile, it.sq.limit - it.t * kTile);
         const int tid = threadIdx.x - kEpiWarp0 * 32;
-        zero_rows<D>(p.dk + it.b * p.dk_sb + static_cast<int64_t>(it.t * kTile) * p.dk_sn +
+        zero_rows<D>(p.dk + seq_row_offset(it.sq, p.dk_sb, p.dk_sn, it.t * kTile) +
                          it.h * p.dk_sh, p.dk_sn, rows, tid, 256);
-        zero_rows<D>(p.dv + it.b * p.dv_sb + static_cast<int64_t>(it.t * kTile) * p.dv_sn +
+        zero_rows<D>(p.dv + seq_row_offset(it.sq, p.dv_sb, p.dv_sn, it.t * kTile) +
                          it.h * p.dv_sh, p.dv_sn, rows, tid, 256);
         continue;
       }
@@ -1854,8 +1862,9 @@ __global__ void dq_zero_kernel(const int4* __restrict__ row_desc, int rows_nonem
 // dQ = bf16(scale * dQacc) on rows of q-tiles with tiles, 0 on every other row.  One thread
 // per 8 elements (16 bytes of dQ).
 __global__ void dq_convert_kernel(const int32_t* __restrict__ row_ptr, const float* __restrict__ dqacc,
-                                  int B, int QT, int Nq, int H, float scale,
-                                  __nv_bfloat16* __restrict__ dq, int64_t sb, int64_t sn, int64_t sh) {
+                                  int B, int QT, int Nq, int H, const int32_t* __restrict__ cu,
+                                  float scale, __nv_bfloat16* __restrict__ dq, int64_t sb, int64_t sn,
+                                  int64_t sh) {
   constexpr int kChunks = 64 / 8;
   const int64_t total = static_cast<int64_t>(B) * Nq * H * kChunks;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
@@ -1865,6 +1874,8 @@ __global__ void dq_convert_kernel(const int32_t* __restrict__ row_ptr, const flo
     const int64_t bq = i / (static_cast<int64_t>(kChunks) * H);
     const int q = static_cast<int>(bq % Nq), b = static_cast<int>(bq / Nq);
     const int r = b * QT + q / kTile;
+    const SeqRows sq = seq_rows(cu, b, Nq);
+    if (q >= sq.limit) continue;  // a packed sequence owns only its own rows
     uint4 out = make_uint4(0u, 0u, 0u, 0u);
     if (row_ptr[r + 1] > row_ptr[r]) {
       const float4* src = reinterpret_cast<const float4*>(dqacc + (bq * H + h) * 64 + c * 8);
@@ -1872,7 +1883,7 @@ __global__ void dq_convert_kernel(const int32_t* __restrict__ row_ptr, const flo
       out = make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
                        pack_bf16x2(e.x * scale, e.y * scale), pack_bf16x2(e.z * scale, e.w * scale));
     }
-    *reinterpret_cast<uint4*>(dq + b * sb + static_cast<int64_t>(q) * sn + h * sh + c * 8) = out;
+    *reinterpret_cast<uint4*>(dq + seq_row_offset(sq, sb, sn, q) + h * sh + c * 8) = out;
   }
 }
 
@@ -1909,6 +1920,7 @@ int launch_bwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.csc_map = plan->csc_map;
   p.row_desc = plan->row_desc;
   p.col_desc = plan->col_desc;
+  p.cu = plan->cu;
   p.B = plan->B;
   p.QT = plan->QT;
   p.KT = plan->KT;
@@ -1940,7 +1952,7 @@ int launch_bwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
     d_preprocess_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o.ptr), o.sb, o.sn, o.sh,
         static_cast<const __nv_bfloat16*>(dout.ptr), dout.sb, dout.sn, dout.sh, plan->B, plan->Nq,
-        H, workspace);
+        H, plan->cu, workspace);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   if (parts & SIGATTN_BWD_DKDV) {
@@ -1982,6 +1994,7 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
   p.bitsT = plan->bitsT;
   p.col_desc = plan->col_desc;
   p.row_desc = plan->row_desc;
+  p.cu = plan->cu;
   p.B = plan->B;
   p.QT = plan->QT;
   p.KT = plan->KT;
@@ -2009,7 +2022,7 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
     d_preprocess_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o.ptr), o.sb, o.sn, o.sh,
         static_cast<const __nv_bfloat16*>(dout.ptr), dout.sb, dout.sn, dout.sh, plan->B, plan->Nq,
-        H, Dws);
+        H, plan->cu, Dws);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   const int sms = num_sms();
@@ -2035,7 +2048,7 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
     const int64_t work = static_cast<int64_t>(plan->B) * plan->Nq * H * (D / 8);
     const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, sms * 8)));
     dq_convert_kernel<<<blocks, 256, 0, stream>>>(plan->row_ptr, dqacc, plan->B, plan->QT, plan->Nq,
-                                                   H, scale,
+                                                   H, plan->cu, scale,
                                                    static_cast<__nv_bfloat16*>(const_cast<void*>(dq.ptr)),
                                                    dq.sb, dq.sn, dq.sh);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);

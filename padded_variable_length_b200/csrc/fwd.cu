@@ -51,6 +51,9 @@ struct FwdParams {
   const int32_t* pidx;
   const uint32_t* bits;
   const int4* row_desc;
+  const int32_t* cu;  // packed batches: cumulative row offsets [B + 1]; nullptr when padded
+  const int4* run;  // runs of consecutive k-tiles of one kind (see sigattn_plan)
+  int run_cap;      // entries allocated in run (reads stay below it)
   int QT, Nq, H, nitems;
   float scale;
   const float* bias;
@@ -76,8 +79,8 @@ struct FwdLayout {
   static constexpr int kMetaKind = kMetaBits + kStages * 2048;
   static constexpr int kBar = kMetaKind + 16 * ((kStages * 4 + 15) / 16);
   // q_full[2] q_empty[2] o_full[2] o_empty[2] s_full[2] p_full[2] pv_done
-  // k_full[S] v_full[S] kv_empty[S]
-  static constexpr int kNumBars = 13 + 3 * kStages;
+  // k_full[S] v_full[S] kv_empty[S] done
+  static constexpr int kNumBars = 14 + 3 * kStages;
   static constexpr int kRed = kBar + 8 * kNumBars;      // float [2][2][128] row maxima
   static constexpr int kRedL = kRed + 2 * 2 * 128 * 4;  // float [2][128] row sums
   static constexpr int kMisc = kRedL + 2 * 128 * 4;      // tmem base, abort, drain flags
@@ -86,7 +89,8 @@ struct FwdLayout {
 };
 
 struct Item {
-  int b, qt, h, e0, n;
+  int b, qt, h, e0, n, run0;  // run0: the row's first run
+  SeqRows sq;                 // where the rows of sequence b live (padded or packed)
 };
 
 __device__ __forceinline__ Item decode_item(const FwdParams& p, int w) {
@@ -97,6 +101,8 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p, int w) {
   it.qt = d.x % p.QT;
   it.e0 = d.y;
   it.n = d.z;
+  it.run0 = d.w;
+  it.sq = seq_rows(p.cu, it.b, p.Nq);
   return it;
 }
 
@@ -143,6 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_full = bars + 13;   // [S]
   uint64_t* v_full = bars + 13 + S;
   uint64_t* kv_empty = bars + 13 + 2 * S;
+  uint64_t* done = bars + 13 + 3 * S;  // every MMA complete (end of the kernel)
   uint32_t* meta_bits = reinterpret_cast<uint32_t*>(smem + L::kMetaBits);
   int* meta_kind = reinterpret_cast<int*>(smem + L::kMetaKind);
   float* red_max = reinterpret_cast<float*>(smem + L::kRed);
@@ -167,6 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(v_full + i, 1);
       mbar_init(kv_empty + i, 1);
     }
+    mbar_init(done, 1);
     *abort_flag = 0;
     *drain_flag = 0;
     fence_barrier_init();
@@ -199,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(q_full + qb, L::kTileBytes);
           for (int x = 0; x < L::kBoxes; ++x)
             tma_load_4d(smem + L::kQ + qb * L::kTileBytes + x * L::kBoxBytes, &tq, q_full + qb,
-                        x * 64, it.qt * kTile, it.h, it.b);
+                        x * 64, it.sq.row0 + it.qt * kTile, it.h, it.sq.tma_b);
         }
       }
       ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
@@ -226,14 +234,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_expect_tx(k_full + s, L::kTileBytes + (kd == 2 ? 2048 : 0));
               for (int x = 0; x < L::kBoxes; ++x)
                 tma_load_4d(smem + L::kK + s * L::kTileBytes + x * L::kBoxBytes, &tk, k_full + s,
-                            x * 64, kt * kTile, it.h, it.b);
+                            x * 64, it.sq.row0 + kt * kTile, it.h, it.sq.tma_b);
               if (kd == 2)
                 bulk_load(meta_bits + s * 512, p.bits + static_cast<int64_t>(pi) * 512, 2048,
                           k_full + s);
               mbar_arrive_expect_tx(v_full + s, L::kTileBytes);
               for (int x = 0; x < L::kBoxes; ++x)
                 tma_load_4d(smem + L::kV + s * L::kTileBytes + x * L::kBoxBytes, &tv, v_full + s,
-                            x * 64, kt * kTile, it.h, it.b);
+                            x * 64, it.sq.row0 + kt * kTile, it.h, it.sq.tma_b);
             }
           }
           ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
@@ -313,6 +321,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++i;
       }
       if (ok && pv_t >= 0) issue_pv();
+      // every MMA complete before the TMEM is released (also after an abort)
+      mma_commit_w(done);
+      const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
+      mbar_wait_w(done, 0, drain);
     }
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- softmax epilogue
@@ -330,7 +342,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int t = 0, i = 0;
     auto row_bias = [&](const Item& x) {
       const int r = x.qt * kTile + row;
-      return (p.bias != nullptr && x.n > 0 && r < p.Nq) ? p.bias[x.b * p.bias_sb + r] : 0.0f;
+      return (p.bias != nullptr && x.n > 0 && r < x.sq.limit)
+                 ? p.bias[static_cast<int64_t>(x.sq.tma_b) * p.bias_sb + x.sq.row0 + r]
+                 : 0.0f;
     };
     ItemIter iter(p);
     float bias_cur = iter.valid() ? row_bias(iter.cur) : 0.0f;
@@ -341,16 +355,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float bias_r = bias_cur;
       bias_cur = bias_nxt;
       if (it.n == 0) {
-        const int rows = min(kTile, p.Nq - it.qt * kTile);
+        const int rows = min(kTile, it.sq.limit - it.qt * kTile);
         constexpr int kChunks = D / 8;
         const int tid = threadIdx.x - kEpiWarp0 * 32;
         for (int c = tid; c < rows * kChunks; c += 256) {
           const int rr = c / kChunks, ch = c % kChunks;
-          *reinterpret_cast<uint4*>(p.o + it.b * p.o_sb +
-                                    static_cast<int64_t>(it.qt * kTile + rr) * p.o_sn +
+          *reinterpret_cast<uint4*>(p.o + seq_row_offset(it.sq, p.o_sb, p.o_sn, it.qt * kTile + rr) +
                                     it.h * p.o_sh + ch * 8) = make_uint4(0u, 0u, 0u, 0u);
         }
-        for (int c = tid; c < rows; c += 256)
+        for (int c = tid; c < min(kTile, p.Nq - it.qt * kTile); c += 256)
           p.lse[(static_cast<int64_t>(it.b) * p.H + it.h) * p.Nq + it.qt * kTile + c] =
               EPI == 1 ? -INFINITY : 0.0f;
         continue;
@@ -467,10 +480,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(o_empty + ob);
-        if (rg < p.Nq) {
-          uint4* d4 = reinterpret_cast<uint4*>(p.o + it.b * p.o_sb +
-                                               static_cast<int64_t>(rg) * p.o_sn + it.h * p.o_sh +
-                                               g * kOc);
+        if (rg < it.sq.limit) {
+          uint4* d4 = reinterpret_cast<uint4*>(p.o + seq_row_offset(it.sq, p.o_sb, p.o_sn, rg) +
+                                               it.h * p.o_sh + g * kOc);
 #pragma unroll
           for (int c = 0; c < kOc / 8; ++c)
             d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
@@ -613,8 +625,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- producers
     // warp 0: Q of each item and the K ring (slot of tile u free after step u); warp 2:
     // the V ring (slot of tile u free after step u + 2); warp 3: each tile's kind and
-    // PARTIAL bitmask (slot released by the epilogue).  All 32 lanes fetch the list
-    // entries of the next 32 tiles in one round trip; lane 0 waits and issues the copies.
+    // PARTIAL bitmask (slot released by the epilogue).  A row is walked by its runs (ranges
+    // of consecutive k-tiles of one kind): all 32 lanes fetch the next 32 runs in one round
+    // trip, and within a run the k-tile and bitmask number just count up, with no per-tile
+    // list lookup.  Lane 0 waits and issues the copies.
     const int role = warp == 0 ? 0 : (warp == 2 ? 1 : 2);
     if (lane == 0 && role < 2) {
       tma_prefetch_desc(role == 0 ? &tk : &tv);
@@ -637,26 +651,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(q_full + qb, L::kTileBytes);
             for (int x = 0; x < L::kBoxes; ++x)
               tma_load_4d(smem + L::kQ + qb * L::kTileBytes + x * L::kBoxBytes, &tq, q_full + qb,
-                          x * 64, it.qt * kTile, it.h, it.b);
+                          x * 64, it.sq.row0 + it.qt * kTile, it.h, it.sq.tma_b);
           }
         }
         ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
       }
       ++i;
-      for (int j0 = 0; ok && j0 < it.n; j0 += 32) {
-        const int jj = j0 + lane;
-        int kt_l = 0, kd_l = 0, pi_l = 0;
-        if (jj < it.n) {
-          if (role < 2) kt_l = p.col_idx[it.e0 + jj];
-          else kd_l = p.kind[it.e0 + jj];
-        }
-        if (kd_l == 2) pi_l = p.pidx[it.e0 + jj];
-        const int jn = min(32, it.n - j0);
-        for (int u = 0; u < jn; ++u, ++t) {
-          const int kt = __shfl_sync(0xFFFFFFFFu, kt_l, u);
-          const int kd = __shfl_sync(0xFFFFFFFFu, kd_l, u);
-          const int pi = __shfl_sync(0xFFFFFFFFu, pi_l, u);
+      for (int rb = it.run0, left = it.n; ok && left > 0;) {
+        // lanes past the row's last run read other rows' runs, or unwritten entries below
+        // run_cap: their values are never used, and the pidx index is kept in bounds
+        int4 run_l = make_int4(0, 0, 0, 0);
+        if (rb + lane < p.run_cap) run_l = p.run[rb + lane];
+        int pi0_l = 0;
+        if (role == 2 && run_l.z == 2 && run_l.w >= 0 && run_l.w < p.run_cap)
+          pi0_l = p.pidx[run_l.w];  // first bitmask number of a PARTIAL run
+        int used = 0;
+        for (int v = 0; ok && v < 32 && left > 0; ++v, ++used) {
+          const int kt0 = __shfl_sync(0xFFFFFFFFu, run_l.x, v);
+          const int len = __shfl_sync(0xFFFFFFFFu, run_l.y, v);
+          const int kd = __shfl_sync(0xFFFFFFFFu, run_l.z, v);
+          const int pi0 = __shfl_sync(0xFFFFFFFFu, pi0_l, v);
+          left -= len;
+        for (int u = 0; u < len; ++u, ++t) {
+          const int kt = kt0 + u;
+          const int pi = pi0 + u;
           const int s = t % NR;
           if (lane == 0) {
             if (t >= NR) {
@@ -673,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx(full + s, L::kTileBytes);
                 for (int x = 0; x < L::kBoxes; ++x)
                   tma_load_4d(smem + ring + s * L::kTileBytes + x * L::kBoxBytes, map, full + s,
-                              x * 64, kt * kTile, it.h, it.b);
+                              x * 64, it.sq.row0 + kt * kTile, it.h, it.sq.tma_b);
               } else {
                 meta_kind[s] = kd;
                 if (kd == 2) {
@@ -689,6 +708,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
           if (!ok) break;
         }
+        }
+        rb += used;
       }
     }
     if (lane == 0 && *abort_flag) {
@@ -803,7 +824,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     auto row_bias = [&](const Item& x) {
       const int r = x.qt * kTile + row;
-      return (p.bias != nullptr && x.n > 0 && r < p.Nq) ? p.bias[x.b * p.bias_sb + r] : 0.0f;
+      return (p.bias != nullptr && x.n > 0 && r < x.sq.limit)
+                 ? p.bias[static_cast<int64_t>(x.sq.tma_b) * p.bias_sb + x.sq.row0 + r]
+                 : 0.0f;
     };
     // O of the last item with tiles, written out late (see above)
     bool pend = false;
@@ -830,8 +853,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(o_empty + ob);
       const int rg = pit.qt * kTile + row;
-      if (rg < p.Nq) {
-        uint4* d4 = reinterpret_cast<uint4*>(p.o + pit.b * p.o_sb + static_cast<int64_t>(rg) * p.o_sn +
+      if (rg < pit.sq.limit) {
+        uint4* d4 = reinterpret_cast<uint4*>(p.o + seq_row_offset(pit.sq, p.o_sb, p.o_sn, rg) +
                                              pit.h * p.o_sh + g * kOc);
 #pragma unroll
         for (int c = 0; c < kOc / 8; ++c)
@@ -851,13 +874,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (it.n == 0) {
         // No tile in this row: the whole q-tile is padding or sees no key.  O = 0.
         if (pend) flush_o();
-        const int rows = min(kTile, p.Nq - it.qt * kTile);
+        const int rows = min(kTile, it.sq.limit - it.qt * kTile);
         constexpr int kChunks = D / 8;
         const int tid = threadIdx.x - kEpiWarp0 * 32;
         for (int c = tid; c < rows * kChunks; c += 256) {
           const int rr = c / kChunks, ch = c % kChunks;
-          *reinterpret_cast<uint4*>(p.o + it.b * p.o_sb +
-                                    static_cast<int64_t>(it.qt * kTile + rr) * p.o_sn +
+          *reinterpret_cast<uint4*>(p.o + seq_row_offset(it.sq, p.o_sb, p.o_sn, it.qt * kTile + rr) +
                                     it.h * p.o_sh + ch * 8) = make_uint4(0u, 0u, 0u, 0u);
         }
         continue;
@@ -954,6 +976,9 @@ int launch_fwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.pidx = plan->pidx;
   p.bits = plan->bits;
   p.row_desc = plan->row_desc;
+  p.cu = plan->cu;
+  p.run = plan->run;
+  p.run_cap = static_cast<int>(plan->nonempty);
   p.QT = plan->QT;
   p.Nq = plan->Nq;
   p.H = H;

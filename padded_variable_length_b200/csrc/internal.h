@@ -16,6 +16,10 @@
 //   col_work[B*KT]  every (b, k-tile) column, columns with no tile last
 struct sigattn_plan {
   int device;
+  // packed batches only (else nullptr / 0): device copy of the cumulative offsets [B + 1]
+  // and the total number of rows T = cu[B]
+  int32_t* cu;
+  int64_t T;
   void* arena[2];  // the two device allocations every buffer below is carved from
   int B, Nq, Nk, QT, KT;
   int64_t nonempty, full, partial;
@@ -32,7 +36,8 @@ struct sigattn_plan {
   int32_t* row_work;
   int32_t* col_work;
   // the work lists again, one 16-byte record per entry: {row or column, first list entry,
-  // number of entries, 0}, so that a kernel decodes a work item with one independent load
+  // number of entries, first run (rows) or 0 (columns)}, so that a kernel decodes a work
+  // item with one independent load
   int4* row_desc;
   int4* col_desc;
   // runs of each q-tile row: maximal ranges of consecutive k-tiles of one kind, one 16-byte
@@ -45,6 +50,28 @@ struct sigattn_plan {
 namespace sigattn {
 
 constexpr int kTile = 128;
+
+// Where the rows of sequence b live.  Padded batches index tensors by (b, row) with a batch
+// stride; a packed batch (a plan built from cumulative offsets cu[0..B]) keeps sequence b in
+// rows cu[b] .. cu[b+1] of one [T, H, d] tensor, so it has no batch coordinate, its rows
+// start at cu[b], and only its own n_b = cu[b+1] - cu[b] rows may be written.
+struct SeqRows {
+  int tma_b;  // batch coordinate for the TMA maps (0 when packed)
+  int row0;   // first row of the sequence in the token dimension (0 when padded)
+  int limit;  // rows of the sequence present in the tensors (N when padded, n_b when packed)
+};
+
+__host__ __device__ __forceinline__ SeqRows seq_rows(const int32_t* cu, int b, int N) {
+  if (cu == nullptr) return SeqRows{b, 0, N};
+  const int a = cu[b];
+  return SeqRows{0, a, cu[b + 1] - a};
+}
+
+// Element offset of row r of a sequence in a tensor with batch / token strides sb, sn.
+__host__ __device__ __forceinline__ int64_t seq_row_offset(const SeqRows& s, int64_t sb, int64_t sn,
+                                                          int r) {
+  return static_cast<int64_t>(s.tma_b) * sb + static_cast<int64_t>(s.row0 + r) * sn;
+}
 
 // Per-tensor description handed to the launchers (element strides).
 struct TensorDesc {

@@ -18,6 +18,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "internal.h"
 
@@ -114,28 +115,39 @@ __global__ void __launch_bounds__(256) k_kinds_from_mask(const uint8_t* __restri
 
 // One warp per q-tile row r < rows (number of listed blocks and of PARTIAL blocks), then
 // one warp per k-tile column c = b*KT + kt (number of listed blocks).
+// A listed block starts a run iff the block before it in the row is not listed or is of
+// the other kind (runs: maximal ranges of consecutive k-tiles of one kind).
+__device__ __forceinline__ bool starts_run(const uint8_t* __restrict__ k, int kt, uint8_t v) {
+  return v != 0 && (kt == 0 || k[kt - 1] != v);
+}
+
+// Row r < rows: number of listed blocks, of PARTIAL blocks and of runs; then one warp per
+// k-tile column c = b*KT + kt: number of listed blocks.
 __global__ void k_count(const uint8_t* __restrict__ kinds, int B, int QT, int KT,
                         int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_pcnt,
-                        int32_t* __restrict__ col_cnt) {
+                        int32_t* __restrict__ run_cnt, int32_t* __restrict__ col_cnt) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int rows = B * QT;
   if (warp < rows) {
     const uint8_t* k = kinds + static_cast<int64_t>(warp) * KT;
-    int c = 0, p = 0;
+    int c = 0, p = 0, n = 0;
     for (int kt = lane; kt < KT; kt += 32) {
       const uint8_t v = k[kt];
       c += v != 0;
       p += v == 2;
+      n += starts_run(k, kt, v);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
       p += __shfl_xor_sync(0xFFFFFFFFu, p, o);
+      n += __shfl_xor_sync(0xFFFFFFFFu, n, o);
     }
     if (lane == 0) {
       row_cnt[warp] = c;
       row_pcnt[warp] = p;
+      run_cnt[warp] = n;
     }
     return;
   }
@@ -183,12 +195,12 @@ struct ScanJob {
   int64_t* total;
 };
 
-// One CTA of 1024 threads per job (blockIdx.x picks one of three), walking its input in
+// One CTA of 1024 threads per job (blockIdx.x picks one of four), walking its input in
 // chunks of 1024.
-__global__ void __launch_bounds__(1024) k_scan3(ScanJob j0, ScanJob j1, ScanJob j2) {
+__global__ void __launch_bounds__(1024) k_scan4(ScanJob j0, ScanJob j1, ScanJob j2, ScanJob j3) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t chunk_total;
-  const ScanJob j = blockIdx.x == 0 ? j0 : (blockIdx.x == 1 ? j1 : j2);
+  const ScanJob j = blockIdx.x == 0 ? j0 : (blockIdx.x == 1 ? j1 : (blockIdx.x == 2 ? j2 : j3));
   int carry = 0;
   for (int base = 0; base < j.n; base += 1024) {
     const int i = base + threadIdx.x;
@@ -280,31 +292,33 @@ __global__ void __launch_bounds__(1024) k_sort_longest_first(SortJob j0, SortJob
 
 // One warp per q-tile row: CSR entries in ascending kt, the PARTIAL numbering, the dense
 // entry index of every listed block and the block of every PARTIAL number.
-// A listed block starts a run iff the block before it in the row is not listed or of the
-// other kind (runs: maximal ranges of consecutive k-tiles of one kind).  Also counts the
-// runs of every row into run_cnt.
+// One warp per q-tile row: CSR entries in ascending kt, the PARTIAL numbering, the dense
+// entry index of every listed block, the block of every PARTIAL number, and the row's runs
+// {first k-tile, number of tiles, kind, first CSR entry} at run[run_ptr[r] ..).
 __global__ void k_fill_csr(const uint8_t* __restrict__ kinds, int rows, int KT,
                            const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ row_poff,
                            int32_t* __restrict__ col_idx, uint8_t* __restrict__ kind,
                            int32_t* __restrict__ pidx, int32_t* __restrict__ eidx,
-                           int64_t* __restrict__ ptile, int32_t* __restrict__ run_cnt) {
+                           int64_t* __restrict__ ptile, const int32_t* __restrict__ run_ptr,
+                           int4* __restrict__ run) {
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
   int e = row_ptr[r];
   int p = row_poff[r];
-  int runs = 0;
-  uint8_t carry = 0;  // kind of the block before this chunk
+  int rpos = run_ptr[r];
   const uint8_t* k = kinds + static_cast<int64_t>(r) * KT;
   for (int base = 0; base < KT; base += 32) {
     const int kt = base + lane;
     const uint8_t v = kt < KT ? k[kt] : 0;
-    const uint8_t before = static_cast<uint8_t>(__shfl_up_sync(0xFFFFFFFFu, v, 1));
-    const uint8_t prev = lane == 0 ? carry : before;
-    carry = static_cast<uint8_t>(__shfl_sync(0xFFFFFFFFu, v, 31));
-    runs += __popc(__ballot_sync(0xFFFFFFFFu, v != 0 && v != prev));
+    const bool start = kt < KT && starts_run(k, kt, v);
+    const unsigned sm = __ballot_sync(0xFFFFFFFFu, start);
     const unsigned nzm = __ballot_sync(0xFFFFFFFFu, v != 0);
     const unsigned pm = __ballot_sync(0xFFFFFFFFu, v == 2);
+    if (start)
+      run[rpos + __popc(sm & ((1u << lane) - 1u))] =
+          make_int4(kt, 0, v, e + __popc(nzm & ((1u << lane) - 1u)));
+    rpos += __popc(sm);
     const unsigned lt = (1u << lane) - 1u;
     if (v != 0) {
       const int my = e + __popc(nzm & lt);
@@ -321,33 +335,6 @@ __global__ void k_fill_csr(const uint8_t* __restrict__ kinds, int rows, int KT,
     }
     e += __popc(nzm);
     p += __popc(pm);
-  }
-  if (lane == 0) run_cnt[r] = runs;
-}
-
-// One warp per q-tile row: its runs {first k-tile, number of tiles, kind, first CSR entry}
-// in ascending order, at run[run_ptr[r] ..).
-__global__ void k_fill_runs(const uint8_t* __restrict__ kinds, const int32_t* __restrict__ eidx,
-                            int rows, int KT, const int32_t* __restrict__ row_ptr,
-                            const int32_t* __restrict__ run_ptr, int4* __restrict__ run) {
-  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
-  int pos = run_ptr[r];
-  uint8_t carry = 0;
-  const uint8_t* k = kinds + static_cast<int64_t>(r) * KT;
-  for (int base = 0; base < KT; base += 32) {
-    const int kt = base + lane;
-    const uint8_t v = kt < KT ? k[kt] : 0;
-    const uint8_t before = static_cast<uint8_t>(__shfl_up_sync(0xFFFFFFFFu, v, 1));
-    const uint8_t prev = lane == 0 ? carry : before;
-    carry = static_cast<uint8_t>(__shfl_sync(0xFFFFFFFFu, v, 31));
-    const bool start = v != 0 && v != prev;
-    const unsigned sm = __ballot_sync(0xFFFFFFFFu, start);
-    if (start)
-      run[pos + __popc(sm & ((1u << lane) - 1u))] =
-          make_int4(kt, 0, v, eidx[static_cast<int64_t>(r) * KT + kt]);
-    pos += __popc(sm);
   }
   __syncwarp();
   // length = first entry of the next run (or the row's end) minus the run's first entry
@@ -381,11 +368,23 @@ __global__ void k_fill_csc(const uint8_t* __restrict__ kinds, const int32_t* __r
   }
 }
 
-// One CTA of 256 threads per PARTIAL block: its 128 x 128 bitmask from the mask.
+// Thread k < 128 of a CTA: column k of the 128 x 128 bitmask w (512 words in shared memory,
+// bit (k % 32) of word (q*4 + k/32)), i.e. bit (q % 32) of word (k*4 + q/32) of the transpose.
+__device__ __forceinline__ void store_transposed(const uint32_t* w, uint32_t* __restrict__ dstT) {
+  const int k = threadIdx.x;
+  uint32_t out[4] = {0u, 0u, 0u, 0u};
+  for (int q = 0; q < 128; ++q) out[q >> 5] |= ((w[q * 4 + (k >> 5)] >> (k & 31)) & 1u) << (q & 31);
+  reinterpret_cast<uint4*>(dstT)[k] = make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// One CTA of 256 threads per PARTIAL block: its 128 x 128 bitmask from the mask, and the
+// transposed copy.
 __global__ void __launch_bounds__(256) k_bits_from_mask(const uint8_t* __restrict__ mask, int Nq,
                                                         int Nk, int64_t sb, int64_t sq, int QT,
                                                         int KT, const int64_t* __restrict__ ptile,
-                                                        uint32_t* __restrict__ bits) {
+                                                        uint32_t* __restrict__ bits,
+                                                        uint32_t* __restrict__ bitsT) {
+  __shared__ uint32_t w[512];
   const int64_t g = ptile[blockIdx.x];
   const int kt = static_cast<int>(g % KT);
   const int qt = static_cast<int>((g / KT) % QT);
@@ -397,14 +396,20 @@ __global__ void __launch_bounds__(256) k_bits_from_mask(const uint8_t* __restric
   uint32_t* dst = bits + static_cast<int64_t>(blockIdx.x) * 512 + q * 4 + half * 2;
   dst[0] = w0;
   dst[1] = w1;
+  w[q * 4 + half * 2] = w0;
+  w[q * 4 + half * 2 + 1] = w1;
+  __syncthreads();
+  if (threadIdx.x < 128) store_transposed(w, bitsT + static_cast<int64_t>(blockIdx.x) * 512);
 }
 
 // One CTA of 128 threads per PARTIAL block of a padded batch: row q is valid iff
-// qt*128 + q < n, column k iff kt*128 + k < n.
+// qt*128 + q < n, column k iff kt*128 + k < n.  Thread q writes row q of the bitmask and
+// (the same rule with the roles swapped) column q of the transposed copy.
 __global__ void __launch_bounds__(128) k_bits_from_lengths(const int32_t* __restrict__ lengths,
                                                            int Npad, int QT, int KT,
                                                            const int64_t* __restrict__ ptile,
-                                                           uint32_t* __restrict__ bits) {
+                                                           uint32_t* __restrict__ bits,
+                                                           uint32_t* __restrict__ bitsT) {
   const int64_t g = ptile[blockIdx.x];
   const int kt = static_cast<int>(g % KT);
   const int qt = static_cast<int>((g / KT) % QT);
@@ -418,13 +423,20 @@ __global__ void __launch_bounds__(128) k_bits_from_lengths(const int32_t* __rest
   w.z = row_ok ? low_bits(n - (kt * kTile + 64)) : 0u;
   w.w = row_ok ? low_bits(n - (kt * kTile + 96)) : 0u;
   reinterpret_cast<uint4*>(bits + static_cast<int64_t>(blockIdx.x) * 512)[q] = w;
+  const bool col_ok = kt * kTile + q < n;
+  uint4 wt;
+  wt.x = col_ok ? low_bits(n - (qt * kTile + 0)) : 0u;
+  wt.y = col_ok ? low_bits(n - (qt * kTile + 32)) : 0u;
+  wt.z = col_ok ? low_bits(n - (qt * kTile + 64)) : 0u;
+  wt.w = col_ok ? low_bits(n - (qt * kTile + 96)) : 0u;
+  reinterpret_cast<uint4*>(bitsT + static_cast<int64_t>(blockIdx.x) * 512)[q] = wt;
 }
 
-// desc[k] = {work[k], ptr[work[k]], ptr[work[k] + 1] - ptr[work[k]], 0} for the row list
-// (k < rows) and then the column list.
+// desc[k] = {work[k], ptr[work[k]], ptr[work[k] + 1] - ptr[work[k]], w} for the row list
+// (k < rows, w = the row's first run) and then the column list (w = 0).
 __global__ void k_work_desc(const int32_t* __restrict__ row_work, const int32_t* __restrict__ row_ptr,
-                            int rows, int4* __restrict__ row_desc,
-                            const int32_t* __restrict__ col_work,
+                            const int32_t* __restrict__ run_ptr, int rows,
+                            int4* __restrict__ row_desc, const int32_t* __restrict__ col_work,
                             const int32_t* __restrict__ col_ptr, int cols,
                             int4* __restrict__ col_desc) {
   for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < rows + cols; k += gridDim.x * blockDim.x) {
@@ -433,22 +445,8 @@ __global__ void k_work_desc(const int32_t* __restrict__ row_work, const int32_t*
     const int r = (is_row ? row_work : col_work)[kk];
     const int32_t* ptr = is_row ? row_ptr : col_ptr;
     const int a = ptr[r];
-    (is_row ? row_desc : col_desc)[kk] = make_int4(r, a, ptr[r + 1] - a, 0);
+    (is_row ? row_desc : col_desc)[kk] = make_int4(r, a, ptr[r + 1] - a, is_row ? run_ptr[r] : 0);
   }
-}
-
-// One CTA of 128 threads per PARTIAL block: thread k gathers column k of the bitmask.
-__global__ void __launch_bounds__(128) k_transpose_bits(const uint32_t* __restrict__ bits,
-                                                        uint32_t* __restrict__ bitsT) {
-  __shared__ uint32_t w[512];
-  const uint32_t* src = bits + static_cast<int64_t>(blockIdx.x) * 512;
-  for (int i = threadIdx.x; i < 512; i += 128) w[i] = src[i];
-  __syncthreads();
-  const int k = threadIdx.x;
-  uint32_t out[4] = {0u, 0u, 0u, 0u};
-  for (int q = 0; q < 128; ++q) out[q >> 5] |= ((w[q * 4 + (k >> 5)] >> (k & 31)) & 1u) << (q & 31);
-  reinterpret_cast<uint4*>(bitsT + static_cast<int64_t>(blockIdx.x) * 512)[k] =
-      make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 // Buffers are carved out of a few large allocations: a byte count laid out first (every
@@ -474,17 +472,54 @@ int alloc_status(cudaError_t e) {
   return e == cudaErrorMemoryAllocation ? SIGATTN_ERR_NOMEM : SIGATTN_ERR_CUDA;
 }
 
-// Plan memory (owned by the plan until sigattn_plan_destroy): cudaMalloc.
-int plan_alloc(void** p, size_t bytes) {
-  *p = nullptr;
-  return alloc_status(cudaMalloc(p, bytes > 0 ? bytes : 256));
+// All plan memory (the plan's arenas and the scratch of a build) comes from one memory pool
+// per device that keeps what it has reserved (release threshold: never), so that building a
+// plan after the first allocates nothing from the driver, and no allocation or free stalls
+// the device: allocations and frees are ordered on streams.
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[kMaxDevices] = {};
+
+int plan_pool(int dev, cudaMemPool_t* out) {
+  if (dev < 0 || dev >= kMaxDevices) return SIGATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_pool_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) return alloc_status(e);
+    uint64_t keep = UINT64_MAX;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return alloc_status(e);
+    }
+    g_pool[dev] = pool;
+  }
+  *out = g_pool[dev];
+  return SIGATTN_OK;
 }
 
-// Scratch of one plan build: stream-ordered, released on the stream at the end.
-int scratch_alloc(void** p, size_t bytes, cudaStream_t s) {
+int pool_alloc(void** p, size_t bytes, cudaStream_t s) {
   *p = nullptr;
-  return alloc_status(cudaMallocAsync(p, bytes > 0 ? bytes : 256, s));
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SIGATTN_ERR_NO_DEVICE;
+  }
+  cudaMemPool_t pool = nullptr;
+  const int rc = plan_pool(dev, &pool);
+  if (rc != SIGATTN_OK) return rc;
+  return alloc_status(cudaMallocFromPoolAsync(p, bytes > 0 ? bytes : 256, pool, s));
 }
+
+// Plan memory (owned by the plan until sigattn_plan_destroy).
+int plan_alloc(void** p, size_t bytes, cudaStream_t s) { return pool_alloc(p, bytes, s); }
+
+// Scratch of one plan build, released on the stream at the end.
+int scratch_alloc(void** p, size_t bytes, cudaStream_t s) { return pool_alloc(p, bytes, s); }
 
 struct Scratch {
   void* block[2] = {nullptr, nullptr};
@@ -505,9 +540,11 @@ struct Scratch {
   }
 };
 
+// The arenas go back to the pool in the order of the legacy default stream (the caller has
+// made sure that no kernel still uses the plan).
 void plan_free_buffers(sigattn_plan* p) {
   for (void*& a : p->arena) {
-    if (a) cudaFree(a);
+    if (a) cudaFreeAsync(a, cudaStreamLegacy);
     a = nullptr;
   }
 }
@@ -533,9 +570,12 @@ int grid_for(int64_t work, int per_block) {
 // Both planners: `classify` writes every block's kind into sc.kinds, `bits_kernel` the
 // bitmasks of the PARTIAL blocks.  Two plan allocations (one sized by the grid, one by the
 // number of listed tiles, known after the one synchronisation), two scratch allocations.
+// cu_src (packed batches only): the cumulative offsets, copied into the plan; check_dev /
+// check_host: one device int read back at the synchronisation (an argument check).
 template <class ClassifyFn, class BitsFn>
 int build_plan(sigattn_plan* plan, cudaStream_t stream, ClassifyFn classify, BitsFn bits_kernel,
-               sigattn_plan** out) {
+               sigattn_plan** out, const int32_t* cu_src = nullptr,
+               const int32_t* check_dev = nullptr, int32_t* check_host = nullptr) {
   Scratch sc;
   const int B = plan->B, QT = plan->QT, KT = plan->KT;
   const int rows = B * QT, cols = B * KT;
@@ -562,8 +602,8 @@ int build_plan(sigattn_plan* plan, cudaStream_t stream, ClassifyFn classify, Bit
     const size_t o_rptr = c.add<int32_t>(rows + 1), o_cptr = c.add<int32_t>(cols + 1),
                  o_rw = c.add<int32_t>(rows), o_cw = c.add<int32_t>(cols),
                  o_rd = c.add<int4>(rows), o_cd = c.add<int4>(cols),
-                 o_rp = c.add<int32_t>(rows + 1);
-    SIGATTN_TRY(plan_alloc(&plan->arena[0], c.bytes));
+                 o_rp = c.add<int32_t>(rows + 1), o_cu = c.add<int32_t>(cu_src ? B + 1 : 0);
+    SIGATTN_TRY(plan_alloc(&plan->arena[0], c.bytes, stream));
     void* m = plan->arena[0];
     plan->row_ptr = Carve::at<int32_t>(m, o_rptr);
     plan->colT_ptr = Carve::at<int32_t>(m, o_cptr);
@@ -572,23 +612,39 @@ int build_plan(sigattn_plan* plan, cudaStream_t stream, ClassifyFn classify, Bit
     plan->row_desc = Carve::at<int4>(m, o_rd);
     plan->col_desc = Carve::at<int4>(m, o_cd);
     plan->run_ptr = Carve::at<int32_t>(m, o_rp);
+    if (cu_src) {
+      plan->cu = Carve::at<int32_t>(m, o_cu);
+      SIGATTN_TRY_CUDA(cudaMemcpyAsync(plan->cu, cu_src, (B + 1) * sizeof(int32_t),
+                                       cudaMemcpyDeviceToDevice, stream));
+    }
   }
   classify(sc.kinds);
   k_count<<<grid_for(static_cast<int64_t>(rows + cols) * 32, 256), 256, 0, stream>>>(
-      sc.kinds, B, QT, KT, sc.row_cnt, sc.row_pcnt, sc.col_cnt);
-  k_scan3<<<3, 1024, 0, stream>>>(ScanJob{sc.row_cnt, rows, plan->row_ptr, sc.totals + 0},
+      sc.kinds, B, QT, KT, sc.row_cnt, sc.row_pcnt, sc.run_cnt, sc.col_cnt);
+  k_scan4<<<4, 1024, 0, stream>>>(ScanJob{sc.row_cnt, rows, plan->row_ptr, sc.totals + 0},
                                   ScanJob{sc.row_pcnt, rows, sc.row_poff, sc.totals + 1},
-                                  ScanJob{sc.col_cnt, cols, plan->colT_ptr, nullptr});
+                                  ScanJob{sc.col_cnt, cols, plan->colT_ptr, nullptr},
+                                  ScanJob{sc.run_cnt, rows, plan->run_ptr, nullptr});
   k_sort_longest_first<<<2, 1024, 0, stream>>>(SortJob{sc.row_cnt, rows, plan->row_work, sc.totals + 2},
                                                SortJob{sc.col_cnt, cols, plan->col_work, sc.totals + 3});
   k_work_desc<<<grid_for(rows + cols, 256), 256, 0, stream>>>(
-      plan->row_work, plan->row_ptr, rows, plan->row_desc, plan->col_work, plan->colT_ptr, cols,
-      plan->col_desc);
+      plan->row_work, plan->row_ptr, plan->run_ptr, rows, plan->row_desc, plan->col_work,
+      plan->colT_ptr, cols, plan->col_desc);
   SIGATTN_TRY_CUDA(cudaGetLastError());
   int64_t totals[4] = {0, 0, 0, 0};
+  int32_t last_row = 0;
   SIGATTN_TRY_CUDA(cudaMemcpyAsync(totals, sc.totals, sizeof(totals), cudaMemcpyDeviceToHost,
                                    stream));
+  if (cu_src)
+    SIGATTN_TRY_CUDA(cudaMemcpyAsync(&last_row, cu_src + B, sizeof(int32_t), cudaMemcpyDeviceToHost,
+                                     stream));
+  if (check_dev)
+    SIGATTN_TRY_CUDA(cudaMemcpyAsync(check_host, check_dev, sizeof(int32_t), cudaMemcpyDeviceToHost,
+                                     stream));
   SIGATTN_TRY_CUDA(cudaStreamSynchronize(stream));
+  if (check_host && *check_host != 0) SIGATTN_TRY(SIGATTN_ERR_INVALID);
+  if (cu_src && last_row < 1) SIGATTN_TRY(SIGATTN_ERR_INVALID);  // a packed batch needs rows
+  plan->T = last_row;
   plan->nonempty = totals[0];
   plan->partial = totals[1];
   plan->full = totals[0] - totals[1];
@@ -601,7 +657,7 @@ int build_plan(sigattn_plan* plan, cudaStream_t stream, ClassifyFn classify, Bit
                  o_ri = c.add<int32_t>(nz), o_cm = c.add<int32_t>(nz),
                  o_b = c.add<uint32_t>(np * 512), o_bt = c.add<uint32_t>(np * 512),
                  o_run = c.add<int4>(nz);  // at most one run per listed tile
-    SIGATTN_TRY(plan_alloc(&plan->arena[1], c.bytes));
+    SIGATTN_TRY(plan_alloc(&plan->arena[1], c.bytes, stream));
     void* m = plan->arena[1];
     plan->col_idx = Carve::at<int32_t>(m, o_ci);
     plan->kind = Carve::at<uint8_t>(m, o_k);
@@ -617,21 +673,12 @@ int build_plan(sigattn_plan* plan, cudaStream_t stream, ClassifyFn classify, Bit
   if (plan->nonempty > 0) {
     k_fill_csr<<<grid_for(static_cast<int64_t>(rows) * 32, 256), 256, 0, stream>>>(
         sc.kinds, rows, KT, plan->row_ptr, sc.row_poff, plan->col_idx, plan->kind, plan->pidx,
-        sc.eidx, sc.ptile, sc.run_cnt);
+        sc.eidx, sc.ptile, plan->run_ptr, plan->run);
     k_fill_csc<<<grid_for(static_cast<int64_t>(cols) * 32, 256), 256, 0, stream>>>(
         sc.kinds, sc.eidx, B, QT, KT, plan->colT_ptr, plan->rowT_idx, plan->csc_map);
-    const ScanJob runs{sc.run_cnt, rows, plan->run_ptr, nullptr};
-    k_scan3<<<1, 1024, 0, stream>>>(runs, runs, runs);
-    k_fill_runs<<<grid_for(static_cast<int64_t>(rows) * 32, 256), 256, 0, stream>>>(
-        sc.kinds, sc.eidx, rows, KT, plan->row_ptr, plan->run_ptr, plan->run);
-  } else {
-    SIGATTN_TRY_CUDA(cudaMemsetAsync(plan->run_ptr, 0, (rows + 1) * sizeof(int32_t), stream));
   }
-  if (plan->partial > 0) {
-    bits_kernel(sc.ptile, plan->bits, static_cast<int>(plan->partial));
-    k_transpose_bits<<<static_cast<unsigned>(plan->partial), 128, 0, stream>>>(plan->bits,
-                                                                               plan->bitsT);
-  }
+  if (plan->partial > 0)
+    bits_kernel(sc.ptile, plan->bits, plan->bitsT, static_cast<int>(plan->partial));
   SIGATTN_TRY_CUDA(cudaGetLastError());
   sc.release(stream);
   *out = plan;
@@ -673,10 +720,68 @@ extern "C" int sigattn_plan_from_lengths(const int32_t* d_lengths, int B, int Np
     k_kinds_from_lengths<<<grid_for(grid_total, 256), 256, 0, stream>>>(d_lengths, B, Npad, QT,
                                                                           QT, kinds);
   };
-  auto bits = [&](const int64_t* ptile, uint32_t* dst, int np) {
-    k_bits_from_lengths<<<np, 128, 0, stream>>>(d_lengths, Npad, QT, QT, ptile, dst);
+  auto bits = [&](const int64_t* ptile, uint32_t* dst, uint32_t* dstT, int np) {
+    k_bits_from_lengths<<<np, 128, 0, stream>>>(d_lengths, Npad, QT, QT, ptile, dst, dstT);
   };
   return build_plan(plan, stream, classify, bits, out);
+}
+
+namespace sigattn {
+namespace {
+
+// lengths[b] = cu[b+1] - cu[b]; *bad = 1 if a length is negative or above maxlen.
+__global__ void k_lengths_from_cu(const int32_t* __restrict__ cu, int B, int maxlen,
+                                  int32_t* __restrict__ lengths, int32_t* __restrict__ bad) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x) {
+    const int n = cu[b + 1] - cu[b];
+    lengths[b] = n;
+    if (n < 0 || n > maxlen) atomicOr(bad, 1);
+  }
+}
+
+}  // namespace
+}  // namespace sigattn
+
+extern "C" int sigattn_plan_from_cu_seqlens(const int32_t* d_cu, int B, int max_seqlen,
+                                            sigattn_stream s, sigattn_plan** out) {
+  if (!out) return SIGATTN_ERR_INVALID;
+  *out = nullptr;
+  if (!d_cu || B < 1 || max_seqlen < 1) return SIGATTN_ERR_INVALID;
+  const int QT = (max_seqlen + kTile - 1) / kTile;
+  if (static_cast<int64_t>(B) * QT * QT > kMaxGrid) return SIGATTN_ERR_UNSUPPORTED;
+  cudaStream_t stream = static_cast<cudaStream_t>(s);
+  // lengths and the argument check live in a scratch block of their own, released at the end
+  void* tmp = nullptr;
+  int rc = scratch_alloc(&tmp, static_cast<size_t>(B + 1) * sizeof(int32_t) + 256, stream);
+  if (rc != SIGATTN_OK) return rc;
+  int32_t* lengths = static_cast<int32_t*>(tmp);
+  int32_t* bad = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(tmp) +
+                                            ((static_cast<size_t>(B) * 4 + 255) & ~size_t(255)));
+  cudaMemsetAsync(bad, 0, sizeof(int32_t), stream);
+  k_lengths_from_cu<<<grid_for(B, 256), 256, 0, stream>>>(d_cu, B, max_seqlen, lengths, bad);
+  sigattn_plan* plan = new sigattn_plan();
+  std::memset(plan, 0, sizeof(*plan));
+  rc = current_device(&plan->device);
+  if (rc != SIGATTN_OK) {
+    delete plan;
+    cudaFreeAsync(tmp, stream);
+    return rc;
+  }
+  plan->B = B;
+  plan->Nq = plan->Nk = max_seqlen;
+  plan->QT = plan->KT = QT;
+  const int64_t grid_total = static_cast<int64_t>(B) * QT * QT;
+  auto classify = [&](uint8_t* kinds) {
+    k_kinds_from_lengths<<<grid_for(grid_total, 256), 256, 0, stream>>>(lengths, B, max_seqlen, QT,
+                                                                          QT, kinds);
+  };
+  auto bits = [&](const int64_t* ptile, uint32_t* dst, uint32_t* dstT, int np) {
+    k_bits_from_lengths<<<np, 128, 0, stream>>>(lengths, max_seqlen, QT, QT, ptile, dst, dstT);
+  };
+  int32_t bad_host = 0;
+  rc = build_plan(plan, stream, classify, bits, out, d_cu, bad, &bad_host);
+  cudaFreeAsync(tmp, stream);
+  return rc;
 }
 
 extern "C" int sigattn_plan_from_mask(const uint8_t* d_mask, int B, int Nq, int Nk,
@@ -703,9 +808,9 @@ extern "C" int sigattn_plan_from_mask(const uint8_t* d_mask, int B, int Nq, int 
     k_kinds_from_mask<<<static_cast<unsigned>(grid_total), 256, 0, stream>>>(
         d_mask, B, Nq, Nk, stride_b, stride_q, QT, KT, kinds);
   };
-  auto bits = [&](const int64_t* ptile, uint32_t* dst, int np) {
+  auto bits = [&](const int64_t* ptile, uint32_t* dst, uint32_t* dstT, int np) {
     k_bits_from_mask<<<np, 256, 0, stream>>>(d_mask, Nq, Nk, stride_b, stride_q, QT, KT, ptile,
-                                             dst);
+                                             dst, dstT);
   };
   return build_plan(plan, stream, classify, bits, out);
 }

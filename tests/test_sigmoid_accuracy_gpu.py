@@ -9,7 +9,9 @@ real kernels:
 * a sweep: one key direction, q_i = alpha_i e_0 and k_j = e_0 with scale 1/8, so that the
   score of query i is exactly x_i = alpha_i / 8, swept over [-30, 10]; every weight of row i
   is sigma(x_i), so O, dV, dQ and dK are sigma(x_i), sigma'(x_i) times exactly known factors,
-  and each element is checked against float64 to 2^-8 relative (two bf16 roundings);
+  and each element is checked against float64 to 2^-8 + 1e-3 relative (two bf16 roundings
+  and the sigmoid's own error) -- the hardware tanh form misses this by 1.4 % at x = -10
+  and by 100 % below x = -12;
 * the Q = 0 closed form at long n: every weight is sigma(-log n) = 1 / (n + 1), so row i of
   O is sum_{j<n} v_j / (n + 1) and dV_j = sum_{i<n} dO_i / (n + 1), checked row by row to
   2^-7 relative.
@@ -25,7 +27,9 @@ from tests import harness as Hn
 
 pytestmark = pytest.mark.gpu
 
-REL = 2.0 ** -8
+# Two bf16 roundings (the weight or dS fed to the MMA, and the output), 2^-9 each, plus the
+# relative error of the kernels' sigmoid (3.0e-4) and of sigma' = e g^2 (twice that).
+REL = 2.0 ** -8 + 1e-3
 
 
 def _sigma(x):
@@ -72,10 +76,11 @@ def test_sigmoid_sweep_through_the_kernels(kind):
         keys = 64
     assert plan.sizes()["full" if kind == "full" else "partial"] == 1
     dq_, dk_, dv_, do_ = (t.cuda() for t in (q, k, v, do))
-    o, _ = Bd.fwd(plan, dq_, dk_, dv_, None)
-    gq, gk, gv = Bd.bwd(plan, dq_, dk_, dv_, o, do_, None)
+    o_dev, _ = Bd.fwd(plan, dq_, dk_, dv_, None)
+    grads = {"split": Bd.bwd(plan, dq_, dk_, dv_, o_dev, do_, None),
+             "fused": Bd.bwd_fused(plan, dq_, dk_, dv_, o_dev, do_, None)}
     assert Bd.get_status() == 0
-    o, gq, gk, gv = (Hn.to_f64(t)[0] for t in (o, gq, gk, gv))  # [N, H, d]
+    o = Hn.to_f64(o_dev)[0]  # [N, H, d]
     s = _sigma(x)                         # [H, 64]
     sp = s * (1.0 - s)
     for h in range(H):
@@ -83,20 +88,25 @@ def test_sigmoid_sweep_through_the_kernels(kind):
         want_o = keys / 128.0 * _sigma(xs_h)
         np.testing.assert_allclose(o[:, h, 0], want_o, rtol=REL, atol=0, err_msg=f"O head {h}")
         assert np.all(o[:, h, 1:] == 0)
+    for algo, g in grads.items():
+        _check_grads(algo, *(Hn.to_f64(t)[0] for t in g), x, s, sp, keys, H)
+
+
+def _check_grads(algo, gq, gk, gv, x, s, sp, keys, H):
     for h in (0, 1):
         want = 2.0 * s[h]
         np.testing.assert_allclose(gv[:keys, h, :], np.broadcast_to(want, (keys, 64)), rtol=REL,
-                                   atol=0, err_msg=f"dV head {h}")
+                                   atol=0, err_msg=f"{algo} dV head {h}")
         assert np.all(gv[keys:, h] == 0)
     for h in (2, 3):
         sp_h = np.concatenate([sp[h], sp[h]])
         np.testing.assert_allclose(gq[:, h, 0], keys * sp_h / 1024.0, rtol=REL, atol=0,
-                                   err_msg=f"dQ head {h}")
+                                   err_msg=f"{algo} dQ head {h}")
         # dK_j[0] = (1/8) sum_i alpha_i ds_ij with ds_ij = sigma'(x_i) / 128, a signed sum
         alpha = 8.0 * np.concatenate([x[h], x[h]])
         terms = alpha * sp_h / 128.0 / 8.0
         err = np.abs(gk[:keys, h, 0] - terms.sum())
-        assert np.all(err <= REL * np.abs(terms).sum() + 1e-30), f"dK head {h}"
+        assert np.all(err <= REL * np.abs(terms).sum() + 1e-30), f"{algo} dK head {h}"
         assert np.all(gk[keys:, h] == 0)
 
 
