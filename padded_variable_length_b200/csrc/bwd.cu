@@ -1386,7 +1386,7 @@ struct FusedLayout {
   static constexpr int kQ = kV + kKVBufs * kTileBytes;
   static constexpr int kDO = kQ + kStages * kTileBytes;
   static constexpr int kDS = kDO + kStages * kTileBytes;       // dS, two 64-query boxes
-  static constexpr int kStg = kDS + 2 * kTileBytes;            // dQ staging, 2 KB per warp
+  static constexpr int kStg = kDS + 2 * kTileBytes;            // dQ staging, 2 x 2 KB per drain warp
   static constexpr int kVec = kStg + 8 * 2048;                 // float [S][2][128]
   static constexpr int kMetaBits = kVec + kStages * 2 * 128 * 4;
   static constexpr int kMetaKind = kMetaBits + kStages * 2048;
@@ -1400,8 +1400,12 @@ struct FusedLayout {
   static_assert(kStages * 4 <= 16, "meta kinds");
 };
 
+// 14 warps: 0 producer, 1 MMA issuer, 4-11 epilogue, and 2, 3, 12, 13 the dQ drain (one
+// warp per TMEM lane quarter: warp w reaches lanes [32 (w % 4), +32)).
+constexpr int kFusedThreads = 448;
+
 template <int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFusedThreads, 1)
     fused_bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                      const __grid_constant__ CUtensorMap tdq, const BwdParams p) {
@@ -1442,7 +1446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(sdp_full + i, 1);
       mbar_init(p_full + i, 8);
       mbar_init(dq_full + i, 1);
-      mbar_init(x_free + i, 8);
+      mbar_init(x_free + i, 4);  // the four drain warps
     }
     for (int i = 0; i < S; ++i) {
       mbar_init(q_full + i, 2);  // TMA bytes + the producer's column vectors
@@ -1635,7 +1639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
       mbar_wait_w(done, 0, drain);
     }
-  } else if (warp >= kEpiWarp0) {
+  } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 8) {
     // ---------------------------------------------------------------- epilogue
     // Warpgroup g owns queries [64g, 64g+64) of every tile; thread = key row (TMEM lane).
     const int g = (warp - kEpiWarp0) >> 2;
@@ -1645,47 +1649,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c1s = p.scale * kLog2e;
     const float2 c1 = make_float2(c1s, c1s);
     uint8_t* ds_box = smem + L::kDS + g * L::kTileBytes;          // this warpgroup's queries
-    uint8_t* stg = smem + L::kStg + (warp - kEpiWarp0) * 2048;   // this warp's dQ staging
     bool ok = true;
-    // previous tile (its dQ is drained one tile late) and previous item (its dV / dK are
-    // read out at the first tile of the next item)
-    int prev_b = 0, prev_h = 0, prev_qt = 0;
+    // previous item (its dV / dK are read out at the first tile of the next item)
     WorkRef pit{};
     bool have_item = false;
     int t = 0, ii = 0;
-    // dQ of tile x (TMEM X[x % 2], columns [32g, 32g+32) of query row `row`) into the fp32
-    // accumulator: TMEM -> registers -> this warp's staging (16 rows at a time, 128-byte
-    // swizzle) -> TMA reduce-add
-    auto drain_dq = [&](int x, int b, int h, int qt, bool release) {
-      ok = ok && mbar_wait(dq_full + (x & 1), (x >> 1) & 1, wctx);
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      if (!ok) return;
-      tc_fence_after();
-      uint32_t r[32];
-      tmem_ld32(t_lane + (x & 1) * 128 + 32 * g, r);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (release && lane == 0) mbar_arrive(x_free + (x & 1));
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        if ((lane >> 4) == half) {
-          const int rr = lane & 15;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(stg + rr * 128 + ((j ^ (rr & 7)) << 4)) =
-                make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_reduce_add_4d(&tdq, stg, 32 * g, qt * kTile + 32 * wq + 16 * half, h, b);
-          bulk_commit_group();
-          bulk_wait_read();
-        }
-        __syncwarp();
-      }
-    };
     // dV / dK of item `x` (number ix) from TMEM to global memory, bf16
     auto read_acc = [&](const WorkRef& x, int ix) {
       ok = ok && mbar_wait(acc_full, ix & 1, wctx);
@@ -1743,7 +1711,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (meta_kind[s] == 2)
           mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * g);
         const float* vs = vec + s * 256 + 64 * g;
-        const int qt_cur = p.rowT_idx[it.e0 + i];
         const uint32_t xb = t_lane + (t & 1) * 128 + 64 * g;
         const uint32_t yb = t_lane + kY + 64 * g;
         // four chunks of 16 queries; the TMEM loads of chunk c + 1 overlap the math of
@@ -1813,19 +1780,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full + (t & 1));
-        // the previous tile's dQ (its MMA completed above): drain it, freeing X[(t-1) % 2]
-        if (t >= 1) drain_dq(t - 1, prev_b, prev_h, prev_qt, true);
-        prev_b = it.b;
-        prev_h = it.h;
-        prev_qt = qt_cur;
       }
       if (!ok) break;
       pit = it;
       have_item = true;
       ++ii;
     }
-    if (ok && t >= 1) drain_dq(t - 1, prev_b, prev_h, prev_qt, false);
     if (ok && have_item) read_acc(pit, ii - 1);
+  } else {
+    // ---------------------------------------------------------------- dQ drain
+    // Warps 2, 3, 12, 13: thread = query row of the dQ tile (TMEM lane).  Per tile: wait for
+    // dQ_t, load its 64 fp32 columns, release X[t % 2] to the MMA warp, and add the tile into
+    // the fp32 accumulator with TMA bulk reduce-adds from two 2 KB staging boxes per warp
+    // (16 rows x 32 fp32, 128-byte swizzle) used alternately, so that writing one box
+    // overlaps the TMA unit reading the other.
+    const int wq = warp & 3;
+    const int di = warp < 4 ? warp - 2 : warp - 10;  // 0..3
+    uint8_t* stg = smem + L::kStg + di * 4096;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    bool ok = true;
+    int t = 0;
+    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+      const WorkRef it = iter.cur;
+      for (int i = 0; i < it.n; ++i, ++t) {
+        const int qt = p.rowT_idx[it.e0 + i];
+        if (ok) ok = mbar_wait(dq_full + (t & 1), (t >> 1) & 1, wctx);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        tmem_ld32(t_lane + (t & 1) * 128, r0);
+        tmem_ld32(t_lane + (t & 1) * 128 + 32, r1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(x_free + (t & 1));
+#pragma unroll
+        for (int part = 0; part < 4; ++part) {
+          const int half = part >> 1, cg = part & 1;  // rows 16 half.., columns 32 cg..
+          uint8_t* box = stg + (part & 1) * 2048;
+          if (lane == 0) bulk_wait_read_1();  // the box's previous reduce has read it
+          __syncwarp();
+          if ((lane >> 4) == half) {
+            const int rr = lane & 15;
+            const uint32_t* r = cg ? r1 : r0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(box + rr * 128 + ((j ^ (rr & 7)) << 4)) =
+                  make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_4d(&tdq, box, 32 * cg, qt * kTile + 32 * wq + 16 * half, it.h, it.b);
+            bulk_commit_group();
+          }
+        }
+      }
+    }
     if (lane == 0) bulk_wait_all();
   }
   // Single-lane roles (MMA issue, copy issue) end at different times than the rest of
@@ -2041,7 +2053,7 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
                                   FusedLayout::kAlloc)) != cudaSuccess)
       return cuda_status(e);
     const int items = plan->B * plan->KT * H;
-    kern<<<std::min(items, sms), kThreads, FusedLayout::kAlloc, stream>>>(tq, tk, tv, tdo, tdq, p);
+    kern<<<std::min(items, sms), kFusedThreads, FusedLayout::kAlloc, stream>>>(tq, tk, tv, tdo, tdq, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   {

@@ -149,6 +149,11 @@ __device__ __forceinline__ void bulk_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// Waits until at most one committed bulk group of this thread is still reading its source.
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 // Waits until every committed bulk group of this thread has completed.
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -410,6 +415,26 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return d;
 }
 
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// a * b clamped to [0, 1] (NaN gives 0); the packed form has no saturation, so two scalar
+// multiplies (FMA pipe)
+__device__ __forceinline__ float2 mul2_sat(float2 a, float2 b) {
+  float2 d;
+  asm("mul.rn.sat.f32 %0, %2, %4;\n\tmul.rn.sat.f32 %1, %3, %5;"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // Packs two floats into bf16x2 (round to nearest even); `lo` lands in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
@@ -446,19 +471,29 @@ __device__ __forceinline__ void sigmoid_parts2(float2 t, float2& e, float2& g) {
   g = fma2(a, e, make_float2(kSigG0, kSigG0));
 }
 
+// sigma from e and g without a compare-and-select (which would load the ALU pipe, the
+// busiest pipe of the sigmoid epilogues): with h = e g (the sigmoid of -|x|) and
+// c = saturate(t 2^126), which is 0 for t <= 0 and 1 for t > 2^-126 (where e rounds to 1),
+// sigma = h + c (g - h): h for x < 0 and g for x >= 0, on the FMA pipe only.
+__device__ __forceinline__ float2 sigmoid_select2(float2 t, float2 g, float2 h) {
+  const float2 c = mul2_sat(t, make_float2(0x1p126f, 0x1p126f));
+  return fma2(c, sub2(g, h), h);
+}
+
 // sigma(x) for two elements given t = x log2(e) (t = -inf for a masked element: 0).
 __device__ __forceinline__ float2 sigmoid2(float2 t) {
   float2 e, g;
   sigmoid_parts2(t, e, g);
-  return mul2(make_float2(t.x < 0.0f ? e.x : 1.0f, t.y < 0.0f ? e.y : 1.0f), g);
+  return sigmoid_select2(t, g, mul2(e, g));
 }
 
-// sigma(x) and sigma'(x) = sigma (1 - sigma) for two elements, t as in sigmoid2.
+// sigma(x) and sigma'(x) = sigma (1 - sigma) = e g^2 for two elements, t as in sigmoid2.
 __device__ __forceinline__ void sigmoid_grad2(float2 t, float2& p, float2& dp) {
   float2 e, g;
   sigmoid_parts2(t, e, g);
-  p = mul2(make_float2(t.x < 0.0f ? e.x : 1.0f, t.y < 0.0f ? e.y : 1.0f), g);
-  dp = mul2(mul2(e, g), g);
+  const float2 h = mul2(e, g);
+  p = sigmoid_select2(t, g, h);
+  dp = mul2(h, g);
 }
 
 }  // namespace sigattn
