@@ -340,6 +340,17 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     roofline = {"bound": "tensor", "kernel": dom, "achieved": kernels[dom]["tflops"],
                 "peak": peak_tf, "unit": "TFLOP/s", "frac": kernels[dom]["tflops"] / peak_tf,
                 "peak_source": f"{peak_src} burst bf16 (cuBLAS)", "traffic": traffic}
+    # the forward's rate against HBM: algorithmic bytes = read Q, K, V and write O once over
+    # the valid tokens (8 bytes per token, head and channel)
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fwd_bytes = 8.0 * w.valid_tokens() * w.H * w.d
+    kernels["fwd"]["bytes"] = fwd_bytes
+    kernels["fwd"]["gb_per_s"] = fwd_bytes / (kernels["fwd"]["ms"] * 1e-3) / 1e9
+    if args.config == 1 and not args.mask:
+        # a handful of tiles: no contraction to speak of, the bound is memory and latency
+        roofline = {"bound": "hbm", "kernel": "fwd", "achieved": kernels["fwd"]["gb_per_s"],
+                    "peak": hbm, "unit": "GB/s", "frac": kernels["fwd"]["gb_per_s"] / hbm,
+                    "peak_source": f"{peak_src} copy", "traffic": traffic}
 
     out = {
         "metric": "valid-token attention TFLOP/s (fwd+bwd)", "value": value, "unit": "TFLOP/s",
@@ -368,6 +379,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timing
     out["e2e"] = run_e2e(Bd, w, t, epi, dev, stream, args, world, fused)
+    packed = run_e2e_packed(Bd, w, t, epi, dev, stream, args, world, fused)
+    if packed is not None:
+        out["e2e_packed"] = packed
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         order = [(b, h) for h in range(w.H) for b in range(w.B)]
         f, s, n = oracle_sample(w, epi, t, order, args.cpu_seconds)
@@ -439,6 +453,55 @@ def run_e2e(Bd, w, t, epi, dev, stream, args, world, fused):
     value = job_throughput(world, 3.5 * fwd_flops(w), steps, ms)
     return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps}
+
+
+def run_e2e_packed(Bd, w, t, epi, dev, stream, args, world, fused):
+    """The e2e leg with PACKED host buffers (valid tokens only, sequence b at rows cu[b]..):
+    every step copies the packed Q, K, V, dO, the cumulative offsets and the per-row counts
+    in, builds the plan from the offsets, runs forward + backward on the packed layout, and
+    copies the packed O, dQ, dK, dV out.  Same valid-token FLOPs as the padded leg."""
+    if w.lengths is None:
+        return None
+    lengths = w.lengths.astype(np.int64)
+    pk = {k: torch.cat([v[b, :int(n)] for b, n in enumerate(lengths)], 0).contiguous().pin_memory()
+          for k, v in t.items()}
+    cu = torch.from_numpy(np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)).pin_memory()
+    counts = torch.from_numpy(np.repeat(lengths, lengths).astype(np.int32)).pin_memory()
+    outs = {k: torch.empty_like(pk["q"]).pin_memory() for k in ("o", "dq", "dk", "dv")}
+    h2d = sum(x.numel() * x.element_size() for x in pk.values()) + cu.numel() * 4 + counts.numel() * 4
+    d2h = sum(x.numel() * x.element_size() for x in outs.values())
+    maxlen = int(lengths.max())
+
+    def step():
+        d = {k: v.to(dev, non_blocking=True) for k, v in pk.items()}
+        plan = Bd.Plan.from_cu_seqlens(cu.to(dev, non_blocking=True), maxlen)
+        bias = Bd.bias_from_counts(counts.to(dev, non_blocking=True)) if epi == W.SIGMOID else None
+        o, lse = Bd.fwd(plan, d["q"], d["k"], d["v"], bias, epi)
+        bwd = Bd.bwd_fused if fused else Bd.bwd
+        dq, dk, dv = bwd(plan, d["q"], d["k"], d["v"], o, d["do"], bias, epi, lse=lse)
+        for name, x in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
+            outs[name].copy_(x, non_blocking=True)
+        return plan
+
+    steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        step().close()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    plans = []
+    e0.record(stream)
+    for _ in range(steps):
+        plans.append(step())
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    for p in plans:
+        p.close()
+    ms = max_over_ranks(ms, dev)
+    value = job_throughput(world, 3.5 * fwd_flops(w), steps, ms)
+    return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps,
+            "layout": "packed host buffers (valid tokens only), plan from cumulative offsets"}
 
 
 def main():

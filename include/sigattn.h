@@ -28,6 +28,10 @@
  *     that order.  Every device pointer must be 16-byte aligned and every stride
  *     a multiple of 8 elements (16 bytes).  Q/O/dO/dQ have N = Nq rows, K/V/dK/dV
  *     have N = Nk rows.  Supported head dims: d = 64 and d = 128.
+ *   - Extents are the caller's promise, as with BLAS leading dimensions: the library
+ *     sees pointers and strides only, so every tensor must hold the B x N x H x d (or
+ *     T x H x d) elements its strides address, for the plan's B and N; a smaller buffer
+ *     is read out of bounds, not reported.
  *   - bias is fp32 [B, Nq] (per query row; row stride 1, batch stride given); NULL
  *     means 0.  For sigmoid attention the caller fills -log(n), e.g. with
  *     sigattn_bias_from_counts.
@@ -71,7 +75,7 @@ enum sigattn_status {
   SIGATTN_ERR_INVALID = -1,     /* null pointer, negative size, bad enum */
   SIGATTN_ERR_UNSUPPORTED = -2, /* head dim other than 64 / 128, sizes past limits */
   SIGATTN_ERR_ALIGNMENT = -3,   /* pointer not 16-byte aligned or stride not a multiple of 8 */
-  SIGATTN_ERR_SHAPE = -4,       /* tensor shapes disagree with the plan */
+  SIGATTN_ERR_SHAPE = -4,       /* the plan belongs to another device than the current one */
   SIGATTN_ERR_CUDA = -5,        /* a CUDA runtime / driver call failed */
   SIGATTN_ERR_TIMEOUT = -6,     /* a device-side bounded wait expired (see sigattn_get_status) */
   SIGATTN_ERR_NO_DEVICE = -7,   /* no sm_100 device is current */

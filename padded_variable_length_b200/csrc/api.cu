@@ -368,7 +368,7 @@ extern "C" const char* sigattn_error_string(int code) {
     case SIGATTN_ERR_INVALID: return "invalid argument";
     case SIGATTN_ERR_UNSUPPORTED: return "unsupported head dim or size";
     case SIGATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned or stride not a multiple of 8 elements";
-    case SIGATTN_ERR_SHAPE: return "tensor shape or device disagrees with the plan";
+    case SIGATTN_ERR_SHAPE: return "the plan belongs to another device";
     case SIGATTN_ERR_CUDA: return "CUDA runtime or driver error";
     case SIGATTN_ERR_TIMEOUT: return "a device-side bounded wait expired";
     case SIGATTN_ERR_NO_DEVICE: return "no CUDA device is current";
