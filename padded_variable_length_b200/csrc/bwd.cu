@@ -46,6 +46,9 @@ struct BwdParams {
   const int4* col_desc;
   const int32_t* cu;  // packed batches: cumulative row offsets [B + 1]; nullptr when padded
   int B, QT, KT, Nq, Nk, H;
+  // items with tiles: the first nwork_cols (k-tile column, head) items of the column list
+  // and the first nwork_rows (q-tile row, head) items of the row list; the rest are empty
+  int nwork_cols, nwork_rows;
   float scale;
   const float* bias;
   int64_t bias_sb;
@@ -81,35 +84,90 @@ __device__ __forceinline__ float row_D(const BwdParams& p, int b, int h, int qg)
   return p.Dws[(static_cast<int64_t>(b) * p.H + h) * p.Nq + qg];
 }
 
-// p and ds of two neighbouring elements (packed fp32 pairs); k0 / k1 are the mask bits.
+// p and ds of two neighbouring elements (packed fp32 pairs); k0 / k1 are the mask bits,
+// looked at only when kMask.
 // SIGMOID: p = sigma(x), ds = dp sigma'(x) with sigma' = sigma (1 - sigma) from the same
 //   exp2 (sigmoid_grad2); a masked element takes t = -inf, which gives p = ds = 0.
 // softmax: p = 2^t, ds = p (dp - D); a masked element takes p = 0.
-template <int EPI>
+template <int EPI, bool kMask>
 __device__ __forceinline__ void weight_grad2(float2 s, float2 dp, float2 c1, float2 off, float2 Dv,
                                              bool k0, bool k1, float2& pw, float2& ds) {
   float2 x = fma2(s, c1, off);
   if (EPI == 0) {
-    x.x = k0 ? x.x : -INFINITY;
-    x.y = k1 ? x.y : -INFINITY;
+    if (kMask) {
+      x.x = k0 ? x.x : -INFINITY;
+      x.y = k1 ? x.y : -INFINITY;
+    }
     float2 w;
     sigmoid_grad2(x, pw, w);
     ds = mul2(w, dp);
   } else {
-    pw = make_float2(k0 ? ex2_approx(x.x) : 0.0f, k1 ? ex2_approx(x.y) : 0.0f);
+    pw = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    if (kMask) pw = make_float2(k0 ? pw.x : 0.0f, k1 ? pw.y : 0.0f);
     ds = mul2(pw, fma2(Dv, make_float2(-1.0f, -1.0f), dp));
   }
 }
 
-template <int D>
-__device__ __forceinline__ void zero_rows(__nv_bfloat16* base, int64_t sn, int rows, int tid,
-                                          int nthreads) {
-  constexpr int kChunks = D / 8;
-  for (int i = tid; i < rows * kChunks; i += nthreads) {
-    const int row = i / kChunks, c = i % kChunks;
-    *reinterpret_cast<uint4*>(base + static_cast<int64_t>(row) * sn + c * 8) =
-        make_uint4(0u, 0u, 0u, 0u);
+// Does a chunk of a row's elements need the per-element mask?  Decided for the whole warp:
+// not on FULL tiles, and not where every lane keeps every element of the chunk (`all` has
+// the chunk's bits set) -- a PARTIAL tile of a padded batch is mostly whole chunks of kept
+// or dropped keys, so only those with a dropped element pay for the mask.
+__device__ __forceinline__ bool chunk_masked(bool masked_tile, uint32_t mw, uint32_t all) {
+  return masked_tile && !__all_sync(0xFFFFFFFFu, (mw & all) == all);
+}
+
+// Clears the bf16 halves of packed pairs whose keep bit is 0 (bit 2e: low half of w[e],
+// bit 2e + 1: high half).  Zeroing the packed result equals the element's P = dS = 0 in
+// every mode, whatever was computed for it.
+template <int N>
+__device__ __forceinline__ void mask_pairs(uint32_t* w, uint32_t mw) {
+#pragma unroll
+  for (int e = 0; e < N / 2; ++e) {
+    const uint32_t lo = 0u - ((mw >> (2 * e)) & 1u), hi = 0u - ((mw >> (2 * e + 1)) & 1u);
+    w[e] &= (lo & 0x0000FFFFu) | (hi & 0xFFFF0000u);
   }
+}
+
+// P and dS of N consecutive elements of one row as packed bf16 pairs: s, dp the raw fp32
+// words of S and dP, vs the elements' row offsets (and, softmax, D at vs + 128) in shared
+// memory, mw their keep bits (bit j = element j), applied when `mask` (chunk_masked).
+template <int EPI, int N>
+__device__ __forceinline__ void grad_chunk(const uint32_t* s, const uint32_t* dp, float2 c1,
+                                           const float* vs, uint32_t mw, bool mask, uint32_t* pk,
+                                           uint32_t* dk) {
+#pragma unroll
+  for (int cc = 0; cc < N; cc += 2) {
+    float2 pw, ds;
+    const float2 off2 = *reinterpret_cast<const float2*>(vs + cc);
+    const float2 D2 =
+        EPI == 0 ? make_float2(0.0f, 0.0f) : *reinterpret_cast<const float2*>(vs + 128 + cc);
+    weight_grad2<EPI, false>(make_float2(__uint_as_float(s[cc]), __uint_as_float(s[cc + 1])),
+                             make_float2(__uint_as_float(dp[cc]), __uint_as_float(dp[cc + 1])),
+                             c1, off2, D2, true, true, pw, ds);
+    pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
+    dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+  }
+  if (mask) {
+    mask_pairs<N>(pk, mw);
+    mask_pairs<N>(dk, mw);
+  }
+}
+
+// dS alone of N consecutive elements of one query row (the row's offset off2 and D2 shared
+// by all of them), as for grad_chunk.
+template <int EPI, int N>
+__device__ __forceinline__ void ds_chunk(const uint32_t* s, const uint32_t* dp, float2 c1,
+                                         float2 off2, float2 D2, uint32_t mw, bool mask,
+                                         uint32_t* dk) {
+#pragma unroll
+  for (int cc = 0; cc < N; cc += 2) {
+    float2 pw, ds;
+    weight_grad2<EPI, false>(make_float2(__uint_as_float(s[cc]), __uint_as_float(s[cc + 1])),
+                             make_float2(__uint_as_float(dp[cc]), __uint_as_float(dp[cc + 1])),
+                             c1, off2, D2, true, true, pw, ds);
+    dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+  }
+  if (mask) mask_pairs<N>(dk, mw);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -191,6 +249,31 @@ __device__ __forceinline__ WorkRef decode_row(const BwdParams& p, int w) {
   return r;
 }
 
+// Zero gradient rows for the items without tiles, [nwork, nitems) of a longest-first list
+// (k-tiles that no query attends to, for dK / dV; q-tiles past their sequence's length or
+// seeing no key, for dQ).  The items are dealt round-robin to every epilogue warp of the
+// grid, one item per warp at a time, with no dependent loads between them; run before the
+// first tile, while the epilogue would otherwise wait for its first S.  x1 may be null.
+template <int D, bool kCols>
+__device__ void zero_empty_items(const BwdParams& p, int nwork, int nitems, int ew, int lane,
+                                 __nv_bfloat16* x0, int64_t sb0, int64_t sn0, int64_t sh0,
+                                 __nv_bfloat16* x1, int64_t sb1, int64_t sn1, int64_t sh1) {
+  constexpr int kChunks = D / 8;
+  const int stride = static_cast<int>(gridDim.x) * 8;
+  for (int w = nwork + static_cast<int>(blockIdx.x) * 8 + ew; w < nitems; w += stride) {
+    const WorkRef x = kCols ? decode_col(p, w) : decode_row(p, w);
+    const int rows = min(kTile, x.sq.limit - x.t * kTile);
+    for (int c = lane; c < rows * kChunks; c += 32) {
+      const int r = x.t * kTile + c / kChunks, ch = (c % kChunks) * 8;
+      *reinterpret_cast<uint4*>(x0 + seq_row_offset(x.sq, sb0, sn0, r) + x.h * sh0 + ch) =
+          make_uint4(0u, 0u, 0u, 0u);
+      if (x1 != nullptr)
+        *reinterpret_cast<uint4*>(x1 + seq_row_offset(x.sq, sb1, sn1, r) + x.h * sh1 + ch) =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
 // Walks this CTA's work items (snake order, see snake_item) with the next item's decode
 // issued one item ahead, so that its global loads overlap the current item.
 template <bool kCols>
@@ -264,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
-  const int nitems = p.B * p.KT * p.H;
+  const int nitems = p.B * p.KT * p.H, nwork = p.nwork_cols;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* kv_full = bars;
@@ -321,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // queries) one tile ahead, so no global load sits between two copies.
     int qc = 0, ii = 0;
     bool ok = true;
-    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+    for (WorkIter<true> iter(p, nwork); ok && iter.valid(); iter.advance()) {
       const WorkRef it = iter.cur;
       if (it.n == 0) continue;
       const int kb = ii % KVB;
@@ -448,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     int qc = 0, ii = 0, u = 0;
     uint32_t b3 = 0;  // u % 3
-    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+    for (WorkIter<true> iter(p, nwork); ok && iter.valid(); iter.advance()) {
       const WorkRef it = iter.cur;
       if (it.n == 0) continue;
       const int kb = ii & 1;
@@ -538,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit_w(s_full + h);
       };
       int qc = 0, ii = 0;
-      for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+      for (WorkIter<true> iter(p, nwork); ok && iter.valid(); iter.advance()) {
         const WorkRef it = iter.cur;
         if (it.n == 0) continue;
         const int kb = ii % KVB, ab = ii % ACB;
@@ -623,19 +706,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     int qc = 0, ii = 0;
-    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+    zero_empty_items<D, true>(p, nwork, nitems, warp - kEpiWarp0, lane, p.dk, p.dk_sb, p.dk_sn, p.dk_sh,
+                              p.dv, p.dv_sb, p.dv_sn, p.dv_sh);
+    for (WorkIter<true> iter(p, nwork); ok && iter.valid(); iter.advance()) {
       const WorkRef it = iter.cur;
-      if (it.n == 0) {
-        // No query attends to this k-tile: dK = dV = 0 on its rows.
-        if (pend) flush();
-        const int rows = min(kTile, it.sq.limit - it.t * kTile);
-        const int tid = threadIdx.x - kEpiWarp0 * 32;
-        zero_rows<D>(p.dk + seq_row_offset(it.sq, p.dk_sb, p.dk_sn, it.t * kTile) +
-                         it.h * p.dk_sh, p.dk_sn, rows, tid, 256);
-        zero_rows<D>(p.dv + seq_row_offset(it.sq, p.dv_sb, p.dv_sn, it.t * kTile) +
-                         it.h * p.dv_sh, p.dv_sn, rows, tid, 256);
-        continue;
-      }
+      if (it.n == 0) continue;  // not in [0, nwork)
       for (int i = 0; i < it.n; ++i, ++qc) {
         const int s = qc & 3, u = 2 * qc + h;
         // q_full of the stage also publishes the kind, bitmask and column vectors
@@ -645,7 +720,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        if (meta_kind[s] == 2)
+        const bool masked = meta_kind[s] == 2;
+        if (masked)
           mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
         const float* vs = vec + s * 256 + 64 * h;
         const uint32_t base = t_lane + (u % 3) * 128;
@@ -660,19 +736,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c == 1) tmem_wait_ld();
           const uint32_t mw = c ? mb.y : mb.x;
           uint32_t pk[16], dk[16];
-#pragma unroll
-          for (int cc = 0; cc < 32; cc += 2) {
-            float2 pw, ds;
-            const float2 off2 = *reinterpret_cast<const float2*>(vs + 32 * c + cc);
-            const float2 D2 = EPI == 0 ? make_float2(0.0f, 0.0f)
-                                       : *reinterpret_cast<const float2*>(vs + 128 + 32 * c + cc);
-            weight_grad2<EPI>(
-                make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
-                make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])), c1, off2,
-                D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
-            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
-            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
-          }
+          grad_chunk<EPI, 32>(sr[c], dpr[c], c1, vs + 32 * c, mw, chunk_masked(masked, mw, 0xFFFFFFFFu),
+                              pk, dk);
           tmem_st16(base + 16 * c, pk);
           tmem_st16(base + 64 + 16 * c, dk);
         }
@@ -699,18 +764,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float2 c1 = make_float2(c1s, c1s);
     bool ok = true;
     int qc = 0, ii = 0;
-    for (WorkIter<true> iter(p, nitems); iter.valid(); iter.advance()) {
+    zero_empty_items<D, true>(p, nwork, nitems, warp - kEpiWarp0, lane, p.dk, p.dk_sb, p.dk_sn, p.dk_sh,
+                              p.dv, p.dv_sb, p.dv_sn, p.dv_sh);
+    for (WorkIter<true> iter(p, nwork); iter.valid(); iter.advance()) {
       const WorkRef it = iter.cur;
-      if (it.n == 0) {
-        // No query attends to this k-tile: dK = dV = 0 on its rows.
-        const int rows = min(kTile, it.sq.limit - it.t * kTile);
-        const int tid = threadIdx.x - kEpiWarp0 * 32;
-        zero_rows<D>(p.dk + seq_row_offset(it.sq, p.dk_sb, p.dk_sn, it.t * kTile) +
-                         it.h * p.dk_sh, p.dk_sn, rows, tid, 256);
-        zero_rows<D>(p.dv + seq_row_offset(it.sq, p.dv_sb, p.dv_sn, it.t * kTile) +
-                         it.h * p.dv_sh, p.dv_sn, rows, tid, 256);
-        continue;
-      }
+      if (it.n == 0) continue;  // not in [0, nwork)
       if (!ok) break;
       const int ab = ii % ACB;
       for (int i = 0; i < it.n; ++i, ++qc) {
@@ -722,7 +780,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        if (meta_kind[s] == 2)
+        const bool masked = meta_kind[s] == 2;
+        if (masked)
           mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
         const float* vs = vec + s * 256 + 64 * h;
         uint32_t sr[2][32], dpr[2][32];
@@ -736,18 +795,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c == 1) tmem_wait_ld();
           const uint32_t mw = c ? mb.y : mb.x;
           uint32_t pk[16], dk[16];
-#pragma unroll
-          for (int cc = 0; cc < 32; cc += 2) {
-            float2 pw, ds;
-            const float2 off2 = *reinterpret_cast<const float2*>(vs + 32 * c + cc);
-            const float2 D2 = EPI == 0 ? make_float2(0.0f, 0.0f)
-                                       : *reinterpret_cast<const float2*>(vs + 128 + 32 * c + cc);
-            weight_grad2<EPI>(make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
-                              make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])),
-                              c1, off2, D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
-            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
-            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
-          }
+          grad_chunk<EPI, 32>(sr[c], dpr[c], c1, vs + 32 * c, mw, chunk_masked(masked, mw, 0xFFFFFFFFu),
+                              pk, dk);
           tmem_st16(t_lane + 64 * h + 16 * c, pk);
           tmem_st16(t_lane + 128 + 64 * h + 16 * c, dk);
         }
@@ -852,7 +901,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
-  const int nitems = p.B * p.QT * p.H;
+  const int nitems = p.B * p.QT * p.H, nwork = p.nwork_rows;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* qd_full = bars;
@@ -907,7 +956,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // 32 k-tiles in one round trip.
     int tk_ = 0, ii = 0;
     bool ok = true;
-    for (WorkIter<false> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+    for (WorkIter<false> iter(p, nwork); ok && iter.valid(); iter.advance()) {
       const WorkRef it = iter.cur;
       if (it.n == 0) continue;
       const int qb = ii % QB;
@@ -1006,7 +1055,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     int tc = 0, ii = 0, u = 0;
     uint32_t b3 = 0;  // u % 3
-    for (WorkIter<false> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+    for (WorkIter<false> iter(p, nwork); ok && iter.valid(); iter.advance()) {
       const WorkRef it = iter.cur;
       if (it.n == 0) continue;
       const int qb = ii & 1;
@@ -1087,7 +1136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit_w(s_full + h);
       };
       int tk_ = 0, ii = 0;
-      for (WorkIter<false> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+      for (WorkIter<false> iter(p, nwork); ok && iter.valid(); iter.advance()) {
         const WorkRef it = iter.cur;
         if (it.n == 0) continue;
         const int qb = ii % QB, ab = ii % ACB;
@@ -1164,7 +1213,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     int tc = 0, ii = 0;
-    WorkIter<false> iter(p, nitems);
+    zero_empty_items<D, false>(p, nwork, nitems, warp - kEpiWarp0, lane, p.dq, p.dq_sb, p.dq_sn, p.dq_sh,
+                               nullptr, 0, 0, 0);
+    WorkIter<false> iter(p, nwork);
     float off_cur = 0.0f, D_cur = 0.0f;
     if (iter.valid()) {
       off_cur = row_offset<EPI>(p, iter.cur.sq, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
@@ -1174,20 +1225,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WorkRef it = iter.cur;
       // the next item's row values, in flight while this one is processed
       float off_nxt = 0.0f, D_nxt = 0.0f;
-      if (iter.wn < nitems && iter.nxt.n > 0) {
+      if (iter.wn < nwork && iter.nxt.n > 0) {
         off_nxt = row_offset<EPI>(p, iter.nxt.sq, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
         D_nxt = row_D<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
       }
       const float off = off_cur, Drow = D_cur;
       off_cur = off_nxt;
       D_cur = D_nxt;
-      if (it.n == 0) {
-        if (pend) flush();
-        const int rows = min(kTile, it.sq.limit - it.t * kTile);
-        zero_rows<D>(p.dq + seq_row_offset(it.sq, p.dq_sb, p.dq_sn, it.t * kTile) +
-                         it.h * p.dq_sh, p.dq_sn, rows, threadIdx.x - kEpiWarp0 * 32, 256);
-        continue;
-      }
+      if (it.n == 0) continue;  // not in [0, nwork)
       const float2 off2 = make_float2(off, off), D2 = make_float2(Drow, Drow);
       for (int j = 0; j < it.n; ++j, ++tc) {
         const int s = tc & 3, u = 2 * tc + h;
@@ -1198,7 +1243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        if (meta_kind[s] == 2)
+        const bool masked = meta_kind[s] == 2;
+        if (masked)
           mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
         const uint32_t base = t_lane + (u % 3) * 128;
         uint32_t sr[2][32], dpr[2][32];
@@ -1212,15 +1258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c == 1) tmem_wait_ld();
           const uint32_t mw = c ? mb.y : mb.x;
           uint32_t dk[16];
-#pragma unroll
-          for (int cc = 0; cc < 32; cc += 2) {
-            float2 pw, ds;
-            weight_grad2<EPI>(
-                make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
-                make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])), c1, off2,
-                D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
-            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
-          }
+          ds_chunk<EPI, 32>(sr[c], dpr[c], c1, off2, D2, mw, chunk_masked(masked, mw, 0xFFFFFFFFu), dk);
           tmem_st16(base + 64 + 16 * c, dk);
         }
         tmem_wait_st();
@@ -1246,7 +1284,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float2 c1 = make_float2(c1s, c1s);
     bool ok = true;
     int tk_ = 0, ii = 0;
-    WorkIter<false> iter(p, nitems);
+    zero_empty_items<D, false>(p, nwork, nitems, warp - kEpiWarp0, lane, p.dq, p.dq_sb, p.dq_sn, p.dq_sh,
+                               nullptr, 0, 0, 0);
+    WorkIter<false> iter(p, nwork);
     float off_cur = 0.0f, D_cur = 0.0f;
     if (iter.valid()) {
       off_cur = row_offset<EPI>(p, iter.cur.sq, iter.cur.b, iter.cur.h, iter.cur.t * kTile + row);
@@ -1256,19 +1296,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WorkRef it = iter.cur;
       // the next item's row values, in flight while this one is processed
       float off_nxt = 0.0f, D_nxt = 0.0f;
-      if (iter.wn < nitems && iter.nxt.n > 0) {
+      if (iter.wn < nwork && iter.nxt.n > 0) {
         off_nxt = row_offset<EPI>(p, iter.nxt.sq, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
         D_nxt = row_D<EPI>(p, iter.nxt.b, iter.nxt.h, iter.nxt.t * kTile + row);
       }
       const float off = off_cur, Drow = D_cur;
       off_cur = off_nxt;
       D_cur = D_nxt;
-      if (it.n == 0) {
-        const int rows = min(kTile, it.sq.limit - it.t * kTile);
-        zero_rows<D>(p.dq + seq_row_offset(it.sq, p.dq_sb, p.dq_sn, it.t * kTile) +
-                         it.h * p.dq_sh, p.dq_sn, rows, threadIdx.x - kEpiWarp0 * 32, 256);
-        continue;
-      }
+      if (it.n == 0) continue;  // not in [0, nwork)
       if (!ok) break;
       const int ab = ii % ACB;
       const int qg = it.t * kTile + row;
@@ -1282,7 +1317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        if (meta_kind[s] == 2)
+        const bool masked = meta_kind[s] == 2;
+        if (masked)
           mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
         uint32_t sr[2][32], dpr[2][32];
         tmem_ld32(t_lane + 64 * h, sr[0]);
@@ -1295,14 +1331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c == 1) tmem_wait_ld();
           const uint32_t mw = c ? mb.y : mb.x;
           uint32_t dk[16];
-#pragma unroll
-          for (int cc = 0; cc < 32; cc += 2) {
-            float2 pw, ds;
-            weight_grad2<EPI>(make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
-                              make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])),
-                              c1, off2, D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
-            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
-          }
+          ds_chunk<EPI, 32>(sr[c], dpr[c], c1, off2, D2, mw, chunk_masked(masked, mw, 0xFFFFFFFFu), dk);
           tmem_st16(t_lane + 128 + 64 * h + 16 * c, dk);
         }
         tmem_wait_st();
@@ -1416,7 +1445,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
-  const int nitems = p.B * p.KT * p.H;
+  const int nitems = p.B * p.KT * p.H, nwork = p.nwork_cols;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* kv_full = bars;
@@ -1480,7 +1509,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     }
     int qc = 0, ii = 0;
     bool ok = true;
-    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+    for (WorkIter<true> iter(p, nwork); ok && iter.valid(); iter.advance()) {
       const WorkRef it = iter.cur;
       if (it.n == 0) continue;
       const int kb = ii & 1;
@@ -1605,7 +1634,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       return true;
     };
     int t = 0, ii = 0;
-    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+    for (WorkIter<true> iter(p, nwork); ok && iter.valid(); iter.advance()) {
       const WorkRef it = iter.cur;
       if (it.n == 0) continue;
       const int kb = ii & 1;
@@ -1687,18 +1716,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         }
       }
     };
-    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+    zero_empty_items<D, true>(p, nwork, nitems, warp - kEpiWarp0, lane, p.dk, p.dk_sb, p.dk_sn, p.dk_sh,
+                              p.dv, p.dv_sb, p.dv_sn, p.dv_sh);
+    for (WorkIter<true> iter(p, nwork); ok && iter.valid(); iter.advance()) {
       const WorkRef it = iter.cur;
-      if (it.n == 0) {
-        // No query attends to this k-tile: dK = dV = 0 on its rows.
-        const int rows = min(kTile, it.sq.limit - it.t * kTile);
-        const int tid = threadIdx.x - kEpiWarp0 * 32;
-        zero_rows<D>(p.dk + seq_row_offset(it.sq, p.dk_sb, p.dk_sn, it.t * kTile) +
-                         it.h * p.dk_sh, p.dk_sn, rows, tid, 256);
-        zero_rows<D>(p.dv + seq_row_offset(it.sq, p.dv_sb, p.dv_sn, it.t * kTile) +
-                         it.h * p.dv_sh, p.dv_sn, rows, tid, 256);
-        continue;
-      }
+      if (it.n == 0) continue;  // not in [0, nwork)
       for (int i = 0; i < it.n; ++i, ++t) {
         const int s = t % S;
         // q_full of the stage also publishes the kind, bitmask and column vectors
@@ -1708,7 +1730,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         if (!ok) break;
         tc_fence_after();
         uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        if (meta_kind[s] == 2)
+        const bool masked = meta_kind[s] == 2;
+        if (masked)
           mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * g);
         const float* vs = vec + s * 256 + 64 * g;
         const uint32_t xb = t_lane + (t & 1) * 128 + 64 * g;
@@ -1728,19 +1751,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           }
           const uint32_t mw = (c < 2 ? mb.x : mb.y) >> (16 * (c & 1));
           uint32_t pk[8], dk[8];
-#pragma unroll
-          for (int cc = 0; cc < 16; cc += 2) {
-            float2 pw, ds;
-            const float2 off2 = *reinterpret_cast<const float2*>(vs + 16 * c + cc);
-            const float2 D2 = EPI == 0 ? make_float2(0.0f, 0.0f)
-                                       : *reinterpret_cast<const float2*>(vs + 128 + 16 * c + cc);
-            weight_grad2<EPI>(
-                make_float2(__uint_as_float(sr[c & 1][cc]), __uint_as_float(sr[c & 1][cc + 1])),
-                make_float2(__uint_as_float(dpr[c & 1][cc]), __uint_as_float(dpr[c & 1][cc + 1])),
-                c1, off2, D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
-            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
-            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
-          }
+          grad_chunk<EPI, 16>(sr[c & 1], dpr[c & 1], c1, vs + 16 * c, mw,
+                              chunk_masked(masked, mw, 0xFFFFu), pk, dk);
           tmem_st8(xb + 16 * c, pk);
           tmem_st8(xb + 16 * c + 8, dk);
           if (c < 3) tmem_wait_ld();
@@ -1800,7 +1812,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     bool ok = true;
     int t = 0;
-    for (WorkIter<true> iter(p, nitems); ok && iter.valid(); iter.advance()) {
+    for (WorkIter<true> iter(p, nwork); ok && iter.valid(); iter.advance()) {
       const WorkRef it = iter.cur;
       for (int i = 0; i < it.n; ++i, ++t) {
         const int qt = p.rowT_idx[it.e0 + i];
@@ -1936,6 +1948,8 @@ int launch_bwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.B = plan->B;
   p.QT = plan->QT;
   p.KT = plan->KT;
+  p.nwork_cols = plan->cols_nonempty * H;
+  p.nwork_rows = plan->rows_nonempty * H;
   p.Nq = plan->Nq;
   p.Nk = plan->Nk;
   p.H = H;
@@ -2010,6 +2024,8 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
   p.B = plan->B;
   p.QT = plan->QT;
   p.KT = plan->KT;
+  p.nwork_cols = plan->cols_nonempty * H;
+  p.nwork_rows = plan->rows_nonempty * H;
   p.Nq = plan->Nq;
   p.Nk = plan->Nk;
   p.H = H;

@@ -54,7 +54,9 @@ struct FwdParams {
   const int32_t* cu;  // packed batches: cumulative row offsets [B + 1]; nullptr when padded
   const int4* run;  // runs of consecutive k-tiles of one kind (see sigattn_plan)
   int run_cap;      // entries allocated in run (reads stay below it)
-  int QT, Nq, H, nitems;
+  int QT, Nq, H;
+  int nitems;  // B QT H items: (q-tile row, head), in the order of the longest-first list
+  int nwork;   // the first nwork items have tiles; the rest are empty
   float scale;
   const float* bias;
   int64_t bias_sb;
@@ -106,26 +108,50 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p, int w) {
   return it;
 }
 
-// Walks this CTA's work items (snake order, see snake_item) with the next item's decode
-// issued one item ahead, so that its global loads overlap the current item.
+// Walks this CTA's items with tiles (snake order over [0, nwork), see snake_item) with the
+// next item's decode issued one item ahead, so that its global loads overlap the current
+// item.
 struct ItemIter {
   const FwdParams& p;
   int k, w, wn;  // round, this item, next item
   Item cur, nxt;
   __device__ explicit ItemIter(const FwdParams& pp)
       : p(pp), k(0), w(snake_item(0)), wn(snake_item(1)) {
-    if (w < p.nitems) cur = decode_item(p, w);
-    if (wn < p.nitems) nxt = decode_item(p, wn);
+    if (w < p.nwork) cur = decode_item(p, w);
+    if (wn < p.nwork) nxt = decode_item(p, wn);
   }
-  __device__ bool valid() const { return w < p.nitems; }
+  __device__ bool valid() const { return w < p.nwork; }
   __device__ void advance() {
     ++k;
     w = wn;
     wn = snake_item(k + 1);
     cur = nxt;
-    if (wn < p.nitems) nxt = decode_item(p, wn);
+    if (wn < p.nwork) nxt = decode_item(p, wn);
   }
 };
+
+// O = 0 on the rows of the items without tiles, [nwork, nitems) of the longest-first list:
+// q-tiles past their sequence's length, or whose rows see no key (and, for the softmax
+// modes, LSE = -inf resp. 0 there).  The items are dealt round-robin to every epilogue warp
+// of the grid, one item per warp at a time, with no dependent loads between them; run
+// before the first tile, while the epilogue would otherwise wait for its first S.
+template <int D, int EPI>
+__device__ void zero_empty_items(const FwdParams& p, int ew, int lane) {
+  constexpr int kChunks = D / 8;
+  const int stride = static_cast<int>(gridDim.x) * 8;
+  for (int w = p.nwork + static_cast<int>(blockIdx.x) * 8 + ew; w < p.nitems; w += stride) {
+    const Item x = decode_item(p, w);
+    const int rows = min(kTile, x.sq.limit - x.qt * kTile);
+    for (int c = lane; c < rows * kChunks; c += 32)
+      *reinterpret_cast<uint4*>(p.o + seq_row_offset(x.sq, p.o_sb, p.o_sn, x.qt * kTile + c / kChunks) +
+                                x.h * p.o_sh + (c % kChunks) * 8) = make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (EPI != 0) {
+      for (int c = lane; c < min(kTile, p.Nq - x.qt * kTile); c += 32)
+        p.lse[(static_cast<int64_t>(x.b) * p.H + x.h) * p.Nq + x.qt * kTile + c] =
+            EPI == 1 ? -INFINITY : 0.0f;
+    }
+  }
+}
 
 template <int D, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -346,28 +372,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                  ? p.bias[static_cast<int64_t>(x.sq.tma_b) * p.bias_sb + x.sq.row0 + r]
                  : 0.0f;
     };
+    zero_empty_items<D, EPI>(p, warp - kEpiWarp0, lane);
     ItemIter iter(p);
     float bias_cur = iter.valid() ? row_bias(iter.cur) : 0.0f;
     for (; iter.valid(); iter.advance()) {
       const Item it = iter.cur;
       const float bias_nxt =
-          iter.wn < p.nitems ? row_bias(iter.nxt) : 0.0f;
+          iter.wn < p.nwork ? row_bias(iter.nxt) : 0.0f;
       const float bias_r = bias_cur;
       bias_cur = bias_nxt;
-      if (it.n == 0) {
-        const int rows = min(kTile, it.sq.limit - it.qt * kTile);
-        constexpr int kChunks = D / 8;
-        const int tid = threadIdx.x - kEpiWarp0 * 32;
-        for (int c = tid; c < rows * kChunks; c += 256) {
-          const int rr = c / kChunks, ch = c % kChunks;
-          *reinterpret_cast<uint4*>(p.o + seq_row_offset(it.sq, p.o_sb, p.o_sn, it.qt * kTile + rr) +
-                                    it.h * p.o_sh + ch * 8) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        for (int c = tid; c < min(kTile, p.Nq - it.qt * kTile); c += 256)
-          p.lse[(static_cast<int64_t>(it.b) * p.H + it.h) * p.Nq + it.qt * kTile + c] =
-              EPI == 1 ? -INFINITY : 0.0f;
-        continue;
-      }
+      if (it.n == 0) continue;  // not in [0, nwork)
       const int ob = i & 1;
       const int rg = it.qt * kTile + row;
       const float c1 = p.scale * kLog2e;  // t = (scale s + bias) log2 e
@@ -742,27 +756,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       static_assert((SK & (SK - 1)) == 0 && (SV & (SV - 1)) == 0 && NS == 4, "ring sizes");
       // O += P_x V_x for the oldest tile x of the FIFO (buffer b3 = x % 3), once the
       // epilogue has finished it; commits step(x)
-      auto pv = [&](int x, uint32_t b3) -> bool {
+      // `ready`: its P and V are known to be in place (tested together with the next K)
+      auto pv = [&](int x, uint32_t b3, bool ready) -> bool {
         const int i = pq0 >> 2;
         const bool first = (pq0 & 2) != 0, last = (pq0 & 1) != 0;
         pq0 = pq1;
         pq1 = pq2;
         const int sv = x & (SV - 1);
-        if (!mbar_wait_w(e_done + (x & 3), (x >> 2) & 1, wctx)) return false;
-        if (!mbar_wait_w(v_full + sv, (x / SV) & 1, wctx)) return false;
+        if (!ready) {
+          if (!mbar_wait_w(e_done + (x & 3), (x >> 2) & 1, wctx)) return false;
+          if (!mbar_wait_w(v_full + sv, (x / SV) & 1, wctx)) return false;
+        }
         const int ob = OB == 1 ? 0 : (i & 1);
         if (first && i >= OB && !mbar_wait_w(o_empty + ob, ((i / OB) - 1) & 1, wctx))
           return false;
         tc_fence_after();
-        const uint32_t v_lo = v_lo0 + sv * kTileLo;
-        const uint32_t o_tmem = tmem + L::kOCol + ob * D;
-        const uint32_t p_tmem = tmem + b3 * 128;
-        mma_ts_lh_w(o_tmem, p_tmem, v_lo, kHiMn, idesc_pv, first ? 0u : 1u);
-#pragma unroll
-        for (int kk = 1; kk < 8; ++kk)
-          mma_ts_lh_w(o_tmem, p_tmem + (kk >> 2) * 64 + (kk & 3) * 8, v_lo + kk * 128, kHiMn,
-                    idesc_pv, 1u);
-        mma_commit_w(step + (x & 3));
+        mma_pv8_commit_w(tmem + L::kOCol + ob * D, tmem + b3 * 128, v_lo0 + sv * kTileLo, kHiMn,
+                         idesc_pv, first ? 0u : 1u, step + (x & 3));
         if (last) mma_commit_w(o_full + ob);
         return true;
       };
@@ -775,19 +785,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait_w(q_full + qb, (i >> 1) & 1, wctx))) break;
         const uint32_t q_lo = q_lo0 + qb * kTileLo;
         for (int j = 0; j < it.n; ++j, ++t) {
-          // S_t goes to the buffer of tile t - 3: its PV first (the pipe runs in order)
-          if (t >= 3 && !(ok = pv(t - 3, b3))) break;
           const int s = t & (SK - 1);
-          if (!(ok = mbar_wait_w(k_full + s, (t / SK) & 1, wctx))) break;
+          // The usual case: P and V of tile t - 3 and K of tile t are all in place.  One
+          // non-blocking test of the three barriers; the bounded waits only when it fails.
+          bool ready = mbar_test_wait(k_full + s, (t / SK) & 1);
+          if (t >= 3)
+            ready = ready & mbar_test_wait(e_done + ((t - 3) & 3), ((t - 3) >> 2) & 1) &
+                    mbar_test_wait(v_full + ((t - 3) & (SV - 1)), ((t - 3) / SV) & 1);
+          ready = __all_sync(0xFFFFFFFFu, ready);
+          // S_t goes to the buffer of tile t - 3: its PV first (the pipe runs in order)
+          if (t >= 3 && !(ok = pv(t - 3, b3, ready))) break;
+          if (!ready && !(ok = mbar_wait_w(k_full + s, (t / SK) & 1, wctx))) break;
           tc_fence_after();
-          const uint32_t k_lo = k_lo0 + s * kTileLo;
-          const uint32_t d_tmem = tmem + b3 * 128;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (L::kBoxBytes >> 4) + (kk & 3) * 2;
-            mma_ss_lh_w(d_tmem, q_lo + off, k_lo + off, kHiKm, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          mma_commit_w(s_ready + (t & 3));
+          static_assert(L::kBoxBytes >> 4 == 1024, "box offset in the S issue");
+          mma_s_commit_w<D / 16>(tmem + b3 * 128, q_lo, k_lo0 + s * kTileLo, kHiKm, idesc_qk,
+                                 s_ready + (t & 3));
           if (j == it.n - 1) mma_commit_w(q_empty + qb);
           const int info = (i << 2) | (j == 0 ? 2 : 0) | (j == it.n - 1 ? 1 : 0);
           if (t == 0) pq0 = info;
@@ -800,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the last PVs: tile x uses buffer x % 3; b3 is t % 3 here
       for (int x = max(0, t - 3); ok && x < t; ++x) {
         const uint32_t bx = static_cast<uint32_t>((x - t + 3) % 3 + static_cast<int>(b3)) % 3;
-        ok = pv(x, bx);
+        ok = pv(x, bx, false);
       }
       // every MMA complete before the TMEM is released
       mma_commit_w(done);
@@ -861,6 +873,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
     };
+    zero_empty_items<D, 0>(p, warp - kEpiWarp0, lane);
     int t = 0, i = 0;
     ItemIter iter(p);
     float bias_cur = iter.valid() ? row_bias(iter.cur) : 0.0f;
@@ -868,22 +881,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = iter.cur;
       // the next item's bias, in flight while this one is processed
       const float bias_nxt =
-          iter.wn < p.nitems ? row_bias(iter.nxt) : 0.0f;
+          iter.wn < p.nwork ? row_bias(iter.nxt) : 0.0f;
       const float bias_r = bias_cur;
       bias_cur = bias_nxt;
-      if (it.n == 0) {
-        // No tile in this row: the whole q-tile is padding or sees no key.  O = 0.
-        if (pend) flush_o();
-        const int rows = min(kTile, it.sq.limit - it.qt * kTile);
-        constexpr int kChunks = D / 8;
-        const int tid = threadIdx.x - kEpiWarp0 * 32;
-        for (int c = tid; c < rows * kChunks; c += 256) {
-          const int rr = c / kChunks, ch = c % kChunks;
-          *reinterpret_cast<uint4*>(p.o + seq_row_offset(it.sq, p.o_sb, p.o_sn, it.qt * kTile + rr) +
-                                    it.h * p.o_sh + ch * 8) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        continue;
-      }
+      if (it.n == 0) continue;  // not in [0, nwork)
       const float2 c0 = make_float2(bias_r * kLog2e, bias_r * kLog2e);
       const int t_end = t + it.n;
       for (int tt = t + ((t & 1) != g ? 1 : 0); tt < t_end; tt += 2) {
@@ -983,6 +984,7 @@ int launch_fwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.Nq = plan->Nq;
   p.H = H;
   p.nitems = plan->B * plan->QT * H;
+  p.nwork = plan->rows_nonempty * H;
   p.scale = scale;
   p.bias = bias;
   p.bias_sb = bias_sb;

@@ -83,6 +83,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test: has the phase with the given parity of `bar` completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits until the phase with the given parity of `bar` has completed.  Gives up when
 // *w.abort becomes nonzero (another role gave up) or after w.limit_ns: then records the
 // timeout in *w.status, raises *w.abort and returns false.  Never traps.
@@ -347,6 +360,66 @@ __device__ __forceinline__ void mma_ts_lh_w(uint32_t d_tmem, uint32_t a_tmem, ui
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}\n" ::"r"(d_tmem),
       "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// One tile's MMAs and the commit after them under a single elect.sync (whole-warp issue,
+// as above).  PV of one 128-key tile: 8 K-steps of 16 keys, A (P, bf16 pairs) from TMEM
+// columns a + 64 (k / 4) + 8 (k % 4), B (V, MN-major) at descriptor lo + 128 k; the first
+// step accumulates iff acc0 != 0, the others always.
+__device__ __forceinline__ void mma_pv8_commit_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                                 uint32_t b_hi, uint32_t idesc, uint32_t acc0,
+                                                 uint64_t* bar) {
+#define SIGATTN_PV_STEP(OA, OB)                                   \
+  "add.u32 ra, %1, " #OA ";\n\tadd.u32 rl, %2, " #OB ";\n\t"     \
+  "mov.b64 db, {rl, %3};\n\t"                                    \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], db, %4, q;\n\t"
+  asm volatile(
+      "{\n\t.reg .pred p, q, e;\n\t.reg .b64 db;\n\t.reg .b32 ra, rl;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\tsetp.ne.b32 q, %7, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t"
+      SIGATTN_PV_STEP(8, 128) SIGATTN_PV_STEP(16, 256) SIGATTN_PV_STEP(24, 384)
+      SIGATTN_PV_STEP(64, 512) SIGATTN_PV_STEP(72, 640) SIGATTN_PV_STEP(80, 768)
+      SIGATTN_PV_STEP(88, 896)
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(acc0), "r"(smem_u32(bar)), "r"(1u)
+      : "memory");
+#undef SIGATTN_PV_STEP
+}
+
+// S = Q K^T of one tile (overwriting D) and the commit after it: K-steps of 16 columns of
+// the 128B-swizzled K-major operands at descriptor offsets 2 (k % 4) + 1024 (k / 4) (16-byte
+// units: 32 bytes within a 64-column box, 16 KB between boxes); 4 steps for d = 64, 8 for
+// d = 128.
+template <int kSteps>
+__device__ __forceinline__ void mma_s_commit_w(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                               uint32_t hi, uint32_t idesc, uint64_t* bar) {
+  static_assert(kSteps == 4 || kSteps == 8, "d = 64 or 128");
+#define SIGATTN_S_STEP(OFF)                                                     \
+  "add.u32 la, %1, " #OFF ";\n\tadd.u32 lb, %2, " #OFF ";\n\t"                \
+  "mov.b64 da, {la, %3};\n\tmov.b64 db, {lb, %3};\n\t"                         \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, q;\n\t"
+#define SIGATTN_S_HEAD                                                           \
+  "{\n\t.reg .pred p, q, e;\n\t.reg .b64 da, db;\n\t.reg .b32 la, lb;\n\t"        \
+  "setp.ne.b32 p, %6, 1;\n\tsetp.ne.b32 q, %6, 0;\n\telect.sync _|e, 0xffffffff;\n\t" \
+  "mov.b64 da, {%1, %3};\n\tmov.b64 db, {%2, %3};\n\t"                              \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t"                   \
+  SIGATTN_S_STEP(2) SIGATTN_S_STEP(4) SIGATTN_S_STEP(6)
+#define SIGATTN_S_TAIL \
+  "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t}\n"
+  if constexpr (kSteps == 4) {
+    asm volatile(SIGATTN_S_HEAD SIGATTN_S_TAIL ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(hi),
+                 "r"(idesc), "r"(smem_u32(bar)), "r"(1u)
+                 : "memory");
+  } else {
+    asm volatile(SIGATTN_S_HEAD SIGATTN_S_STEP(1024) SIGATTN_S_STEP(1026) SIGATTN_S_STEP(1028)
+                     SIGATTN_S_STEP(1030) SIGATTN_S_TAIL ::"r"(d_tmem),
+                 "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(smem_u32(bar)), "r"(1u)
+                 : "memory");
+  }
+#undef SIGATTN_S_STEP
+#undef SIGATTN_S_HEAD
+#undef SIGATTN_S_TAIL
 }
 
 // Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, dense.
