@@ -84,90 +84,35 @@ __device__ __forceinline__ float row_D(const BwdParams& p, int b, int h, int qg)
   return p.Dws[(static_cast<int64_t>(b) * p.H + h) * p.Nq + qg];
 }
 
-// p and ds of two neighbouring elements (packed fp32 pairs); k0 / k1 are the mask bits,
-// looked at only when kMask.
+// p and ds of two neighbouring elements (packed fp32 pairs); k0 / k1 are the mask bits.
 // SIGMOID: p = sigma(x), ds = dp sigma'(x) with sigma' = sigma (1 - sigma) from the same
 //   exp2 (sigmoid_grad2); a masked element takes t = -inf, which gives p = ds = 0.
 // softmax: p = 2^t, ds = p (dp - D); a masked element takes p = 0.
-template <int EPI, bool kMask>
+template <int EPI>
 __device__ __forceinline__ void weight_grad2(float2 s, float2 dp, float2 c1, float2 off, float2 Dv,
                                              bool k0, bool k1, float2& pw, float2& ds) {
   float2 x = fma2(s, c1, off);
   if (EPI == 0) {
-    if (kMask) {
-      x.x = k0 ? x.x : -INFINITY;
-      x.y = k1 ? x.y : -INFINITY;
-    }
+    x.x = k0 ? x.x : -INFINITY;
+    x.y = k1 ? x.y : -INFINITY;
     float2 w;
     sigmoid_grad2(x, pw, w);
     ds = mul2(w, dp);
   } else {
-    pw = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-    if (kMask) pw = make_float2(k0 ? pw.x : 0.0f, k1 ? pw.y : 0.0f);
+    pw = make_float2(k0 ? ex2_approx(x.x) : 0.0f, k1 ? ex2_approx(x.y) : 0.0f);
     ds = mul2(pw, fma2(Dv, make_float2(-1.0f, -1.0f), dp));
   }
 }
 
-// Does a chunk of a row's elements need the per-element mask?  Decided for the whole warp:
-// not on FULL tiles, and not where every lane keeps every element of the chunk (`all` has
-// the chunk's bits set) -- a PARTIAL tile of a padded batch is mostly whole chunks of kept
-// or dropped keys, so only those with a dropped element pay for the mask.
-__device__ __forceinline__ bool chunk_masked(bool masked_tile, uint32_t mw, uint32_t all) {
-  return masked_tile && !__all_sync(0xFFFFFFFFu, (mw & all) == all);
-}
-
-// Clears the bf16 halves of packed pairs whose keep bit is 0 (bit 2e: low half of w[e],
-// bit 2e + 1: high half).  Zeroing the packed result equals the element's P = dS = 0 in
-// every mode, whatever was computed for it.
-template <int N>
-__device__ __forceinline__ void mask_pairs(uint32_t* w, uint32_t mw) {
-#pragma unroll
-  for (int e = 0; e < N / 2; ++e) {
-    const uint32_t lo = 0u - ((mw >> (2 * e)) & 1u), hi = 0u - ((mw >> (2 * e + 1)) & 1u);
-    w[e] &= (lo & 0x0000FFFFu) | (hi & 0xFFFF0000u);
+template <int D>
+__device__ __forceinline__ void zero_rows(__nv_bfloat16* base, int64_t sn, int rows, int tid,
+                                          int nthreads) {
+  constexpr int kChunks = D / 8;
+  for (int i = tid; i < rows * kChunks; i += nthreads) {
+    const int row = i / kChunks, c = i % kChunks;
+    *reinterpret_cast<uint4*>(base + static_cast<int64_t>(row) * sn + c * 8) =
+        make_uint4(0u, 0u, 0u, 0u);
   }
-}
-
-// P and dS of N consecutive elements of one row as packed bf16 pairs: s, dp the raw fp32
-// words of S and dP, vs the elements' row offsets (and, softmax, D at vs + 128) in shared
-// memory, mw their keep bits (bit j = element j), applied when `mask` (chunk_masked).
-template <int EPI, int N>
-__device__ __forceinline__ void grad_chunk(const uint32_t* s, const uint32_t* dp, float2 c1,
-                                           const float* vs, uint32_t mw, bool mask, uint32_t* pk,
-                                           uint32_t* dk) {
-#pragma unroll
-  for (int cc = 0; cc < N; cc += 2) {
-    float2 pw, ds;
-    const float2 off2 = *reinterpret_cast<const float2*>(vs + cc);
-    const float2 D2 =
-        EPI == 0 ? make_float2(0.0f, 0.0f) : *reinterpret_cast<const float2*>(vs + 128 + cc);
-    weight_grad2<EPI, false>(make_float2(__uint_as_float(s[cc]), __uint_as_float(s[cc + 1])),
-                             make_float2(__uint_as_float(dp[cc]), __uint_as_float(dp[cc + 1])),
-                             c1, off2, D2, true, true, pw, ds);
-    pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
-    dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
-  }
-  if (mask) {
-    mask_pairs<N>(pk, mw);
-    mask_pairs<N>(dk, mw);
-  }
-}
-
-// dS alone of N consecutive elements of one query row (the row's offset off2 and D2 shared
-// by all of them), as for grad_chunk.
-template <int EPI, int N>
-__device__ __forceinline__ void ds_chunk(const uint32_t* s, const uint32_t* dp, float2 c1,
-                                         float2 off2, float2 D2, uint32_t mw, bool mask,
-                                         uint32_t* dk) {
-#pragma unroll
-  for (int cc = 0; cc < N; cc += 2) {
-    float2 pw, ds;
-    weight_grad2<EPI, false>(make_float2(__uint_as_float(s[cc]), __uint_as_float(s[cc + 1])),
-                             make_float2(__uint_as_float(dp[cc]), __uint_as_float(dp[cc + 1])),
-                             c1, off2, D2, true, true, pw, ds);
-    dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
-  }
-  if (mask) mask_pairs<N>(dk, mw);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -720,8 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        const bool masked = meta_kind[s] == 2;
-        if (masked)
+        if (meta_kind[s] == 2)
           mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
         const float* vs = vec + s * 256 + 64 * h;
         const uint32_t base = t_lane + (u % 3) * 128;
@@ -736,8 +680,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c == 1) tmem_wait_ld();
           const uint32_t mw = c ? mb.y : mb.x;
           uint32_t pk[16], dk[16];
-          grad_chunk<EPI, 32>(sr[c], dpr[c], c1, vs + 32 * c, mw, chunk_masked(masked, mw, 0xFFFFFFFFu),
-                              pk, dk);
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            float2 pw, ds;
+            const float2 off2 = *reinterpret_cast<const float2*>(vs + 32 * c + cc);
+            const float2 D2 = EPI == 0 ? make_float2(0.0f, 0.0f)
+                                       : *reinterpret_cast<const float2*>(vs + 128 + 32 * c + cc);
+            weight_grad2<EPI>(
+                make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
+                make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])), c1, off2,
+                D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
+            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
+            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+          }
           tmem_st16(base + 16 * c, pk);
           tmem_st16(base + 64 + 16 * c, dk);
         }
@@ -780,8 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        const bool masked = meta_kind[s] == 2;
-        if (masked)
+        if (meta_kind[s] == 2)
           mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
         const float* vs = vec + s * 256 + 64 * h;
         uint32_t sr[2][32], dpr[2][32];
@@ -795,8 +749,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c == 1) tmem_wait_ld();
           const uint32_t mw = c ? mb.y : mb.x;
           uint32_t pk[16], dk[16];
-          grad_chunk<EPI, 32>(sr[c], dpr[c], c1, vs + 32 * c, mw, chunk_masked(masked, mw, 0xFFFFFFFFu),
-                              pk, dk);
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            float2 pw, ds;
+            const float2 off2 = *reinterpret_cast<const float2*>(vs + 32 * c + cc);
+            const float2 D2 = EPI == 0 ? make_float2(0.0f, 0.0f)
+                                       : *reinterpret_cast<const float2*>(vs + 128 + 32 * c + cc);
+            weight_grad2<EPI>(make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
+                              make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])),
+                              c1, off2, D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
+            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
+            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+          }
           tmem_st16(t_lane + 64 * h + 16 * c, pk);
           tmem_st16(t_lane + 128 + 64 * h + 16 * c, dk);
         }
@@ -1243,8 +1207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        const bool masked = meta_kind[s] == 2;
-        if (masked)
+        if (meta_kind[s] == 2)
           mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
         const uint32_t base = t_lane + (u % 3) * 128;
         uint32_t sr[2][32], dpr[2][32];
@@ -1258,7 +1221,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c == 1) tmem_wait_ld();
           const uint32_t mw = c ? mb.y : mb.x;
           uint32_t dk[16];
-          ds_chunk<EPI, 32>(sr[c], dpr[c], c1, off2, D2, mw, chunk_masked(masked, mw, 0xFFFFFFFFu), dk);
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            float2 pw, ds;
+            weight_grad2<EPI>(
+                make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
+                make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])), c1, off2,
+                D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
+            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+          }
           tmem_st16(base + 64 + 16 * c, dk);
         }
         tmem_wait_st();
@@ -1317,8 +1288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        const bool masked = meta_kind[s] == 2;
-        if (masked)
+        if (meta_kind[s] == 2)
           mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * h);
         uint32_t sr[2][32], dpr[2][32];
         tmem_ld32(t_lane + 64 * h, sr[0]);
@@ -1331,7 +1301,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c == 1) tmem_wait_ld();
           const uint32_t mw = c ? mb.y : mb.x;
           uint32_t dk[16];
-          ds_chunk<EPI, 32>(sr[c], dpr[c], c1, off2, D2, mw, chunk_masked(masked, mw, 0xFFFFFFFFu), dk);
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            float2 pw, ds;
+            weight_grad2<EPI>(make_float2(__uint_as_float(sr[c][cc]), __uint_as_float(sr[c][cc + 1])),
+                              make_float2(__uint_as_float(dpr[c][cc]), __uint_as_float(dpr[c][cc + 1])),
+                              c1, off2, D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
+            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+          }
           tmem_st16(t_lane + 128 + 64 * h + 16 * c, dk);
         }
         tmem_wait_st();
@@ -1730,8 +1707,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         if (!ok) break;
         tc_fence_after();
         uint2 mb = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        const bool masked = meta_kind[s] == 2;
-        if (masked)
+        if (meta_kind[s] == 2)
           mb = *reinterpret_cast<const uint2*>(meta_bits + s * 512 + row * 4 + 2 * g);
         const float* vs = vec + s * 256 + 64 * g;
         const uint32_t xb = t_lane + (t & 1) * 128 + 64 * g;
@@ -1751,8 +1727,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           }
           const uint32_t mw = (c < 2 ? mb.x : mb.y) >> (16 * (c & 1));
           uint32_t pk[8], dk[8];
-          grad_chunk<EPI, 16>(sr[c & 1], dpr[c & 1], c1, vs + 16 * c, mw,
-                              chunk_masked(masked, mw, 0xFFFFu), pk, dk);
+#pragma unroll
+          for (int cc = 0; cc < 16; cc += 2) {
+            float2 pw, ds;
+            const float2 off2 = *reinterpret_cast<const float2*>(vs + 16 * c + cc);
+            const float2 D2 = EPI == 0 ? make_float2(0.0f, 0.0f)
+                                       : *reinterpret_cast<const float2*>(vs + 128 + 16 * c + cc);
+            weight_grad2<EPI>(
+                make_float2(__uint_as_float(sr[c & 1][cc]), __uint_as_float(sr[c & 1][cc + 1])),
+                make_float2(__uint_as_float(dpr[c & 1][cc]), __uint_as_float(dpr[c & 1][cc + 1])),
+                c1, off2, D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
+            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
+            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+          }
           tmem_st8(xb + 16 * c, pk);
           tmem_st8(xb + 16 * c + 8, dk);
           if (c < 3) tmem_wait_ld();
