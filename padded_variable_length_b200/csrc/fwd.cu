@@ -771,8 +771,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (first && i >= OB && !mbar_wait_w(o_empty + ob, ((i / OB) - 1) & 1, wctx))
           return false;
         tc_fence_after();
-        mma_pv8_commit_w(tmem + L::kOCol + ob * D, tmem + b3 * 128, v_lo0 + sv * kTileLo, kHiMn,
-                         idesc_pv, first ? 0u : 1u, step + (x & 3));
+        if constexpr (D == 64) {
+          // Paced: a tcgen05.mma that finds the tensor pipe's queue full holds the issuing
+          // SM sub-partition (and the two epilogue warps beside this warp) until there is
+          // room.  The PV of a d = 64 tile is eight short MMAs (32 tensor cycles each) right
+          // before S: issued four at a time with a short sleep between, the queue keeps room
+          // and the neighbours keep issuing (measured 4 % on the single-cell batch; d = 128,
+          // whose MMAs are twice as long and whose epilogue has more slack, is better off
+          // unpaced).
+          const uint32_t o_tmem = tmem + L::kOCol + ob * D, p_tmem = tmem + b3 * 128;
+          const uint32_t v_lo = v_lo0 + sv * kTileLo;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            if (kk == 4) __nanosleep(64);
+            mma_ts_lh_w(o_tmem, p_tmem + (kk >> 2) * 64 + (kk & 3) * 8, v_lo + kk * 128, kHiMn,
+                        idesc_pv, (first && kk == 0) ? 0u : 1u);
+          }
+          mma_commit_w(step + (x & 3));
+          __nanosleep(64);
+        } else {
+          mma_pv8_commit_w(tmem + L::kOCol + ob * D, tmem + b3 * 128, v_lo0 + sv * kTileLo,
+                           kHiMn, idesc_pv, first ? 0u : 1u, step + (x & 3));
+        }
         if (last) mma_commit_w(o_full + ob);
         return true;
       };
