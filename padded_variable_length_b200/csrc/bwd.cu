@@ -1852,44 +1852,41 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
 // Zeroes the fp32 dQ accumulator rows of every q-tile that has tiles (the others are never
 // read): rows qt*128 .. of batch entry b for each listed row r = b*QT + qt.
-__global__ void dq_zero_kernel(const int4* __restrict__ row_desc, int rows_nonempty, int QT, int Nq,
-                               int H, float* __restrict__ dqacc) {
-  constexpr int kVec = 64 / 4;  // float4 per (row, head), d = 64
-  const int64_t per_tile = static_cast<int64_t>(kTile) * H * kVec;
-  const int64_t total = per_tile * rows_nonempty;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int r = row_desc[i / per_tile].x;
-    const int64_t w = i % per_tile;
-    const int rr = static_cast<int>(w / (H * kVec));
-    const int b = r / QT, qt = r % QT;
-    const int q = qt * kTile + rr;
-    if (q >= Nq) continue;
-    const int64_t off = ((static_cast<int64_t>(b) * Nq + q) * H) * 64 + (w % (H * kVec)) * 4;
-    *reinterpret_cast<float4*>(dqacc + off) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  }
+__global__ void dq_zero_kernel(const int4* __restrict__ row_desc, int QT, int Nq, int H,
+                               float* __restrict__ dqacc) {
+  // one block per listed q-tile (the first rows_nonempty entries of the sorted row list):
+  // its rows are one contiguous span of the [B, Nq, H, 64] accumulator
+  const int r = row_desc[blockIdx.x].x;
+  const int b = r / QT, qt = r % QT;
+  const int rows = min(kTile, Nq - qt * kTile);
+  float4* base = reinterpret_cast<float4*>(
+      dqacc + (static_cast<int64_t>(b) * Nq + static_cast<int64_t>(qt) * kTile) * H * 64);
+  const int n = rows * H * 16;  // float4 per row: 64 H / 4
+  for (int i = threadIdx.x; i < n; i += blockDim.x) base[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 }
 
-// dQ = bf16(scale * dQacc) on rows of q-tiles with tiles, 0 on every other row.  One thread
-// per 8 elements (16 bytes of dQ).
+// dQ = bf16(scale * dQacc) on rows of q-tiles with tiles, 0 on every other row.  One block
+// per (q-tile, sequence); one thread per 8 elements (16 bytes of dQ) of the tile's rows.
 __global__ void dq_convert_kernel(const int32_t* __restrict__ row_ptr, const float* __restrict__ dqacc,
-                                  int B, int QT, int Nq, int H, const int32_t* __restrict__ cu,
+                                  int QT, int Nq, int H, const int32_t* __restrict__ cu,
                                   float scale, __nv_bfloat16* __restrict__ dq, int64_t sb, int64_t sn,
                                   int64_t sh) {
-  constexpr int kChunks = 64 / 8;
-  const int64_t total = static_cast<int64_t>(B) * Nq * H * kChunks;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(i % kChunks);
-    const int h = static_cast<int>((i / kChunks) % H);
-    const int64_t bq = i / (static_cast<int64_t>(kChunks) * H);
-    const int q = static_cast<int>(bq % Nq), b = static_cast<int>(bq / Nq);
-    const int r = b * QT + q / kTile;
-    const SeqRows sq = seq_rows(cu, b, Nq);
-    if (q >= sq.limit) continue;  // a packed sequence owns only its own rows
+  const int qt = blockIdx.x, b = blockIdx.y;
+  const SeqRows sq = seq_rows(cu, b, Nq);
+  const int rows = min(kTile, sq.limit - qt * kTile);  // a packed sequence owns only its rows
+  if (rows <= 0) return;
+  const int r = b * QT + qt;
+  const bool listed = row_ptr[r + 1] > row_ptr[r];
+  const int per_row = H * 8;
+  const int n = rows * per_row;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int rr = i / per_row, hc = i - rr * per_row;
+    const int h = hc >> 3, c = hc & 7;
+    const int q = qt * kTile + rr;
     uint4 out = make_uint4(0u, 0u, 0u, 0u);
-    if (row_ptr[r + 1] > row_ptr[r]) {
-      const float4* src = reinterpret_cast<const float4*>(dqacc + (bq * H + h) * 64 + c * 8);
+    if (listed) {
+      const float4* src = reinterpret_cast<const float4*>(
+          dqacc + ((static_cast<int64_t>(b) * Nq + q) * H + h) * 64 + c * 8);
       const float4 a = src[0], e = src[1];
       out = make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
                        pack_bf16x2(e.x * scale, e.y * scale), pack_bf16x2(e.z * scale, e.w * scale));
@@ -2042,10 +2039,8 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
   }
   const int sms = num_sms();
   if (plan->rows_nonempty > 0) {
-    const int64_t work = static_cast<int64_t>(plan->rows_nonempty) * kTile * H * (D / 4);
-    const int blocks = static_cast<int>(std::min<int64_t>((work + 255) / 256, sms * 8));
-    dq_zero_kernel<<<blocks, 256, 0, stream>>>(plan->row_desc, plan->rows_nonempty, plan->QT,
-                                                plan->Nq, H, dqacc);
+    dq_zero_kernel<<<plan->rows_nonempty, 512, 0, stream>>>(plan->row_desc, plan->QT, plan->Nq,
+                                                             H, dqacc);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   static_assert(FusedLayout::kAlloc <= 227 * 1024, "shared memory");
@@ -2060,10 +2055,8 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   {
-    const int64_t work = static_cast<int64_t>(plan->B) * plan->Nq * H * (D / 8);
-    const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, sms * 8)));
-    dq_convert_kernel<<<blocks, 256, 0, stream>>>(plan->row_ptr, dqacc, plan->B, plan->QT, plan->Nq,
-                                                   H, plan->cu, scale,
+    dq_convert_kernel<<<dim3(plan->QT, plan->B), 256, 0, stream>>>(plan->row_ptr, dqacc, plan->QT,
+                                                                     plan->Nq, H, plan->cu, scale,
                                                    static_cast<__nv_bfloat16*>(const_cast<void*>(dq.ptr)),
                                                    dq.sb, dq.sn, dq.sh);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
