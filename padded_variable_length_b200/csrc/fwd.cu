@@ -999,7 +999,7 @@ int launch_fwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.row_desc = plan->row_desc;
   p.cu = plan->cu;
   p.run = plan->run;
-  p.run_cap = static_cast<int>(plan->nonempty);
+  p.run_cap = static_cast<int>(plan->run_cap);
   p.QT = plan->QT;
   p.Nq = plan->Nq;
   p.H = H;

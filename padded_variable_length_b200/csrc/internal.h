@@ -23,6 +23,7 @@ struct sigattn_plan {
   void* arena[2];  // the two device allocations every buffer below is carved from
   int B, Nq, Nk, QT, KT;
   int64_t nonempty, full, partial;
+  int64_t run_cap;  // entries allocated in the per-tile arrays (>= nonempty)
   int32_t rows_nonempty, cols_nonempty;
   int32_t* row_ptr;
   int32_t* col_idx;

@@ -95,22 +95,56 @@ __device__ __forceinline__ void half_row_bits(const uint8_t* __restrict__ mask, 
 
 // One CTA of 256 threads per block (b, qt, kt): thread t covers row t/2, columns
 // (t%2)*64 .. +64 of the block.
+// One warp per block of the grid (grid-stride): lane l reads 16 bytes at column
+// 16 (l % 8) of rows l / 8, l / 8 + 4, ... -- every load instruction of the warp covers four
+// whole 128-byte rows -- and the warp votes on "any element kept" and "all kept".  Rows
+// past Nq and columns past Nk count as not kept.  Masks whose rows are not 16-byte aligned
+// take a byte-wise path.
 __global__ void __launch_bounds__(256) k_kinds_from_mask(const uint8_t* __restrict__ mask, int B,
                                                          int Nq, int Nk, int64_t sb, int64_t sq,
                                                          int QT, int KT,
                                                          uint8_t* __restrict__ kinds) {
-  const int64_t blk = blockIdx.x;
-  const int kt = static_cast<int>(blk % KT);
-  const int qt = static_cast<int>((blk / KT) % QT);
-  const int b = static_cast<int>(blk / (static_cast<int64_t>(KT) * QT));
-  const int row = qt * kTile + (threadIdx.x >> 1);
-  const int col0 = kt * kTile + (threadIdx.x & 1) * 64;
-  uint32_t w0, w1;
-  bool all;
-  half_row_bits(mask, Nq, Nk, sb, sq, b, row, col0, w0, w1, all);
-  const int any_b = __syncthreads_or((w0 | w1) != 0u);
-  const int all_b = __syncthreads_and(all);
-  if (threadIdx.x == 0) kinds[blk] = all_b ? 1 : (any_b ? 2 : 0);
+  const int64_t total = static_cast<int64_t>(B) * QT * KT;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const bool vec = ((reinterpret_cast<uintptr_t>(mask) | static_cast<uintptr_t>(sb) |
+                     static_cast<uintptr_t>(sq)) & 15u) == 0;
+  for (int64_t blk = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+       blk < total; blk += nwarps) {
+    const int kt = static_cast<int>(blk % KT);
+    const int qt = static_cast<int>((blk / KT) % QT);
+    const int b = static_cast<int>(blk / (static_cast<int64_t>(KT) * QT));
+    const int col = kt * kTile + (lane & 7) * 16;
+    const uint8_t* base = mask + b * sb + col;
+    bool any = false, all = true;
+    if (vec && kt * kTile + kTile <= Nk) {
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) {
+        const int row = qt * kTile + (lane >> 3) + 4 * i;
+        if (row < Nq) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + row * sq));
+          any |= (v.x | v.y | v.z | v.w) != 0u;
+          all &= (nonzero_bytes(v.x) & nonzero_bytes(v.y) & nonzero_bytes(v.z) &
+                  nonzero_bytes(v.w)) == 0x80808080u;
+        } else {
+          all = false;
+        }
+      }
+    } else {
+      for (int i = 0; i < 32; ++i) {
+        const int row = qt * kTile + (lane >> 3) + 4 * i;
+        for (int j = 0; j < 16; ++j) {
+          const bool in = row < Nq && col + j < Nk;
+          const bool kept = in && base[row * sq + j] != 0;
+          any |= kept;
+          all &= kept;
+        }
+      }
+    }
+    any = __any_sync(0xFFFFFFFFu, any);
+    all = __all_sync(0xFFFFFFFFu, all);
+    if (lane == 0) kinds[blk] = all ? 1 : (any ? 2 : 0);
+  }
 }
 
 // One warp per q-tile row r < rows (number of listed blocks and of PARTIAL blocks), then
@@ -382,10 +416,13 @@ __device__ __forceinline__ void store_transposed(const uint32_t* w, uint32_t* __
 __global__ void __launch_bounds__(256) k_bits_from_mask(const uint8_t* __restrict__ mask, int Nq,
                                                         int Nk, int64_t sb, int64_t sq, int QT,
                                                         int KT, const int64_t* __restrict__ ptile,
+                                                        const int64_t* __restrict__ np,
                                                         uint32_t* __restrict__ bits,
                                                         uint32_t* __restrict__ bitsT) {
   __shared__ uint32_t w[512];
-  const int64_t g = ptile[blockIdx.x];
+  const int64_t n = *np;  // PARTIAL blocks, from the counting step
+  for (int64_t pb = blockIdx.x; pb < n; pb += gridDim.x) {
+  const int64_t g = ptile[pb];
   const int kt = static_cast<int>(g % KT);
   const int qt = static_cast<int>((g / KT) % QT);
   const int b = static_cast<int>(g / (static_cast<int64_t>(KT) * QT));
@@ -393,13 +430,15 @@ __global__ void __launch_bounds__(256) k_bits_from_mask(const uint8_t* __restric
   uint32_t w0, w1;
   bool all;
   half_row_bits(mask, Nq, Nk, sb, sq, b, qt * kTile + q, kt * kTile + half * 64, w0, w1, all);
-  uint32_t* dst = bits + static_cast<int64_t>(blockIdx.x) * 512 + q * 4 + half * 2;
+  uint32_t* dst = bits + pb * 512 + q * 4 + half * 2;
   dst[0] = w0;
   dst[1] = w1;
   w[q * 4 + half * 2] = w0;
   w[q * 4 + half * 2 + 1] = w1;
   __syncthreads();
-  if (threadIdx.x < 128) store_transposed(w, bitsT + static_cast<int64_t>(blockIdx.x) * 512);
+  if (threadIdx.x < 128) store_transposed(w, bitsT + pb * 512);
+  __syncthreads();
+  }
 }
 
 // One CTA of 128 threads per PARTIAL block of a padded batch: row q is valid iff
@@ -408,9 +447,12 @@ __global__ void __launch_bounds__(256) k_bits_from_mask(const uint8_t* __restric
 __global__ void __launch_bounds__(128) k_bits_from_lengths(const int32_t* __restrict__ lengths,
                                                            int Npad, int QT, int KT,
                                                            const int64_t* __restrict__ ptile,
+                                                           const int64_t* __restrict__ np,
                                                            uint32_t* __restrict__ bits,
                                                            uint32_t* __restrict__ bitsT) {
-  const int64_t g = ptile[blockIdx.x];
+  const int64_t npart = *np;  // PARTIAL blocks, from the counting step
+  for (int64_t pb = blockIdx.x; pb < npart; pb += gridDim.x) {
+  const int64_t g = ptile[pb];
   const int kt = static_cast<int>(g % KT);
   const int qt = static_cast<int>((g / KT) % QT);
   const int b = static_cast<int>(g / (static_cast<int64_t>(KT) * QT));
@@ -422,14 +464,15 @@ __global__ void __launch_bounds__(128) k_bits_from_lengths(const int32_t* __rest
   w.y = row_ok ? low_bits(n - (kt * kTile + 32)) : 0u;
   w.z = row_ok ? low_bits(n - (kt * kTile + 64)) : 0u;
   w.w = row_ok ? low_bits(n - (kt * kTile + 96)) : 0u;
-  reinterpret_cast<uint4*>(bits + static_cast<int64_t>(blockIdx.x) * 512)[q] = w;
+  reinterpret_cast<uint4*>(bits + pb * 512)[q] = w;
   const bool col_ok = kt * kTile + q < n;
   uint4 wt;
   wt.x = col_ok ? low_bits(n - (qt * kTile + 0)) : 0u;
   wt.y = col_ok ? low_bits(n - (qt * kTile + 32)) : 0u;
   wt.z = col_ok ? low_bits(n - (qt * kTile + 64)) : 0u;
   wt.w = col_ok ? low_bits(n - (qt * kTile + 96)) : 0u;
-  reinterpret_cast<uint4*>(bitsT + static_cast<int64_t>(blockIdx.x) * 512)[q] = wt;
+  reinterpret_cast<uint4*>(bitsT + pb * 512)[q] = wt;
+  }
 }
 
 // desc[k] = {work[k], ptr[work[k]], ptr[work[k] + 1] - ptr[work[k]], w} for the row list
@@ -567,14 +610,49 @@ int grid_for(int64_t work, int per_block) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(g, 1 << 30)));
 }
 
+// Plan memory for the tile lists: nz listed tiles, np of them PARTIAL.
+struct TileArena {
+  size_t ci, k, pi, ri, cm, b, bt, run, bytes;
+  TileArena(size_t nz, size_t np) {
+    Carve c;
+    ci = c.add<int32_t>(nz);
+    k = c.add<uint8_t>(nz);
+    pi = c.add<int32_t>(nz);
+    ri = c.add<int32_t>(nz);
+    cm = c.add<int32_t>(nz);
+    b = c.add<uint32_t>(np * 512);
+    bt = c.add<uint32_t>(np * 512);
+    run = c.add<int4>(nz);  // at most one run per listed tile
+    bytes = c.bytes;
+  }
+  void place(sigattn_plan* plan, void* m) const {
+    plan->col_idx = Carve::at<int32_t>(m, ci);
+    plan->kind = Carve::at<uint8_t>(m, k);
+    plan->pidx = Carve::at<int32_t>(m, pi);
+    plan->rowT_idx = Carve::at<int32_t>(m, ri);
+    plan->csc_map = Carve::at<int32_t>(m, cm);
+    plan->bits = Carve::at<uint32_t>(m, b);
+    plan->bitsT = Carve::at<uint32_t>(m, bt);
+    plan->run = Carve::at<int4>(m, run);
+  }
+};
+
+// Tile arrays sized for the worst case up to this many bytes, so that the whole plan is
+// queued before the one synchronisation; above it the counts are read back first.
+constexpr size_t kOnePassBytes = size_t(256) << 20;
+
 // Both planners: `classify` writes every block's kind into sc.kinds, `bits_kernel` the
-// bitmasks of the PARTIAL blocks.  Two plan allocations (one sized by the grid, one by the
-// number of listed tiles, known after the one synchronisation), two scratch allocations.
-// cu_src (packed batches only): the cumulative offsets, copied into the plan; check_dev /
-// check_host: one device int read back at the synchronisation (an argument check).
+// bitmasks of the PARTIAL blocks (their number read on the device).  np_bound: most
+// PARTIAL blocks the classification can yield (the grid for a mask; two tile strips per
+// sequence for lengths).  When the tile arrays sized for the grid and np_bound fit
+// kOnePassBytes, every step is queued and the host synchronises once at the end, for the
+// counts and the argument checks; otherwise it synchronises after the counting step and
+// sizes the arrays exactly.  cu_src (packed batches only): the cumulative offsets, copied
+// into the plan; check_dev / check_host: one device int read back at the synchronisation
+// (an argument check).
 template <class ClassifyFn, class BitsFn>
 int build_plan(sigattn_plan* plan, cudaStream_t stream, ClassifyFn classify, BitsFn bits_kernel,
-               sigattn_plan** out, const int32_t* cu_src = nullptr,
+               sigattn_plan** out, int64_t np_bound, const int32_t* cu_src = nullptr,
                const int32_t* check_dev = nullptr, int32_t* check_host = nullptr) {
   Scratch sc;
   const int B = plan->B, QT = plan->QT, KT = plan->KT;
@@ -631,6 +709,29 @@ int build_plan(sigattn_plan* plan, cudaStream_t stream, ClassifyFn classify, Bit
       plan->row_work, plan->row_ptr, plan->run_ptr, rows, plan->row_desc, plan->col_work,
       plan->colT_ptr, cols, plan->col_desc);
   SIGATTN_TRY_CUDA(cudaGetLastError());
+  const int64_t np_max = std::min<int64_t>(grid_total, np_bound);
+  const TileArena worst(static_cast<size_t>(grid_total), static_cast<size_t>(np_max));
+  const bool one_pass = worst.bytes <= kOnePassBytes;
+  // the fill steps, on arrays of capacity for (nz_cap, np_cap) tiles
+  auto fill = [&](int64_t np_cap) -> int {
+    SIGATTN_TRY(scratch_alloc(&sc.block[1], std::max<int64_t>(np_cap, 1) * sizeof(int64_t),
+                              stream));
+    sc.ptile = static_cast<int64_t*>(sc.block[1]);
+    k_fill_csr<<<grid_for(static_cast<int64_t>(rows) * 32, 256), 256, 0, stream>>>(
+        sc.kinds, rows, KT, plan->row_ptr, sc.row_poff, plan->col_idx, plan->kind, plan->pidx,
+        sc.eidx, sc.ptile, plan->run_ptr, plan->run);
+    k_fill_csc<<<grid_for(static_cast<int64_t>(cols) * 32, 256), 256, 0, stream>>>(
+        sc.kinds, sc.eidx, B, QT, KT, plan->colT_ptr, plan->rowT_idx, plan->csc_map);
+    if (np_cap > 0)
+      bits_kernel(sc.ptile, sc.totals + 1, plan->bits, plan->bitsT,
+                  static_cast<int>(std::min<int64_t>(np_cap, 2048)));
+    return cuda_status(cudaGetLastError());
+  };
+  if (one_pass) {
+    SIGATTN_TRY(plan_alloc(&plan->arena[1], worst.bytes, stream));
+    worst.place(plan, plan->arena[1]);
+    SIGATTN_TRY(fill(np_max));
+  }
   int64_t totals[4] = {0, 0, 0, 0};
   int32_t last_row = 0;
   SIGATTN_TRY_CUDA(cudaMemcpyAsync(totals, sc.totals, sizeof(totals), cudaMemcpyDeviceToHost,
@@ -650,36 +751,14 @@ int build_plan(sigattn_plan* plan, cudaStream_t stream, ClassifyFn classify, Bit
   plan->full = totals[0] - totals[1];
   plan->rows_nonempty = static_cast<int32_t>(totals[2]);
   plan->cols_nonempty = static_cast<int32_t>(totals[3]);
-  const size_t nz = static_cast<size_t>(plan->nonempty), np = static_cast<size_t>(plan->partial);
-  {
-    Carve c;
-    const size_t o_ci = c.add<int32_t>(nz), o_k = c.add<uint8_t>(nz), o_pi = c.add<int32_t>(nz),
-                 o_ri = c.add<int32_t>(nz), o_cm = c.add<int32_t>(nz),
-                 o_b = c.add<uint32_t>(np * 512), o_bt = c.add<uint32_t>(np * 512),
-                 o_run = c.add<int4>(nz);  // at most one run per listed tile
-    SIGATTN_TRY(plan_alloc(&plan->arena[1], c.bytes, stream));
-    void* m = plan->arena[1];
-    plan->col_idx = Carve::at<int32_t>(m, o_ci);
-    plan->kind = Carve::at<uint8_t>(m, o_k);
-    plan->pidx = Carve::at<int32_t>(m, o_pi);
-    plan->rowT_idx = Carve::at<int32_t>(m, o_ri);
-    plan->csc_map = Carve::at<int32_t>(m, o_cm);
-    plan->bits = Carve::at<uint32_t>(m, o_b);
-    plan->bitsT = Carve::at<uint32_t>(m, o_bt);
-    plan->run = Carve::at<int4>(m, o_run);
+  if (!one_pass) {
+    const TileArena exact(static_cast<size_t>(plan->nonempty), static_cast<size_t>(plan->partial));
+    SIGATTN_TRY(plan_alloc(&plan->arena[1], exact.bytes, stream));
+    exact.place(plan, plan->arena[1]);
+    SIGATTN_TRY(fill(plan->partial));
   }
-  SIGATTN_TRY(scratch_alloc(&sc.block[1], np * sizeof(int64_t), stream));
-  sc.ptile = static_cast<int64_t*>(sc.block[1]);
-  if (plan->nonempty > 0) {
-    k_fill_csr<<<grid_for(static_cast<int64_t>(rows) * 32, 256), 256, 0, stream>>>(
-        sc.kinds, rows, KT, plan->row_ptr, sc.row_poff, plan->col_idx, plan->kind, plan->pidx,
-        sc.eidx, sc.ptile, plan->run_ptr, plan->run);
-    k_fill_csc<<<grid_for(static_cast<int64_t>(cols) * 32, 256), 256, 0, stream>>>(
-        sc.kinds, sc.eidx, B, QT, KT, plan->colT_ptr, plan->rowT_idx, plan->csc_map);
-  }
-  if (plan->partial > 0)
-    bits_kernel(sc.ptile, plan->bits, plan->bitsT, static_cast<int>(plan->partial));
-  SIGATTN_TRY_CUDA(cudaGetLastError());
+  // one entry past the listed tiles stays readable: kernels bound their reads by it
+  plan->run_cap = one_pass ? grid_total : plan->nonempty;
   sc.release(stream);
   *out = plan;
   return SIGATTN_OK;
@@ -720,10 +799,12 @@ extern "C" int sigattn_plan_from_lengths(const int32_t* d_lengths, int B, int Np
     k_kinds_from_lengths<<<grid_for(grid_total, 256), 256, 0, stream>>>(d_lengths, B, Npad, QT,
                                                                           QT, kinds);
   };
-  auto bits = [&](const int64_t* ptile, uint32_t* dst, uint32_t* dstT, int np) {
-    k_bits_from_lengths<<<np, 128, 0, stream>>>(d_lengths, Npad, QT, QT, ptile, dst, dstT);
+  auto bits = [&](const int64_t* ptile, const int64_t* np, uint32_t* dst, uint32_t* dstT,
+                  int grid) {
+    k_bits_from_lengths<<<grid, 128, 0, stream>>>(d_lengths, Npad, QT, QT, ptile, np, dst, dstT);
   };
-  return build_plan(plan, stream, classify, bits, out);
+  // PARTIAL blocks of a length: the last q-tile row and k-tile column of the sequence
+  return build_plan(plan, stream, classify, bits, out, 2 * static_cast<int64_t>(B) * QT);
 }
 
 namespace sigattn {
@@ -775,11 +856,14 @@ extern "C" int sigattn_plan_from_cu_seqlens(const int32_t* d_cu, int B, int max_
     k_kinds_from_lengths<<<grid_for(grid_total, 256), 256, 0, stream>>>(lengths, B, max_seqlen, QT,
                                                                           QT, kinds);
   };
-  auto bits = [&](const int64_t* ptile, uint32_t* dst, uint32_t* dstT, int np) {
-    k_bits_from_lengths<<<np, 128, 0, stream>>>(lengths, max_seqlen, QT, QT, ptile, dst, dstT);
+  auto bits = [&](const int64_t* ptile, const int64_t* np, uint32_t* dst, uint32_t* dstT,
+                  int grid) {
+    k_bits_from_lengths<<<grid, 128, 0, stream>>>(lengths, max_seqlen, QT, QT, ptile, np, dst,
+                                                  dstT);
   };
   int32_t bad_host = 0;
-  rc = build_plan(plan, stream, classify, bits, out, d_cu, bad, &bad_host);
+  rc = build_plan(plan, stream, classify, bits, out, 2 * static_cast<int64_t>(B) * QT, d_cu, bad,
+                  &bad_host);
   cudaFreeAsync(tmp, stream);
   return rc;
 }
@@ -805,14 +889,17 @@ extern "C" int sigattn_plan_from_mask(const uint8_t* d_mask, int B, int Nq, int 
   plan->KT = KT;
   const int64_t grid_total = static_cast<int64_t>(B) * QT * KT;
   auto classify = [&](uint8_t* kinds) {
-    k_kinds_from_mask<<<static_cast<unsigned>(grid_total), 256, 0, stream>>>(
+    // one warp per block, eight per CTA, at most 16 CTAs per SM's worth of work at once
+    const int64_t ctas = std::min<int64_t>((grid_total + 7) / 8, 148 * 16);
+    k_kinds_from_mask<<<static_cast<unsigned>(ctas), 256, 0, stream>>>(
         d_mask, B, Nq, Nk, stride_b, stride_q, QT, KT, kinds);
   };
-  auto bits = [&](const int64_t* ptile, uint32_t* dst, uint32_t* dstT, int np) {
-    k_bits_from_mask<<<np, 256, 0, stream>>>(d_mask, Nq, Nk, stride_b, stride_q, QT, KT, ptile,
-                                             dst, dstT);
+  auto bits = [&](const int64_t* ptile, const int64_t* np, uint32_t* dst, uint32_t* dstT,
+                  int grid) {
+    k_bits_from_mask<<<grid, 256, 0, stream>>>(d_mask, Nq, Nk, stride_b, stride_q, QT, KT, ptile,
+                                               np, dst, dstT);
   };
-  return build_plan(plan, stream, classify, bits, out);
+  return build_plan(plan, stream, classify, bits, out, grid_total);
 }
 
 extern "C" int sigattn_plan_get_sizes(const sigattn_plan* plan, sigattn_plan_sizes* sz) {
