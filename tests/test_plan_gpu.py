@@ -138,3 +138,66 @@ def test_plan_runs_bit_exact(case):
     ref_ptr, ref_runs = OT.row_runs(ref)
     assert np.array_equal(run_ptr, ref_ptr)
     assert np.array_equal(runs, ref_runs)
+
+
+def _lengths_plan_closed_form(lengths, npad):
+    """The tile list of a lengths plan written out directly (no oracle pass over the grid):
+    sequence b with n valid rows lists the T x T tiles of its first T = ceil(n / 128)
+    q-tiles and k-tiles; a tile is FULL iff both of its 128-row ranges lie inside n."""
+    QT = (npad + 127) // 128
+    n = np.clip(np.asarray(lengths, dtype=np.int64), 0, npad)
+    T, F = (n + 127) // 128, n // 128
+    row_cnt = np.zeros((len(n), QT), dtype=np.int64)
+    for b in range(len(n)):
+        row_cnt[b, :T[b]] = T[b]
+    row_ptr = np.concatenate([[0], np.cumsum(row_cnt.ravel())]).astype(np.int32)
+    col_idx, kind, csc_map = [], [], []
+    for b in range(len(n)):
+        t, f = int(T[b]), int(F[b])
+        if t == 0:
+            continue
+        qt, kt = np.meshgrid(np.arange(t), np.arange(t), indexing="ij")
+        col_idx.append(kt.ravel())
+        kind.append(np.where((qt < f) & (kt < f), 1, 2).ravel())
+        base = row_ptr[b * QT: b * QT + t].astype(np.int64)
+        csc_map.append((base[None, :] + np.arange(t)[:, None]).ravel())  # column kt, row qt
+    col_idx = np.concatenate(col_idx).astype(np.int32)
+    kind = np.concatenate(kind).astype(np.uint8)
+    pidx = np.full(len(kind), -1, dtype=np.int32)
+    pidx[kind == 2] = np.arange(int((kind == 2).sum()), dtype=np.int32)
+    return {"row_ptr": row_ptr, "col_idx": col_idx, "kind": kind, "pidx": pidx,
+            "colT_ptr": row_ptr, "rowT_idx": col_idx,
+            "csc_map": np.concatenate(csc_map).astype(np.int32)}
+
+
+def test_plan_large_grid_sizes_after_counting():
+    """A grid large enough (4.2 M blocks) that the planner reads the counts back before it
+    sizes the tile arrays, instead of sizing them for the worst case: the lists equal the
+    closed form, and sampled PARTIAL bitmasks equal the rows and columns inside n."""
+    from padded_variable_length_b200 import binding as Bd
+    rng = np.random.default_rng(31)
+    npad = 16384
+    lengths = rng.integers(0, npad + 1, 256).astype(np.int32)
+    lengths[:3] = [npad, 0, 128 * 7]
+    plan = Bd.Plan.from_lengths(torch.from_numpy(lengths).cuda(), npad)
+    got = plan.export()
+    ref = _lengths_plan_closed_form(lengths, npad)
+    for k in ("row_ptr", "col_idx", "kind", "pidx", "colT_ptr", "rowT_idx", "csc_map"):
+        assert np.array_equal(got[k], ref[k]), f"{k} differs"
+    z = plan.sizes()
+    assert z["nonempty"] == len(ref["col_idx"]) and z["partial"] == got["bits"].shape[0]
+    # PARTIAL bitmasks, sampled: row q keeps column k iff both lie inside the sequence
+    QT = (npad + 127) // 128
+    ends = np.repeat(np.arange(len(lengths)), QT)  # batch entry of each q-tile row
+    part = np.flatnonzero(ref["kind"] == 2)
+    rows_of = np.searchsorted(ref["row_ptr"], np.arange(len(ref["kind"])), side="right") - 1
+    for e in rng.choice(part, 64, replace=False):
+        r = rows_of[e]
+        b, qt, kt = ends[r], r % QT, ref["col_idx"][e]
+        nv = int(min(max(lengths[b], 0), npad))
+        q_ok = qt * 128 + np.arange(128) < nv
+        k_ok = kt * 128 + np.arange(128) < nv
+        dense = q_ok[:, None] & k_ok[None, :]
+        words = np.packbits(dense.reshape(128, 4, 32)[:, :, ::-1], axis=-1, bitorder="big")
+        want = words.view(">u4").reshape(128, 4).astype(np.uint32).ravel()
+        assert np.array_equal(got["bits"][ref["pidx"][e]], want), f"bits of tile {e}"
