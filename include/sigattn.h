@@ -96,8 +96,12 @@ typedef struct sigattn_plan_sizes {
 /*
  * Plan for a padded batch: query i of batch entry b sees key j iff i < n_b and
  * j < n_b (Nq = Nk = Npad).  d_lengths: device int32 [B], each in [0, Npad].
- * Builds the tile list on the device; synchronises `stream` once to size the
- * plan's buffers.  On success *out owns device memory until sigattn_plan_destroy.
+ * Builds the tile list on the device and synchronises `stream` once, at the end, to read
+ * the counts and the argument checks.  Plan memory: the tile arrays are sized for the
+ * worst case (every block listed; for lengths, two PARTIAL tile strips per sequence, for a
+ * mask every block PARTIAL at 4 KB each) when that is at most 256 MB, so that nothing waits
+ * for the counts; a larger worst case reads the counts back first and sizes the arrays
+ * exactly.  On success *out owns device memory until sigattn_plan_destroy.
  * Errors: INVALID (null, B < 1, Npad < 1), UNSUPPORTED (B * QT * KT > 2^28),
  * CUDA, NOMEM.  Lengths outside [0, Npad] are clamped into it.
  */
@@ -108,7 +112,8 @@ SIGATTN_API int sigattn_plan_from_lengths(const int32_t* d_lengths, int B, int N
  * Plan for an element mask: d_mask is device uint8 [B, Nq, Nk], nonzero = attend;
  * element (b, i, j) at d_mask[b * stride_b + i * stride_q + j].  The mask is shared by
  * all heads.  Reads the mask once to classify blocks and once more for the PARTIAL
- * blocks' bitmasks.  Synchronises `stream` once.  Errors as for the lengths plan.
+ * blocks' bitmasks.  Synchronises `stream` once; plan memory as for the lengths plan.
+ * Errors as for the lengths plan.
  */
 SIGATTN_API int sigattn_plan_from_mask(const uint8_t* d_mask, int B, int Nq, int Nk, int64_t stride_b,
                            int64_t stride_q, sigattn_stream stream, sigattn_plan** out);
