@@ -188,7 +188,11 @@ def key_columns_backward(q, k, v, do, mask_rows, bias, scale, epilogue, cols, o=
             a, e = _key_range(m)
             s = scale * (q[i0:i1] @ k[a:e].T) + bias[i0:i1, None]
             pf, _ = weights(s, m[:, a:e], epilogue)
-            p = pf[:, cols - a]
+            # a key outside the chunk's key range is masked for every row of the chunk:
+            # its weight is 0
+            p = np.zeros((i1 - i0, cols.size))
+            inside = (cols >= a) & (cols < e)
+            p[:, inside] = pf[:, cols[inside] - a]
         dp = do[i0:i1] @ v[cols].T
         if epilogue == SIGMOID:
             ds = dp * p * (1.0 - p)

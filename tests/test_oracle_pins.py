@@ -333,6 +333,29 @@ def test_sampled_row_and_column_helpers_match_full():
         np.testing.assert_allclose(dv_s, dv[cols], rtol=1e-11, atol=1e-14)
 
 
+def test_column_helper_with_narrow_key_ranges():
+    """Causal documents: each row chunk sees a narrow key range, so sampled key columns lie
+    outside it for most chunks (weight 0 there).  The column helper still equals the full
+    backward, for every epilogue (the softmax forms read the chunk's range of keys)."""
+    docs = [300, 250, 150, 320]
+    n = sum(docs)
+    m = np.zeros((n, n), dtype=bool)
+    o0 = 0
+    for ln in docs:
+        m[o0:o0 + ln, o0:o0 + ln] = np.tril(np.ones((ln, ln), dtype=bool))
+        o0 += ln
+    rng = np.random.default_rng(61)
+    q, k, v, do = (rng.standard_normal((n, 5)) for _ in range(4))
+    bias = -np.log(np.repeat(np.array(docs, dtype=np.float64), docs))
+    mr = lambda i0, i1: m[i0:i1]
+    cols = np.array([0, 5, 299, 300, 420, 549, 550, 640, 700, 1019])
+    for epi in EPIS:
+        dq, dk, dv = A.head_backward(q, k, v, do, mr, bias, 0.3, epi)
+        dk_s, dv_s = A.key_columns_backward(q, k, v, do, mr, bias, 0.3, epi, cols)
+        np.testing.assert_allclose(dk_s, dk[cols], rtol=1e-11, atol=1e-14)
+        np.testing.assert_allclose(dv_s, dv[cols], rtol=1e-11, atol=1e-14)
+
+
 # ----------------------------------------------------------------------------------------
 # tile list
 # ----------------------------------------------------------------------------------------
