@@ -3,7 +3,8 @@ d=128) and the packed-document mask (B=4, N=8192, H=16, d=128), in the launch co
 bench.py times: the whole batch goes through the CUDA path, and the oracle recomputes
 sampled rows of O and dQ and sampled key rows of dK and dV one by one (tile edges, sequence
 ends and random rows) for a few (batch entry, head) pairs.  Pad rows are checked exactly
-zero over the whole tensors."""
+zero over the whole tensors.  Sigmoid on both; the softmax and softmax_1 epilogues on one
+each (their d = 128 kernels at full size)."""
 import math
 
 import numpy as np
@@ -24,14 +25,16 @@ def _sample_rows(rng, n, count=24):
     return np.array(sorted(set(base + extra)))
 
 
-@pytest.mark.parametrize("cfg", [3, 4])
-def test_full_size_sampled(cfg):
+@pytest.mark.parametrize("cfg,epi", [(3, W.SIGMOID), (4, W.SIGMOID), (3, W.SOFTMAX),
+                                     (4, W.SOFTMAX1)])
+def test_full_size_sampled(cfg, epi):
     from padded_variable_length_b200 import binding as Bd
-    w = W.config(cfg)
+    w = W.config(cfg, epilogue=epi)
     t = W.tensors(w)
     d, plan, bias = Hn.device_setup(w, t)
-    o, _ = Bd.fwd(plan, d["q"], d["k"], d["v"], bias)
-    dq, dk, dv = Bd.bwd(plan, d["q"], d["k"], d["v"], o, d["do"], bias)
+    b_arg = bias if epi == W.SIGMOID else None
+    o, lse = Bd.fwd(plan, d["q"], d["k"], d["v"], b_arg, epi)
+    dq, dk, dv = Bd.bwd(plan, d["q"], d["k"], d["v"], o, d["do"], b_arg, epi, lse=lse)
     assert Bd.get_status() == 0
     # pad rows exactly zero, everywhere
     if w.lengths is not None:
@@ -42,7 +45,7 @@ def test_full_size_sampled(cfg):
         assert torch.isfinite(x).all()
     rng = np.random.default_rng(cfg)
     scale = 1.0 / math.sqrt(w.d)
-    bias_ref = A.bias_from_counts(w.counts)
+    bias_ref = Hn.oracle_bias(w, epi)
     mp = A.mask_provider(w.lengths, w.mask, w.Nq, w.Nk)
     got = {"o": [], "dq": [], "dk": [], "dv": []}
     ref = {"o": [], "dq": [], "dk": [], "dv": []}
@@ -52,9 +55,9 @@ def test_full_size_sampled(cfg):
         rows = _sample_rows(rng, n)
         q, k, v, do = (Hn.to_f64(t[x][b, :, h]) for x in ("q", "k", "v", "do"))
         mr = mp(b)
-        o_ref, _ = A.head_forward(q, k, v, mr, bias_ref[b], scale, A.SIGMOID, rows=rows)
-        dq_ref = A.query_rows_backward(q, k, v, do, mr, bias_ref[b], scale, A.SIGMOID, rows)
-        dk_ref, dv_ref = A.key_columns_backward(q, k, v, do, mr, bias_ref[b], scale, A.SIGMOID, rows)
+        o_ref, _ = A.head_forward(q, k, v, mr, bias_ref[b], scale, epi, rows=rows)
+        dq_ref = A.query_rows_backward(q, k, v, do, mr, bias_ref[b], scale, epi, rows)
+        dk_ref, dv_ref = A.key_columns_backward(q, k, v, do, mr, bias_ref[b], scale, epi, rows)
         got["o"].append(Hn.to_f64(o[b, rows, h]))
         got["dq"].append(Hn.to_f64(dq[b, rows, h]))
         got["dk"].append(Hn.to_f64(dk[b, rows, h]))
