@@ -29,12 +29,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t global_timer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
@@ -214,36 +208,6 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T  (both K-major unless the idesc says MN-major for B)
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem]
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive once on `bar` when every tcgen05 operation issued so far by this thread is done.
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-
 #define SIGATTN_R8(i) "=r"(r[i + 0]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), \
                       "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
 #define SIGATTN_W8(i) "r"(r[i + 0]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), \
@@ -314,18 +278,7 @@ __device__ __forceinline__ void tmem_wait_st() {
 // K-major: rows of 128 bytes (64 bf16 along K), 8-row groups SBO = 1024 bytes apart,
 //   LBO unused (1).  MN-major: 128-byte rows hold 64 consecutive N elements, one row per
 //   K index; 8-row K groups SBO = 1024 apart; 64-wide N chunks LBO apart.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
-                                                    uint32_t sbo_bytes) {
-  uint64_t desc = 0;
-  desc |= static_cast<uint64_t>((saddr & 0x3FFFF) >> 4);
-  desc |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16;
-  desc |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32;
-  desc |= 1ull << 46;
-  desc |= 2ull << 61;
-  return desc;
-}
-
-// The same descriptor split into 32-bit halves, for issue loops that step the start
+// The descriptor is kept as two 32-bit halves, for issue loops that step the start
 // address: lo = start >> 4 | (lbo >> 4) << 16, hi = sbo >> 4 | version | layout.  Adding
 // n to lo moves the start address by 16 n bytes; shared-memory addresses stay below
 // 256 KB, so the 14-bit start field never carries into the offset field.
@@ -457,12 +410,6 @@ __device__ __forceinline__ bool mbar_wait_w(uint64_t* bar, uint32_t parity, cons
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ float rcp_approx(float x) {
-  float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
