@@ -735,8 +735,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    // The whole warp runs the issue loop on warp-uniform values; lane 0 waits on barriers
-    // (the result is broadcast) and an elected lane issues each MMA and commit.
+    // The whole warp runs the issue loop on warp-uniform values: every lane tests or waits
+    // on the barriers and a vote combines them, and an elected lane issues the MMAs (a
+    // tile's S, or its PV, with the commit after them, under one elect.sync).
     {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
