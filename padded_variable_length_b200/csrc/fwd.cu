@@ -755,9 +755,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t v_lo0 = sw128_desc_lo(smem_u32(smem + L::kV), L::kBoxBytes);
       constexpr uint32_t kTileLo = L::kTileBytes >> 4;
       static_assert((SK & (SK - 1)) == 0 && (SV & (SV - 1)) == 0 && NS == 4, "ring sizes");
-      // O += P_x V_x for the oldest tile x of the FIFO (buffer b3 = x % 3), once the
-      // epilogue has finished it; commits step(x)
-      // `ready`: its P and V are known to be in place (tested together with the next K)
+      // O += P_x V_x for the oldest tile x of the FIFO (buffer b3 = x % 3) once the
+      // epilogue has finished it, then commit step(x); `ready` says its P and V are
+      // already known to be in place (tested together with the next K)
       auto pv = [&](int x, uint32_t b3, bool ready) -> bool {
         const int i = pq0 >> 2;
         const bool first = (pq0 & 2) != 0, last = (pq0 & 1) != 0;
