@@ -772,28 +772,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (first && i >= OB && !mbar_wait_w(o_empty + ob, ((i / OB) - 1) & 1, wctx))
           return false;
         tc_fence_after();
-        if constexpr (D == 64) {
-          // Paced: a tcgen05.mma that finds the tensor pipe's queue full holds the issuing
-          // SM sub-partition (and the two epilogue warps beside this warp) until there is
-          // room.  The PV of a d = 64 tile is eight short MMAs (32 tensor cycles each) right
-          // before S: issued four at a time with a short sleep between, the queue keeps room
-          // and the neighbours keep issuing (measured 4 % on the single-cell batch; d = 128,
-          // whose MMAs are twice as long and whose epilogue has more slack, is better off
-          // unpaced).
-          const uint32_t o_tmem = tmem + L::kOCol + ob * D, p_tmem = tmem + b3 * 128;
-          const uint32_t v_lo = v_lo0 + sv * kTileLo;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            if (kk == 4) __nanosleep(64);
-            mma_ts_lh_w(o_tmem, p_tmem + (kk >> 2) * 64 + (kk & 3) * 8, v_lo + kk * 128, kHiMn,
-                        idesc_pv, (first && kk == 0) ? 0u : 1u);
-          }
-          mma_commit_w(step + (x & 3));
-          __nanosleep(64);
-        } else {
-          mma_pv8_commit_w(tmem + L::kOCol + ob * D, tmem + b3 * 128, v_lo0 + sv * kTileLo,
-                           kHiMn, idesc_pv, first ? 0u : 1u, step + (x & 3));
-        }
+        mma_pv8_commit_w(tmem + L::kOCol + ob * D, tmem + b3 * 128, v_lo0 + sv * kTileLo,
+                         kHiMn, idesc_pv, first ? 0u : 1u, step + (x & 3));
         if (last) mma_commit_w(o_full + ob);
         return true;
       };
@@ -924,16 +904,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(m_empty + ms);
         tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c < 3) tmem_ld32(sp + 32 * (c + 1), buf[(c + 1) & 1]);
-          const uint32_t mw = c == 0 ? mb.x : (c == 1 ? mb.y : (c == 2 ? mb.z : mb.w));
+        // one chunk: sigma of 32 columns from b, P into 16 columns at `dst`
+        auto chunk = [&](const uint32_t (&b)[32], uint32_t mw, uint32_t dst) {
           uint32_t pk[16];
 #pragma unroll
           for (int cc = 0; cc < 32; cc += 2) {
-            float2 x = fma2(make_float2(__uint_as_float(buf[c & 1][cc]),
-                                        __uint_as_float(buf[c & 1][cc + 1])),
-                            c1, c0);
+            float2 x = fma2(make_float2(__uint_as_float(b[cc]), __uint_as_float(b[cc + 1])), c1, c0);
             if (masked) {
               x.x = ((mw >> cc) & 1u) ? x.x : -INFINITY;
               x.y = ((mw >> (cc + 1)) & 1u) ? x.y : -INFINITY;
@@ -941,8 +917,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 pw = sigmoid2(x);
             pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
           }
-          tmem_st16(sp + (c >> 1) * 64 + (c & 1) * 16, pk);
-          if (c < 3) tmem_wait_ld();
+          tmem_st16(dst, pk);
+        };
+        // chunks c2 and c2 + 1 per pass (buffers 0 and 1); a loop, not unrolled, keeps the
+        // epilogue's code small
+#pragma unroll 1
+        for (int c2 = 0; c2 < 4; c2 += 2) {
+          tmem_ld32(sp + 32 * (c2 + 1), buf[1]);
+          chunk(buf[0], c2 == 0 ? mb.x : mb.z, sp + (c2 >> 1) * 64);
+          tmem_wait_ld();
+          if (c2 == 0) tmem_ld32(sp + 64, buf[0]);
+          chunk(buf[1], c2 == 0 ? mb.y : mb.w, sp + (c2 >> 1) * 64 + 16);
+          if (c2 == 0) tmem_wait_ld();
         }
         tmem_wait_st();
         tc_fence_before();

@@ -455,6 +455,15 @@ __device__ __forceinline__ float2 mul2_sat(float2 a, float2 b) {
   return d;
 }
 
+// a + b clamped to [0, 1] (NaN gives 0), two scalar adds as mul2_sat
+__device__ __forceinline__ float2 add2_sat(float2 a, float2 b) {
+  float2 d;
+  asm("add.rn.sat.f32 %0, %2, %4;\n\tadd.rn.sat.f32 %1, %3, %5;"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // Packs two floats into bf16x2 (round to nearest even); `lo` lands in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
@@ -491,29 +500,28 @@ __device__ __forceinline__ void sigmoid_parts2(float2 t, float2& e, float2& g) {
   g = fma2(a, e, make_float2(kSigG0, kSigG0));
 }
 
-// sigma from e and g without a compare-and-select (which would load the ALU pipe, the
-// busiest pipe of the sigmoid epilogues): with h = e g (the sigmoid of -|x|) and
-// c = saturate(t 2^126), which is 0 for t <= 0 and 1 for t > 2^-126 (where e rounds to 1),
-// sigma = h + c (g - h): h for x < 0 and g for x >= 0, on the FMA pipe only.
-__device__ __forceinline__ float2 sigmoid_select2(float2 t, float2 g, float2 h) {
+// sigma from t, e and g without a compare-and-select (which would load the ALU pipe, the
+// busiest pipe of the sigmoid epilogues): sigma = g m with m = 1 for x >= 0 and m = e for
+// x < 0.  c = saturate(t 2^126) is 0 for t <= 0 and 1 for t > 2^-126 (values in between
+// occur only where e rounds to 1), so m = saturate(e + c): three FMA-pipe operations.
+__device__ __forceinline__ float2 sigmoid_select2(float2 t, float2 e, float2 g) {
   const float2 c = mul2_sat(t, make_float2(0x1p126f, 0x1p126f));
-  return fma2(c, sub2(g, h), h);
+  return mul2(g, add2_sat(e, c));
 }
 
 // sigma(x) for two elements given t = x log2(e) (t = -inf for a masked element: 0).
 __device__ __forceinline__ float2 sigmoid2(float2 t) {
   float2 e, g;
   sigmoid_parts2(t, e, g);
-  return sigmoid_select2(t, g, mul2(e, g));
+  return sigmoid_select2(t, e, g);
 }
 
 // sigma(x) and sigma'(x) = sigma (1 - sigma) = e g^2 for two elements, t as in sigmoid2.
 __device__ __forceinline__ void sigmoid_grad2(float2 t, float2& p, float2& dp) {
   float2 e, g;
   sigmoid_parts2(t, e, g);
-  const float2 h = mul2(e, g);
-  p = sigmoid_select2(t, g, h);
-  dp = mul2(h, g);
+  p = sigmoid_select2(t, e, g);
+  dp = mul2(mul2(e, g), g);
 }
 
 }  // namespace sigattn
