@@ -21,6 +21,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -1716,53 +1717,56 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         // chunk c.  P and dS of chunk c overwrite its own S^T columns [16c, 16c+16): P in
         // the first 8, dS in the last 8.
         uint32_t sr[2][16], dpr[2][16];
+        uint32_t dsr[4][8];  // dS of the four chunks, kept for the shared-memory copy
         tmem_ld16(xb, sr[0]);
         tmem_ld16(yb, dpr[0]);
         tmem_wait_ld();
+        // the chunk loop, in two versions: with the PARTIAL bitmask, and without
+        auto chunks = [&](auto masked_tag) {
+          constexpr bool kMasked = decltype(masked_tag)::value;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c < 3) {
-            tmem_ld16(xb + 16 * (c + 1), sr[(c + 1) & 1]);
-            tmem_ld16(yb + 16 * (c + 1), dpr[(c + 1) & 1]);
-          }
-          const uint32_t mw = (c < 2 ? mb.x : mb.y) >> (16 * (c & 1));
-          uint32_t pk[8], dk[8];
+          for (int c = 0; c < 4; ++c) {
+            if (c < 3) {
+              tmem_ld16(xb + 16 * (c + 1), sr[(c + 1) & 1]);
+              tmem_ld16(yb + 16 * (c + 1), dpr[(c + 1) & 1]);
+            }
+            const uint32_t mw = (c < 2 ? mb.x : mb.y) >> (16 * (c & 1));
+            uint32_t pk[8];
+            uint32_t (&dk)[8] = dsr[c];
 #pragma unroll
-          for (int cc = 0; cc < 16; cc += 2) {
-            float2 pw, ds;
-            const float2 off2 = *reinterpret_cast<const float2*>(vs + 16 * c + cc);
-            const float2 D2 = EPI == 0 ? make_float2(0.0f, 0.0f)
-                                       : *reinterpret_cast<const float2*>(vs + 128 + 16 * c + cc);
-            weight_grad2<EPI>(
-                make_float2(__uint_as_float(sr[c & 1][cc]), __uint_as_float(sr[c & 1][cc + 1])),
-                make_float2(__uint_as_float(dpr[c & 1][cc]), __uint_as_float(dpr[c & 1][cc + 1])),
-                c1, off2, D2, (mw >> cc) & 1u, (mw >> (cc + 1)) & 1u, pw, ds);
-            pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
-            dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+            for (int cc = 0; cc < 16; cc += 2) {
+              float2 pw, ds;
+              const float2 off2 = *reinterpret_cast<const float2*>(vs + 16 * c + cc);
+              const float2 D2 = EPI == 0 ? make_float2(0.0f, 0.0f)
+                                         : *reinterpret_cast<const float2*>(vs + 128 + 16 * c + cc);
+              weight_grad2<EPI>(
+                  make_float2(__uint_as_float(sr[c & 1][cc]), __uint_as_float(sr[c & 1][cc + 1])),
+                  make_float2(__uint_as_float(dpr[c & 1][cc]), __uint_as_float(dpr[c & 1][cc + 1])),
+                  c1, off2, D2, !kMasked || ((mw >> cc) & 1u) != 0,
+                  !kMasked || ((mw >> (cc + 1)) & 1u) != 0, pw, ds);
+              pk[cc >> 1] = pack_bf16x2(pw.x, pw.y);
+              dk[cc >> 1] = pack_bf16x2(ds.x, ds.y);
+            }
+            tmem_st8(xb + 16 * c, pk);
+            tmem_st8(xb + 16 * c + 8, dk);
+            if (c < 3) tmem_wait_ld();
+            if (c == 2) {
+              // every dP^T column read: the next tile's dP^T may go into Y
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(y_free);
+            }
           }
-          tmem_st8(xb + 16 * c, pk);
-          tmem_st8(xb + 16 * c + 8, dk);
-          if (c < 3) tmem_wait_ld();
-          if (c == 2) {
-            // every dP^T column read: the next tile's dP^T may go into Y
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(y_free);
-          }
-        }
+        };
+        if (meta_kind[s] == 2) chunks(std::true_type{});
+        else chunks(std::false_type{});
         // dS into shared memory for the dQ MMA, once dQ of the previous tile has read it:
         // row = key, 64 queries of this warpgroup, 128-byte swizzled (16-byte chunk j of row
-        // k at position j ^ (k % 8)).  The values are read back from TMEM rather than kept
-        // in registers across the wait.
+        // k at position j ^ (k % 8)), from the registers that also went to TMEM.
         if (t >= 1) ok = mbar_wait(dq_full + ((t - 1) & 1), ((t - 1) >> 1) & 1, wctx);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) break;
         {
-          uint32_t dsr[4][8];
-          tmem_wait_st();
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld8(xb + 16 * c + 8, dsr[c]);
-          tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const uint32_t* w = &dsr[j >> 1][4 * (j & 1)];
