@@ -335,8 +335,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if os.path.exists(tpath):
         with open(tpath) as f:
             tr = json.load(f)
-        key = f"{dom}|{args.config}|{args.epilogue}"
-        traffic = tr.get(key)
+        # the mask families and the reduced (--batch) captures have no entry of their own
+        key = f"{dom}|{args.mask or args.config}|{args.epilogue}"
+        traffic = None if args.batch else tr.get(key)
     roofline = {"bound": "tensor", "kernel": dom, "achieved": kernels[dom]["tflops"],
                 "peak": peak_tf, "unit": "TFLOP/s", "frac": kernels[dom]["tflops"] / peak_tf,
                 "peak_source": f"{peak_src} burst bf16 (cuBLAS)", "traffic": traffic}
