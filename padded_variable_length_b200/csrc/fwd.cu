@@ -30,6 +30,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "internal.h"
@@ -57,6 +58,7 @@ struct FwdParams {
   int QT, Nq, H;
   int nitems;  // B QT H items: (q-tile row, head), in the order of the longest-first list
   int nwork;   // the first nwork items have tiles; the rest are empty
+  int zero_tma;  // sigmoid kernel: zero rows of the empty items by tensor-map stores of O
   float scale;
   const float* bias;
   int64_t bias_sb;
@@ -134,7 +136,9 @@ struct ItemIter {
 // q-tiles past their sequence's length, or whose rows see no key (and, for the softmax
 // modes, LSE = -inf resp. 0 there).  The items are dealt round-robin to every epilogue warp
 // of the grid, one item per warp at a time, with no dependent loads between them; run
-// before the first tile, while the epilogue would otherwise wait for its first S.
+// before the first tile, while the epilogue would otherwise wait for its first S.  The
+// sigmoid kernel uses this for packed layouts only: on padded ones its tile-kind producer
+// writes these rows with tensor-map stores in the background.
 template <int D, int EPI>
 __device__ void zero_empty_items(const FwdParams& p, int ew, int lane) {
   constexpr int kChunks = D / 8;
@@ -561,7 +565,8 @@ struct SigLayout {
   static constexpr int kQ = 0;
   static constexpr int kK = 2 * kTileBytes;
   static constexpr int kV = kK + kKStages * kTileBytes;
-  static constexpr int kMetaBits = kV + kVStages * kTileBytes;
+  static constexpr int kZero = kV + kVStages * kTileBytes;  // a 64-column box of zeros
+  static constexpr int kMetaBits = kZero + kBoxBytes;
   static constexpr int kMetaKind = kMetaBits + kMStages * 2048;
   static constexpr int kBar = kMetaKind + 16 * ((kMStages * 4 + 15) / 16);
   // q_full[2] q_empty[2] o_full[2] o_empty[2] e_done[4] done, s_ready[kSteps],
@@ -576,7 +581,8 @@ struct SigLayout {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sigmoid_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                       const __grid_constant__ CUtensorMap tv, const FwdParams p) {
+                       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                       const FwdParams p) {
   using L = SigLayout<D>;
   constexpr int SK = L::kKStages, SV = L::kVStages, SM = L::kMStages, NS = L::kSteps;
   constexpr int OB = L::kOBufs;
@@ -628,6 +634,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     *drain_flag = 0;
     fence_barrier_init();
   }
+  if (p.zero_tma) {
+    uint4* z = reinterpret_cast<uint4*>(smem + L::kZero);
+    for (int i = threadIdx.x; i < L::kBoxBytes / 16; i += kThreads) z[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
   __syncwarp();
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -654,6 +665,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const CUtensorMap* map = role == 0 ? &tk : &tv;
     int t = 0, i = 0;
     bool ok = true;
+    // meta producer, lane 0: the zero rows of this CTA's empty items (items nwork +
+    // blockIdx.x + k gridDim.x), one item after each tile it produces, as tensor-map stores
+    // of a box of zeros; the next item's descriptor is loaded one store ahead.
+    int zw = p.nwork + static_cast<int>(blockIdx.x);
+    const bool zeroing = p.zero_tma && role == 2 && lane == 0;
+    int4 zd = make_int4(0, 0, 0, 0);
+    if (zeroing && zw < p.nitems) zd = p.row_desc[zw / p.H];
+    auto zero_one = [&]() {
+      if (!zeroing || zw >= p.nitems) return;
+      const int b = zd.x / p.QT, qt = zd.x % p.QT, h = zw % p.H;
+#pragma unroll
+      for (int x = 0; x < L::kBoxes; ++x) tma_store_4d(&to, smem + L::kZero, x * 64, qt * kTile, h, b);
+      bulk_commit_group();
+      zw += static_cast<int>(gridDim.x);
+      if (zw < p.nitems) zd = p.row_desc[zw / p.H];
+    };
     for (ItemIter iter(p); ok && iter.valid(); iter.advance()) {
       const Item it = iter.cur;
       if (it.n == 0) continue;
@@ -716,6 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else {
                   mbar_arrive(full + s);
                 }
+                zero_one();
               }
             }
           }
@@ -726,6 +754,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         rb += used;
       }
     }
+    if (ok)
+      while (zeroing && zw < p.nitems) zero_one();
+    if (zeroing) bulk_wait_all();  // the stores have read the box before shared memory goes
     if (lane == 0 && *abort_flag) {
       // Let the copies still in flight land before the CTA's shared memory goes away.
       const WaitCtx drain{p.status, kDrainWaitNs, drain_flag};
@@ -874,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
     };
-    zero_empty_items<D, 0>(p, warp - kEpiWarp0, lane);
+    if (!p.zero_tma) zero_empty_items<D, 0>(p, warp - kEpiWarp0, lane);
     int t = 0, i = 0;
     ItemIter iter(p);
     float bias_cur = iter.valid() ? row_bias(iter.cur) : 0.0f;
@@ -959,7 +990,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D>
 int launch_fwd_sigmoid_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
-                         const CUtensorMap& tv, cudaStream_t stream) {
+                         const CUtensorMap& tv, const CUtensorMap& to, cudaStream_t stream) {
   using L = SigLayout<D>;
   static_assert(L::kAlloc <= 227 * 1024, "shared memory");
   auto kern = fwd_sigmoid_kernel<D>;
@@ -967,7 +998,7 @@ int launch_fwd_sigmoid_t(const FwdParams& p, const CUtensorMap& tq, const CUtens
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return cuda_status(e);
   const int grid = std::min(p.nitems, num_sms());
-  kern<<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
+  kern<<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -992,6 +1023,7 @@ int launch_fwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.H = H;
   p.nitems = plan->B * plan->QT * H;
   p.nwork = plan->rows_nonempty * H;
+  p.zero_tma = 0;
   p.scale = scale;
   p.bias = bias;
   p.bias_sb = bias_sb;
@@ -1003,7 +1035,13 @@ int launch_fwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.status = status;
   p.wait_ns = wait_ns;
   if constexpr (EPI == 0) {
-    return launch_fwd_sigmoid_t<D>(p, tq, tk, tv, stream);
+    // padded layouts: the zero rows of the empty items go out as tensor-map stores (rows
+    // past the tensor's extent are clipped); packed ones keep the per-row stores, which
+    // stop at each sequence's end
+    CUtensorMap to;
+    std::memset(&to, 0, sizeof(to));
+    p.zero_tma = (plan->cu == nullptr && make_tmap_bf16(&to, o, plan->B, H, D) == SIGATTN_OK) ? 1 : 0;
+    return launch_fwd_sigmoid_t<D>(p, tq, tk, tv, to, stream);
   } else {
     auto kern = fwd_kernel<D, EPI>;
     cudaError_t e =

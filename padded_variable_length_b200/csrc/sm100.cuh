@@ -147,6 +147,17 @@ __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const 
       : "memory");
 }
 
+// Tiled bulk store shared -> global through a tensor map (rows and columns past the
+// tensor's extent are not written); same completion rules as tma_reduce_add_4d.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* smem_src, int x,
+                                             int y, int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group"
+      " [%0, {%1, %2, %3, %4}], [%5];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(smem_src))
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
