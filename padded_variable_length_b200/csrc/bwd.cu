@@ -1855,22 +1855,26 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 }
 
 // Zeroes the fp32 dQ accumulator rows of every q-tile that has tiles (the others are never
-// read): rows qt*128 .. of batch entry b for each listed row r = b*QT + qt.
+// read): rows qt*128 .. of batch entry b for each listed row r = b*QT + qt.  Block
+// (k, part) takes part `part` of listed row k's span (one contiguous range of the
+// [B, Nq, H, 64] accumulator), four 16-byte stores per thread in flight.
+constexpr int kZeroParts = 8;
 __global__ void dq_zero_kernel(const int4* __restrict__ row_desc, int QT, int Nq, int H,
                                float* __restrict__ dqacc) {
-  // one block per listed q-tile (the first rows_nonempty entries of the sorted row list):
-  // its rows are one contiguous span of the [B, Nq, H, 64] accumulator
   const int r = row_desc[blockIdx.x].x;
   const int b = r / QT, qt = r % QT;
   const int rows = min(kTile, Nq - qt * kTile);
   float4* base = reinterpret_cast<float4*>(
       dqacc + (static_cast<int64_t>(b) * Nq + static_cast<int64_t>(qt) * kTile) * H * 64);
   const int n = rows * H * 16;  // float4 per row: 64 H / 4
-  for (int i = threadIdx.x; i < n; i += blockDim.x) base[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  const int per = (n + kZeroParts - 1) / kZeroParts;
+  const int i0 = blockIdx.y * per, i1 = min(n, i0 + per);
+  for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) base[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 }
 
-// dQ = bf16(scale * dQacc) on rows of q-tiles with tiles, 0 on every other row.  One block
-// per (q-tile, sequence); one thread per 8 elements (16 bytes of dQ) of the tile's rows.
+// dQ = bf16(scale acc) on the rows of the listed q-tiles, 0 on the others: one block per
+// (q-tile, batch entry); each thread converts four 8-column pieces at a time, all loads
+// issued before the stores.
 __global__ void dq_convert_kernel(const int32_t* __restrict__ row_ptr, const float* __restrict__ dqacc,
                                   int QT, int Nq, int H, const int32_t* __restrict__ cu,
                                   float scale, __nv_bfloat16* __restrict__ dq, int64_t sb, int64_t sn,
@@ -1883,19 +1887,35 @@ __global__ void dq_convert_kernel(const int32_t* __restrict__ row_ptr, const flo
   const bool listed = row_ptr[r + 1] > row_ptr[r];
   const int per_row = H * 8;
   const int n = rows * per_row;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const int rr = i / per_row, hc = i - rr * per_row;
-    const int h = hc >> 3, c = hc & 7;
-    const int q = qt * kTile + rr;
-    uint4 out = make_uint4(0u, 0u, 0u, 0u);
-    if (listed) {
-      const float4* src = reinterpret_cast<const float4*>(
-          dqacc + ((static_cast<int64_t>(b) * Nq + q) * H + h) * 64 + c * 8);
-      const float4 a = src[0], e = src[1];
-      out = make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
-                       pack_bf16x2(e.x * scale, e.y * scale), pack_bf16x2(e.z * scale, e.w * scale));
+  constexpr int kU = 4;
+  for (int i0 = threadIdx.x; i0 < n; i0 += kU * blockDim.x) {
+    float4 a[kU], e[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * blockDim.x;
+      a[u] = e[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (listed && i < n) {
+        const int rr = i / per_row, hc = i - rr * per_row;
+        const float4* src = reinterpret_cast<const float4*>(
+            dqacc + ((static_cast<int64_t>(b) * Nq + qt * kTile + rr) * H + (hc >> 3)) * 64 +
+            (hc & 7) * 8);
+        a[u] = src[0];
+        e[u] = src[1];
+      }
     }
-    *reinterpret_cast<uint4*>(dq + seq_row_offset(sq, sb, sn, q) + h * sh + c * 8) = out;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < n) {
+        const int rr = i / per_row, hc = i - rr * per_row;
+        *reinterpret_cast<uint4*>(dq + seq_row_offset(sq, sb, sn, qt * kTile + rr) + (hc >> 3) * sh +
+                                  (hc & 7) * 8) =
+            make_uint4(pack_bf16x2(a[u].x * scale, a[u].y * scale),
+                       pack_bf16x2(a[u].z * scale, a[u].w * scale),
+                       pack_bf16x2(e[u].x * scale, e[u].y * scale),
+                       pack_bf16x2(e[u].z * scale, e[u].w * scale));
+      }
+    }
   }
 }
 
@@ -2043,8 +2063,8 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
   }
   const int sms = num_sms();
   if (plan->rows_nonempty > 0) {
-    dq_zero_kernel<<<plan->rows_nonempty, 512, 0, stream>>>(plan->row_desc, plan->QT, plan->Nq,
-                                                             H, dqacc);
+    dq_zero_kernel<<<dim3(plan->rows_nonempty, kZeroParts), 256, 0, stream>>>(
+        plan->row_desc, plan->QT, plan->Nq, H, dqacc);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   static_assert(FusedLayout::kAlloc <= 227 * 1024, "shared memory");
