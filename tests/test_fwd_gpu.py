@@ -104,6 +104,9 @@ def test_strided_views():
     ref, _ = A.forward(Hn.to_f64(t["q"]), Hn.to_f64(t["k"]), Hn.to_f64(t["v"]),
                        Hn.oracle_bias(w, 0), 1 / 8.0, 0, lengths=w.lengths)
     Hn.check_close(Hn.to_f64(o), ref, "O strided", Hn.valid_rows_q(w))
+    # pad rows, including the q-tile of the short sequence that has no tile (written by
+    # tensor-map stores through the view's strides), are exactly zero
+    Hn.check_pad_zero(Hn.to_f64(o), w, "O strided")
     assert torch.all(out_buf[:, :, 0] == 7.0)  # untouched head slot
 
 
