@@ -136,8 +136,9 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m
 
 // 4-D tiled reduce-add shared -> global (element type and box from the tensor map; box
 // rows past the tensor's extent are not written).  Tracked as a bulk async-group of the
-// issuing thread: bulk_commit_group() after it, then bulk_wait_read() before the shared
-// source is rewritten and bulk_wait_all() before the kernel ends.
+// issuing thread: bulk_commit_group() after it, then bulk_wait_read_1() (all but the newest
+// group have read their sources) before a shared source is rewritten, and bulk_wait_all()
+// before the kernel ends.
 __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* smem_src,
                                                   int x, int y, int z, int w) {
   asm volatile(
@@ -160,11 +161,6 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void*
 
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Waits until every committed bulk group of this thread has finished reading its source.
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // Waits until at most one committed bulk group of this thread is still reading its source.
@@ -435,16 +431,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
       "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
       "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
