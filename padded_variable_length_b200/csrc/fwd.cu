@@ -544,8 +544,8 @@ int num_sms() {
 // epilogue has finished tile t - 3.  One commit per MMA group: s_ready (S_t ready, K_t
 // consumed) and step (V_t consumed).
 // Warps: 0 Q/K producer, 1 TMEM allocator + MMA issuer, 2 V producer, 3 kind / bitmask
-// producer, 4-11 two epilogue warpgroups that take alternate tiles (thread = query row =
-// TMEM lane).  The O of an item is written out after the first tile of the next item,
+// producer (and writer of the empty items' zero rows), 4-11 two epilogue warpgroups that
+// take alternate tiles (thread = query row = TMEM lane).  The O of an item is written out after the first tile of the next item,
 // when the last PV of the item has long completed; warpgroup g writes O columns
 // [g d/2, (g+1) d/2).
 // TMEM columns: S/P buffers [0,128), [128,256), [256,384); O in [384,512) (two buffers
@@ -648,9 +648,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 || warp == 2 || warp == 3) {
     // ---------------------------------------------------------------- producers
-    // warp 0: Q of each item and the K ring (slot of tile u free after step u); warp 2:
-    // the V ring (slot of tile u free after step u + 2); warp 3: each tile's kind and
-    // PARTIAL bitmask (slot released by the epilogue).  A row is walked by its runs (ranges
+    // warp 0: Q of each item and the K ring (a slot is free again once the S of the tile
+    // that used it has completed: s_ready); warp 2: the V ring (free once that tile's PV has
+    // completed: step); warp 3: each tile's kind and PARTIAL bitmask (slot released by the
+    // epilogue) and, on padded layouts, the zero rows of this CTA's empty items.  A row is walked by its runs (ranges
     // of consecutive k-tiles of one kind): all 32 lanes fetch the next 32 runs in one round
     // trip, and within a run the k-tile and bitmask number just count up, with no per-tile
     // list lookup.  Lane 0 waits and issues the copies.
