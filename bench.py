@@ -217,13 +217,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             return Bd.Plan.from_lengths(plan_in, w.Nq)
         return Bd.Plan.from_mask(plan_in)
 
-    # plan build time (reported, not part of the step): median of a few builds, each
-    # bracketed by events on the stream (the build synchronises once inside)
-    for _ in range(2):
+    # plan build time (reported, not part of the step): median of 15 builds, each bracketed
+    # by events on the stream (a lengths or mask build returns without waiting for the
+    # device, so the events span its kernels and the host time before the first of them)
+    for _ in range(3):
         build_plan().close()
     torch.cuda.synchronize()
     plan_times = []
-    for _ in range(5):
+    for _ in range(15):
         pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         pe0.record(stream)
         p_ = build_plan()

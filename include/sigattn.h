@@ -96,14 +96,21 @@ typedef struct sigattn_plan_sizes {
 /*
  * Plan for a padded batch: query i of batch entry b sees key j iff i < n_b and
  * j < n_b (Nq = Nk = Npad).  d_lengths: device int32 [B], each in [0, Npad].
- * Builds the tile list on the device and synchronises `stream` once, at the end, to read
- * the counts and the argument checks.  Plan memory: the tile arrays are sized for the
- * worst case (every block listed; for lengths, two PARTIAL tile strips per sequence, for a
- * mask every block PARTIAL at 4 KB each) when that is at most 256 MB, so that nothing waits
- * for the counts; a larger worst case reads the counts back first and sizes the arrays
- * exactly.  On success *out owns device memory until sigattn_plan_destroy.
- * Errors: INVALID (null, B < 1, Npad < 1), UNSUPPORTED (B * QT * KT > 2^28),
- * CUDA, NOMEM.  Lengths outside [0, Npad] are clamped into it.
+ * Builds the tile list on the device: a classification kernel and one cooperative launch
+ * (grid-wide barriers with a time limit) on `stream`.  Plan memory: the tile arrays are
+ * sized for the worst case (every block listed; for lengths, two PARTIAL tile strips per
+ * sequence, for a mask every block PARTIAL at 4 KB each) when that is at most 256 MB (one
+ * allocation, which also keeps the build's scratch: 5 bytes per block of the grid and 8 per
+ * possible PARTIAL block); then the call returns as soon as the work is queued, without waiting for the device: the
+ * attention calls on any stream wait for the build (an event), and
+ * sigattn_plan_get_sizes / the exports wait for it on the host; d_lengths (d_mask) must
+ * stay valid until the build has run on `stream`.  A larger worst case
+ * synchronises `stream` to read the counts, sizes the arrays exactly and synchronises once
+ * more at the end.  On success *out owns device memory until sigattn_plan_destroy.
+ * Errors: INVALID (null, B < 1, Npad < 1), UNSUPPORTED (B * QT * KT > 2^28, or a device
+ * without cooperative launches), CUDA, NOMEM; TIMEOUT (a barrier of the build gave up:
+ * reported by the call when it synchronises, else by sigattn_plan_get_sizes, the exports
+ * and sigattn_get_status).  Lengths outside [0, Npad] are clamped into it.
  */
 SIGATTN_API int sigattn_plan_from_lengths(const int32_t* d_lengths, int B, int Npad, sigattn_stream stream,
                               sigattn_plan** out);
@@ -112,8 +119,7 @@ SIGATTN_API int sigattn_plan_from_lengths(const int32_t* d_lengths, int B, int N
  * Plan for an element mask: d_mask is device uint8 [B, Nq, Nk], nonzero = attend;
  * element (b, i, j) at d_mask[b * stride_b + i * stride_q + j].  The mask is shared by
  * all heads.  Reads the mask once to classify blocks and once more for the PARTIAL
- * blocks' bitmasks.  Synchronises `stream` once; plan memory as for the lengths plan.
- * Errors as for the lengths plan.
+ * blocks' bitmasks.  Asynchrony, plan memory and errors as for the lengths plan.
  */
 SIGATTN_API int sigattn_plan_from_mask(const uint8_t* d_mask, int B, int Nq, int Nk, int64_t stride_b,
                            int64_t stride_q, sigattn_stream stream, sigattn_plan** out);
@@ -128,13 +134,16 @@ SIGATTN_API int sigattn_plan_from_mask(const uint8_t* d_mask, int B, int Nq, int
  * such a plan, every tensor argument of the attention calls is [T, H, d]: pass strides
  * {any, token, head} (the batch stride is ignored), bias is fp32 [T] (bias_stride_b
  * ignored), and lse / the softmax workspace keep their [B, H, max_seqlen] layout.  The plan
- * keeps a copy of cu.  Synchronises `stream` once.  Errors: INVALID (null, B < 1,
- * max_seqlen < 1, a length outside [0, max_seqlen], T < 1), UNSUPPORTED, CUDA, NOMEM.
+ * keeps a copy of cu.  Synchronises `stream` once (the argument checks and T are read on
+ * the host).  Errors: INVALID (null, B < 1, max_seqlen < 1, a length outside
+ * [0, max_seqlen], T < 1), UNSUPPORTED, CUDA, NOMEM, TIMEOUT.
  */
 SIGATTN_API int sigattn_plan_from_cu_seqlens(const int32_t* d_cu, int B, int max_seqlen,
                                              sigattn_stream stream, sigattn_plan** out);
 
-/* Fills *sizes (host struct).  No device work. */
+/* Fills *sizes (host struct).  The first call on a plan whose build returned without
+ * synchronising waits for the build and reads its counts (TIMEOUT if a barrier of the
+ * build gave up); later calls do no device work. */
 SIGATTN_API int sigattn_plan_get_sizes(const sigattn_plan* plan, sigattn_plan_sizes* sizes);
 
 /*

@@ -98,8 +98,16 @@ def _check(rc: int, what: str):
         raise SigattnError(rc, what)
 
 
+# torch's current stream of the current device as a raw handle, without building a Stream
+# object on every call (the public route below is the fallback)
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+_current_device = getattr(torch._C, "_cuda_getDevice", None)
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
+        if _raw_current_stream is not None and _current_device is not None:
+            return _raw_current_stream(_current_device())
         stream = torch.cuda.current_stream()
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
@@ -114,8 +122,18 @@ def _strides(t: torch.Tensor) -> ctypes.Array:
     return _I64x3(t.stride(0), t.stride(1), t.stride(2))
 
 
+def _keep_until_run(t: torch.Tensor, stream):
+    """The plan builds return before the device has read their input: when the build runs
+    on another torch stream than the current one, the caching allocator is told that the
+    input is in use there (on the current stream, stream order already covers it)."""
+    if isinstance(stream, torch.cuda.Stream):
+        t.record_stream(stream)
+
+
 class Plan:
-    """A tile plan (owns device buffers; destroyed with the object)."""
+    """A tile plan (owns device buffers; destroyed with the object).  Lengths and mask
+    plans are built asynchronously on the stream: the attention calls wait for the build,
+    and sizes() / the exports wait for it on the host."""
 
     def __init__(self, handle: int):
         self._h = ctypes.c_void_p(handle)
@@ -125,6 +143,7 @@ class Plan:
         if lengths.dtype != torch.int32 or not lengths.is_cuda or not lengths.is_contiguous():
             raise ValueError("lengths must be a contiguous int32 CUDA tensor")
         h = ctypes.c_void_p()
+        _keep_until_run(lengths, stream)
         _check(_lib.sigattn_plan_from_lengths(lengths.data_ptr(), lengths.numel(), int(npad),
                                               _stream(stream), ctypes.byref(h)), "plan_from_lengths")
         return cls(h.value)
@@ -144,6 +163,7 @@ class Plan:
         if mask.dtype != torch.uint8 or not mask.is_cuda or mask.dim() != 3 or mask.stride(2) != 1:
             raise ValueError("mask must be a uint8 CUDA tensor [B, Nq, Nk] with Nk contiguous")
         h = ctypes.c_void_p()
+        _keep_until_run(mask, stream)
         B, Nq, Nk = mask.shape
         _check(_lib.sigattn_plan_from_mask(mask.data_ptr(), B, Nq, Nk, mask.stride(0), mask.stride(1),
                                            _stream(stream), ctypes.byref(h)), "plan_from_mask")

@@ -38,6 +38,15 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
 
 std::atomic<int> g_last_cuda_error{0};
 
+SymbolAddressCache g_status_addr;
+
+int status_ptr(int** out) {
+  void* p = nullptr;
+  const int rc = g_status_addr.get(g_status_word, &p);
+  *out = static_cast<int*>(p);
+  return rc;
+}
+
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return SIGATTN_OK;
   g_last_cuda_error.store(static_cast<int>(e));
@@ -48,16 +57,6 @@ int cuda_status(cudaError_t e) {
 namespace {
 
 std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
-
-SymbolAddressCache g_status_addr;
-
-// Device address of this device's status word.
-int status_ptr(int** out) {
-  void* p = nullptr;
-  const int rc = g_status_addr.get(g_status_word, &p);
-  *out = static_cast<int*>(p);
-  return rc;
-}
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -192,6 +191,7 @@ extern "C" int sigattn_fwd(const sigattn_plan* plan, int epilogue, int H, int d,
   if ((rc = check_tensor(v, v_strides, rows_k(plan), &tv)) != SIGATTN_OK) return rc;
   if ((rc = check_tensor(o, o_strides, rows_q(plan), &to)) != SIGATTN_OK) return rc;
   if ((rc = check_plan_device(plan)) != SIGATTN_OK) return rc;
+  if ((rc = plan_wait(plan, static_cast<cudaStream_t>(s))) != SIGATTN_OK) return rc;
   int* status = nullptr;
   if ((rc = status_ptr(&status)) != SIGATTN_OK) return rc;
   CUtensorMap mq, mk, mv;
@@ -234,6 +234,7 @@ extern "C" int sigattn_bwd_ex(const sigattn_plan* plan, int epilogue, int H, int
   if ((rc = check_tensor(dk, dk_strides, rows_k(plan), &tdk)) != SIGATTN_OK) return rc;
   if ((rc = check_tensor(dv, dv_strides, rows_k(plan), &tdv)) != SIGATTN_OK) return rc;
   if ((rc = check_plan_device(plan)) != SIGATTN_OK) return rc;
+  if ((rc = plan_wait(plan, static_cast<cudaStream_t>(s))) != SIGATTN_OK) return rc;
   int* status = nullptr;
   if ((rc = status_ptr(&status)) != SIGATTN_OK) return rc;
   CUtensorMap mq, mk, mv, mdo;
@@ -290,6 +291,7 @@ extern "C" int sigattn_bwd_fused(const sigattn_plan* plan, int epilogue, int H, 
   if ((rc = check_tensor(dk, dk_strides, rows_k(plan), &tdk)) != SIGATTN_OK) return rc;
   if ((rc = check_tensor(dv, dv_strides, rows_k(plan), &tdv)) != SIGATTN_OK) return rc;
   if ((rc = check_plan_device(plan)) != SIGATTN_OK) return rc;
+  if ((rc = plan_wait(plan, static_cast<cudaStream_t>(s))) != SIGATTN_OK) return rc;
   int* status = nullptr;
   if ((rc = status_ptr(&status)) != SIGATTN_OK) return rc;
   float* dqacc = static_cast<float*>(workspace);

@@ -47,9 +47,11 @@ struct BwdParams {
   const int4* col_desc;
   const int32_t* cu;  // packed batches: cumulative row offsets [B + 1]; nullptr when padded
   int B, QT, KT, Nq, Nk, H;
-  // items with tiles: the first nwork_cols (k-tile column, head) items of the column list
-  // and the first nwork_rows (q-tile row, head) items of the row list; the rest are empty
-  int nwork_cols, nwork_rows;
+  // items with tiles: the first counts[kCountCols] * H (k-tile column, head) items of the
+  // column list and the first counts[kCountRows] * H (q-tile row, head) items of the row
+  // list; the rest are empty (the plan's device counts: its build need not have been waited
+  // for on the host)
+  const int64_t* counts;
   float scale;
   const float* bias;
   int64_t bias_sb;
@@ -293,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
-  const int nitems = p.B * p.KT * p.H, nwork = p.nwork_cols;
+  const int nitems = p.B * p.KT * p.H, nwork = static_cast<int>(__ldg(p.counts + kCountCols)) * p.H;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* kv_full = bars;
@@ -866,7 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
-  const int nitems = p.B * p.QT * p.H, nwork = p.nwork_rows;
+  const int nitems = p.B * p.QT * p.H, nwork = static_cast<int>(__ldg(p.counts + kCountRows)) * p.H;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* qd_full = bars;
@@ -1423,7 +1425,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
-  const int nitems = p.B * p.KT * p.H, nwork = p.nwork_cols;
+  const int nitems = p.B * p.KT * p.H, nwork = static_cast<int>(__ldg(p.counts + kCountCols)) * p.H;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* kv_full = bars;
@@ -1859,8 +1861,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 // (k, part) takes part `part` of listed row k's span (one contiguous range of the
 // [B, Nq, H, 64] accumulator), four 16-byte stores per thread in flight.
 constexpr int kZeroParts = 8;
-__global__ void dq_zero_kernel(const int4* __restrict__ row_desc, int QT, int Nq, int H,
-                               float* __restrict__ dqacc) {
+__global__ void dq_zero_kernel(const int4* __restrict__ row_desc, const int64_t* __restrict__ counts,
+                               int QT, int Nq, int H, float* __restrict__ dqacc) {
+  if (blockIdx.x >= counts[kCountRows]) return;  // the grid may cover every row
   const int r = row_desc[blockIdx.x].x;
   const int b = r / QT, qt = r % QT;
   const int rows = min(kTile, Nq - qt * kTile);
@@ -1956,8 +1959,7 @@ int launch_bwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.B = plan->B;
   p.QT = plan->QT;
   p.KT = plan->KT;
-  p.nwork_cols = plan->cols_nonempty * H;
-  p.nwork_rows = plan->rows_nonempty * H;
+  p.counts = plan->dcount;
   p.Nq = plan->Nq;
   p.Nk = plan->Nk;
   p.H = H;
@@ -2032,8 +2034,7 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
   p.B = plan->B;
   p.QT = plan->QT;
   p.KT = plan->KT;
-  p.nwork_cols = plan->cols_nonempty * H;
-  p.nwork_rows = plan->rows_nonempty * H;
+  p.counts = plan->dcount;
   p.Nq = plan->Nq;
   p.Nk = plan->Nk;
   p.H = H;
@@ -2062,9 +2063,11 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   const int sms = num_sms();
-  if (plan->rows_nonempty > 0) {
-    dq_zero_kernel<<<dim3(plan->rows_nonempty, kZeroParts), 256, 0, stream>>>(
-        plan->row_desc, plan->QT, plan->Nq, H, dqacc);
+  // one block per listed row: the count is on the device when the host has not read it
+  const int zero_rows = plan->counts_known ? plan->rows_nonempty : plan->B * plan->QT;
+  if (zero_rows > 0) {
+    dq_zero_kernel<<<dim3(zero_rows, kZeroParts), 256, 0, stream>>>(
+        plan->row_desc, plan->dcount, plan->QT, plan->Nq, H, dqacc);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   static_assert(FusedLayout::kAlloc <= 227 * 1024, "shared memory");

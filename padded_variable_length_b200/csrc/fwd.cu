@@ -57,7 +57,9 @@ struct FwdParams {
   int run_cap;      // entries allocated in run (reads stay below it)
   int QT, Nq, H;
   int nitems;  // B QT H items: (q-tile row, head), in the order of the longest-first list
-  int nwork;   // the first nwork items have tiles; the rest are empty
+  // the first counts[kCountRows] * H items have tiles; the rest are empty (the plan's
+  // device counts: its build need not have been waited for on the host)
+  const int64_t* counts;
   int zero_tma;  // sigmoid kernel: zero rows of the empty items by tensor-map stores of O
   float scale;
   const float* bias;
@@ -115,20 +117,21 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p, int w) {
 // item.
 struct ItemIter {
   const FwdParams& p;
+  int nw;        // items with tiles
   int k, w, wn;  // round, this item, next item
   Item cur, nxt;
-  __device__ explicit ItemIter(const FwdParams& pp)
-      : p(pp), k(0), w(snake_item(0)), wn(snake_item(1)) {
-    if (w < p.nwork) cur = decode_item(p, w);
-    if (wn < p.nwork) nxt = decode_item(p, wn);
+  __device__ ItemIter(const FwdParams& pp, int nwork)
+      : p(pp), nw(nwork), k(0), w(snake_item(0)), wn(snake_item(1)) {
+    if (w < nw) cur = decode_item(p, w);
+    if (wn < nw) nxt = decode_item(p, wn);
   }
-  __device__ bool valid() const { return w < p.nwork; }
+  __device__ bool valid() const { return w < nw; }
   __device__ void advance() {
     ++k;
     w = wn;
     wn = snake_item(k + 1);
     cur = nxt;
-    if (wn < p.nwork) nxt = decode_item(p, wn);
+    if (wn < nw) nxt = decode_item(p, wn);
   }
 };
 
@@ -140,10 +143,10 @@ struct ItemIter {
 // sigmoid kernel uses this for packed layouts only: on padded ones its tile-kind producer
 // writes these rows with tensor-map stores in the background.
 template <int D, int EPI>
-__device__ void zero_empty_items(const FwdParams& p, int ew, int lane) {
+__device__ void zero_empty_items(const FwdParams& p, int nwork, int ew, int lane) {
   constexpr int kChunks = D / 8;
   const int stride = static_cast<int>(gridDim.x) * 8;
-  for (int w = p.nwork + static_cast<int>(blockIdx.x) * 8 + ew; w < p.nitems; w += stride) {
+  for (int w = nwork + static_cast<int>(blockIdx.x) * 8 + ew; w < p.nitems; w += stride) {
     const Item x = decode_item(p, w);
     const int rows = min(kTile, x.sq.limit - x.qt * kTile);
     for (int c = lane; c < rows * kChunks; c += 32)
@@ -167,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
+  const int nwork = static_cast<int>(__ldg(p.counts + kCountRows)) * p.H;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* q_full = bars + 0;    // [2]
@@ -227,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     int t = 0, i = 0;
     bool ok = true;
-    for (ItemIter iter(p); ok && iter.valid(); iter.advance()) {
+    for (ItemIter iter(p, nwork); ok && iter.valid(); iter.advance()) {
       const Item it = iter.cur;
       if (it.n == 0) continue;
       const int qb = i & 1;
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       int t = 0, i = 0;
-      for (ItemIter iter(p); ok && iter.valid(); iter.advance()) {
+      for (ItemIter iter(p, nwork); ok && iter.valid(); iter.advance()) {
         const Item it = iter.cur;
         if (it.n == 0) continue;
         const int qb = i & 1;
@@ -376,13 +380,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                  ? p.bias[static_cast<int64_t>(x.sq.tma_b) * p.bias_sb + x.sq.row0 + r]
                  : 0.0f;
     };
-    zero_empty_items<D, EPI>(p, warp - kEpiWarp0, lane);
-    ItemIter iter(p);
+    zero_empty_items<D, EPI>(p, nwork, warp - kEpiWarp0, lane);
+    ItemIter iter(p, nwork);
     float bias_cur = iter.valid() ? row_bias(iter.cur) : 0.0f;
     for (; iter.valid(); iter.advance()) {
       const Item it = iter.cur;
       const float bias_nxt =
-          iter.wn < p.nwork ? row_bias(iter.nxt) : 0.0f;
+          iter.wn < nwork ? row_bias(iter.nxt) : 0.0f;
       const float bias_r = bias_cur;
       bias_cur = bias_nxt;
       if (it.n == 0) continue;  // not in [0, nwork)
@@ -590,6 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
+  const int nwork = static_cast<int>(__ldg(p.counts + kCountRows)) * p.H;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* q_full = bars + 0;
@@ -669,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // meta producer, lane 0: the zero rows of this CTA's empty items (items nwork +
     // blockIdx.x + k gridDim.x), one item after each tile it produces, as tensor-map stores
     // of a box of zeros; the next item's descriptor is loaded one store ahead.
-    int zw = p.nwork + static_cast<int>(blockIdx.x);
+    int zw = nwork + static_cast<int>(blockIdx.x);
     const bool zeroing = p.zero_tma && role == 2 && lane == 0;
     int4 zd = make_int4(0, 0, 0, 0);
     if (zeroing && zw < p.nitems) zd = p.row_desc[zw / p.H];
@@ -682,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       zw += static_cast<int>(gridDim.x);
       if (zw < p.nitems) zd = p.row_desc[zw / p.H];
     };
-    for (ItemIter iter(p); ok && iter.valid(); iter.advance()) {
+    for (ItemIter iter(p, nwork); ok && iter.valid(); iter.advance()) {
       const Item it = iter.cur;
       if (it.n == 0) continue;
       if (role == 0) {
@@ -811,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       int t = 0, i = 0;
       uint32_t b3 = 0;  // t % 3
-      for (ItemIter iter(p); ok && iter.valid(); iter.advance()) {
+      for (ItemIter iter(p, nwork); ok && iter.valid(); iter.advance()) {
         const Item it = iter.cur;
         if (it.n == 0) continue;
         const int qb = i & 1;
@@ -906,15 +911,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
     };
-    if (!p.zero_tma) zero_empty_items<D, 0>(p, warp - kEpiWarp0, lane);
+    if (!p.zero_tma) zero_empty_items<D, 0>(p, nwork, warp - kEpiWarp0, lane);
     int t = 0, i = 0;
-    ItemIter iter(p);
+    ItemIter iter(p, nwork);
     float bias_cur = iter.valid() ? row_bias(iter.cur) : 0.0f;
     for (; ok && iter.valid(); iter.advance()) {
       const Item it = iter.cur;
       // the next item's bias, in flight while this one is processed
       const float bias_nxt =
-          iter.wn < p.nwork ? row_bias(iter.nxt) : 0.0f;
+          iter.wn < nwork ? row_bias(iter.nxt) : 0.0f;
       const float bias_r = bias_cur;
       bias_cur = bias_nxt;
       if (it.n == 0) continue;  // not in [0, nwork)
@@ -1023,7 +1028,7 @@ int launch_fwd_t(const sigattn_plan* plan, int H, float scale, const CUtensorMap
   p.Nq = plan->Nq;
   p.H = H;
   p.nitems = plan->B * plan->QT * H;
-  p.nwork = plan->rows_nonempty * H;
+  p.counts = plan->dcount;
   p.zero_tma = 0;
   p.scale = scale;
   p.bias = bias;

@@ -20,11 +20,19 @@ struct sigattn_plan {
   // and the total number of rows T = cu[B]
   int32_t* cu;
   int64_t T;
-  void* arena[2];  // the two device allocations every buffer below is carved from
+  // the device allocations every buffer below is carved from: one for a plan whose tile
+  // arrays are sized for the worst case (it also holds the build's scratch), else two
+  void* arena[2];
   int B, Nq, Nk, QT, KT;
+  // the counts below are written by the build's kernels into dcount (device, indexed by
+  // sigattn::PlanCount) and copied into these host fields on first use (plan_counts), so
+  // that a build queues its work and returns without waiting for the device
   int64_t nonempty, full, partial;
   int64_t run_cap;  // entries allocated in the per-tile arrays (>= nonempty)
   int32_t rows_nonempty, cols_nonempty;
+  int64_t* dcount;
+  bool counts_known;
+  cudaEvent_t ready;  // recorded after the build's last kernel (nullptr: the build waited)
   int32_t* row_ptr;
   int32_t* col_idx;
   uint8_t* kind;
@@ -51,6 +59,27 @@ struct sigattn_plan {
 namespace sigattn {
 
 constexpr int kTile = 128;
+
+// Slots of a plan's device counts (int64 each): listed tiles, PARTIAL tiles, q-tile rows
+// with tiles, k-tile columns with tiles, the build's barrier-timeout flag, and the arrival
+// counters of the build's grid barriers (two 32-bit counters in one slot).
+enum PlanCount : int {
+  kCountListed = 0,
+  kCountPartial,
+  kCountRows,
+  kCountCols,
+  kCountTimeout,
+  kCountArrive,
+  kCountSlots
+};
+
+// Host copies of the plan's counts: waits for the build (if it has not been waited for),
+// reads the device counts once.  Errors: TIMEOUT (a grid barrier of the build gave up),
+// CUDA.
+int plan_counts(sigattn_plan* plan);
+
+// Makes work queued on `stream` from now on wait for the plan's build.
+int plan_wait(const sigattn_plan* plan, cudaStream_t stream);
 
 // Where the rows of sequence b live.  Padded batches index tensors by (b, row) with a batch
 // stride; a packed batch (a plan built from cumulative offsets cu[0..B]) keeps sequence b in
@@ -90,6 +119,9 @@ int make_tmap_bf16(CUtensorMap* map, const TensorDesc& t, int B, int H, int d);
 int make_tmap_f32_acc(CUtensorMap* map, float* base, int B, int N, int H, int d);
 
 int cuda_status(cudaError_t e);
+
+// Device address of this device's status word (the record of bounded waits that gave up).
+int status_ptr(int** out);
 
 // Per-device cache of the device address of one file-scope __device__ variable.  In host
 // code such a variable's name is only a host-side stand-in, so its address is looked up with
