@@ -809,11 +809,13 @@ int launch_steps(const StepArgs& a, const Src& src, int grid, cudaStream_t strea
 // come from.  np_bound: most PARTIAL blocks the classification can yield (the grid for a
 // mask; two tile strips per sequence for lengths).  When the tile arrays sized for the grid
 // and np_bound fit kOnePassBytes, the classification and one cooperative launch of every
-// later step are queued and the host synchronises once at the end, for the counts and the
-// argument checks; otherwise the launch stops after the counts and the work lists, the host
-// sizes the arrays exactly, and a second launch fills them.  cu_src (packed batches only):
-// the cumulative offsets, copied into the plan; check_dev / check_host: one device int read
-// back at the synchronisation (an argument check).
+// later step are queued, and the call returns without waiting (the counts stay on the
+// device until plan_counts) unless there is a host check to make: packed batches then
+// synchronise once at the end.  Otherwise the launch stops after the counts and the work
+// lists, the host reads the counts, sizes the arrays exactly, and a second launch fills
+// them.  cu_src (packed batches only): the cumulative offsets, copied into the plan;
+// check_dev / check_host: one device int read back at the synchronisation (an argument
+// check).
 template <class ClassifyFn, class Src>
 int build_plan(sigattn_plan* plan, cudaStream_t stream, ClassifyFn classify, const Src& src,
                sigattn_plan** out, int64_t np_bound, const int32_t* cu_src = nullptr,
