@@ -101,12 +101,12 @@ typedef struct sigattn_plan_sizes {
  * sized for the worst case (every block listed; for lengths, two PARTIAL tile strips per
  * sequence, for a mask every block PARTIAL at 4 KB each) when that is at most 256 MB (one
  * allocation, which also keeps the build's scratch: 5 bytes per block of the grid and 8 per
- * possible PARTIAL block); then the call returns as soon as the work is queued, without waiting for the device: the
- * attention calls on any stream wait for the build (an event), and
- * sigattn_plan_get_sizes / the exports wait for it on the host; d_lengths (d_mask) must
- * stay valid until the build has run on `stream`.  A larger worst case
- * synchronises `stream` to read the counts, sizes the arrays exactly and synchronises once
- * more at the end.  On success *out owns device memory until sigattn_plan_destroy.
+ * possible PARTIAL block); then the call returns as soon as the work is queued, without
+ * waiting for the device: the attention calls on any stream wait for the build (an
+ * event), sigattn_plan_get_sizes / the exports wait for it on the host, and
+ * sigattn_plan_destroy releases the memory after it; d_lengths (d_mask) must stay valid
+ * until the build has run on `stream`.  A larger worst case synchronises `stream` to read
+ * the counts, sizes the arrays exactly and synchronises once more at the end.  On success *out owns device memory until sigattn_plan_destroy.
  * Errors: INVALID (null, B < 1, Npad < 1), UNSUPPORTED (B * QT * KT > 2^28, or a device
  * without cooperative launches), CUDA, NOMEM; TIMEOUT (a barrier of the build gave up:
  * reported by the call when it synchronises, else by sigattn_plan_get_sizes, the exports
@@ -183,8 +183,9 @@ SIGATTN_API int sigattn_plan_export_work(const sigattn_plan* plan, int32_t* row_
 SIGATTN_API int sigattn_plan_export_runs(const sigattn_plan* plan, int32_t* run_ptr, int32_t* runs,
                                          int64_t* nruns);
 
-/* Releases the plan's device memory.  Safe on NULL.  The caller must ensure no
- * kernel that uses the plan is still running. */
+/* Releases the plan's device memory, in the order of the legacy default stream and after
+ * the plan's own build.  Safe on NULL.  The caller must ensure that no attention kernel that
+ * uses the plan is still running on a non-blocking stream. */
 SIGATTN_API void sigattn_plan_destroy(sigattn_plan* plan);
 
 /*

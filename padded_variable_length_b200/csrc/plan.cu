@@ -704,9 +704,10 @@ struct Scratch {
   }
 };
 
-// The arenas go back to the pool in the order of the legacy default stream (the caller has
-// made sure that no kernel still uses the plan).
+// The arenas go back to the pool in the order of the legacy default stream, after the
+// plan's build (the caller has made sure that no other kernel still uses the plan).
 void plan_free_buffers(sigattn_plan* p) {
+  if (p->ready && !p->counts_known) cudaStreamWaitEvent(cudaStreamLegacy, p->ready, 0);
   for (void*& a : p->arena) {
     if (a) cudaFreeAsync(a, cudaStreamLegacy);
     a = nullptr;

@@ -63,3 +63,29 @@ def test_plan_build_does_not_wait_and_is_waited_for(kind):
     assert z["rows_nonempty"] == int((np.diff(tl["row_ptr"]) > 0).sum())
     assert z["cols_nonempty"] == int((np.diff(tl["colT_ptr"]) > 0).sum())
     plan.close()
+
+
+def test_destroy_before_the_build_has_run():
+    """A plan destroyed while its build still waits behind a spin on a non-blocking stream:
+    its memory goes back to the pool only after the build, so a plan built next (which may
+    take the same memory) is not overwritten by the late build.  The first plan comes from
+    a different mask, so that a late write would change the second plan's lists."""
+    from padded_variable_length_b200 import binding as Bd
+    rng = np.random.default_rng(74)
+    m_old = W.random_mask(rng, 2, 400, 520, density=0.6, empty_rows=0)
+    w = _workload("mask")
+    old_src = torch.from_numpy(m_old).cuda()
+    new_src = torch.from_numpy(w.mask).cuda()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        torch.cuda._sleep(SPIN_CYCLES)
+        old = Bd.Plan.from_mask(old_src, stream=side)
+    old.close()
+    plan = Bd.Plan.from_mask(new_src)
+    torch.cuda.synchronize()
+    got = plan.export()
+    ref = OT.tile_list(w.mask)
+    for k in ("row_ptr", "col_idx", "kind", "pidx", "colT_ptr", "rowT_idx", "csc_map", "bits"):
+        assert np.array_equal(got[k], ref[k]), f"{k} differs"
+    plan.close()
