@@ -985,7 +985,13 @@ int build_plan(sigattn_plan* plan, cudaStream_t stream, ClassifyFn classify, con
 
 }  // namespace
 
+namespace {
+// Serialises the first read of a plan's counts between host threads that share the plan.
+std::mutex g_counts_mu;
+}  // namespace
+
 int plan_counts(sigattn_plan* plan) {
+  std::lock_guard<std::mutex> lock(g_counts_mu);
   if (plan->counts_known) return SIGATTN_OK;
   int64_t c[kCountSlots] = {};
   int rc = cuda_status(cudaEventSynchronize(plan->ready));
