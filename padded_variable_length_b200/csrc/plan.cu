@@ -1010,7 +1010,14 @@ int plan_counts(sigattn_plan* plan) {
 
 int plan_wait(const sigattn_plan* plan, cudaStream_t stream) {
   if (!plan->ready || plan->counts_known) return SIGATTN_OK;
-  return cuda_status(cudaStreamWaitEvent(stream, plan->ready, 0));
+  // inside a stream capture the wait becomes an external-event node of the graph (the
+  // build's event was recorded outside the capture)
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  int rc = cuda_status(cudaStreamIsCapturing(stream, &cs));
+  if (rc != SIGATTN_OK) return rc;
+  return cuda_status(cudaStreamWaitEvent(
+      stream, plan->ready,
+      cs == cudaStreamCaptureStatusActive ? cudaEventWaitExternal : cudaEventWaitDefault));
 }
 
 namespace {

@@ -38,6 +38,9 @@ def test_plan_build_does_not_wait_and_is_waited_for(kind):
     bias = Bd.bias_from_counts(counts)
     src = (torch.from_numpy(w.lengths.astype(np.int32)) if kind == "lengths"
            else torch.from_numpy(w.mask)).cuda()
+    # one build beforehand: the first use of the planner's kernels loads their module, which
+    # the CUDA runtime may do with a device-wide wait
+    (Bd.Plan.from_lengths(src, w.Nq) if kind == "lengths" else Bd.Plan.from_mask(src)).close()
     torch.cuda.synchronize()
     side = torch.cuda.Stream()
     with torch.cuda.stream(side):
@@ -88,4 +91,35 @@ def test_destroy_before_the_build_has_run():
     ref = OT.tile_list(w.mask)
     for k in ("row_ptr", "col_idx", "kind", "pidx", "colT_ptr", "rowT_idx", "csc_map", "bits"):
         assert np.array_equal(got[k], ref[k]), f"{k} differs"
+    plan.close()
+
+
+def test_graph_captured_with_a_plan_not_yet_waited_for():
+    """A forward captured into a CUDA graph right after an asynchronous build (no sizes()
+    call, so the attention call still has to wait for the build's event): capture succeeds
+    and every replay equals the eager forward."""
+    from padded_variable_length_b200 import binding as Bd
+    w = _workload("lengths")
+    t = W.tensors(w, with_grad=False)
+    d = {k: v.cuda() for k, v in t.items()}
+    counts = torch.from_numpy(np.ascontiguousarray(w.counts, dtype=np.int32)).cuda()
+    bias = Bd.bias_from_counts(counts)
+    src = torch.from_numpy(w.lengths.astype(np.int32)).cuda()
+    torch.cuda.synchronize()
+    plan = Bd.Plan.from_lengths(src, w.Nq)
+    o = torch.empty_like(d["q"])
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        Bd.fwd(plan, d["q"], d["k"], d["v"], bias, W.SIGMOID, out=o)
+    torch.cuda.synchronize()
+    eager, _ = Bd.fwd(plan, d["q"], d["k"], d["v"], bias, W.SIGMOID)
+    for _ in range(2):
+        o.fill_(7.0)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o, eager)
+    assert Bd.get_status() == 0
+    del g
     plan.close()
