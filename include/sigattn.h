@@ -103,7 +103,8 @@ typedef struct sigattn_plan_sizes {
  * allocation, which also keeps the build's scratch: 5 bytes per block of the grid and 8 per
  * possible PARTIAL block); then the call returns as soon as the work is queued, without
  * waiting for the device: the attention calls on any stream wait for the build (an
- * event), sigattn_plan_get_sizes / the exports wait for it on the host, and
+ * event; inside a stream capture, an external-event wait node of the graph),
+ * sigattn_plan_get_sizes / the exports wait for it on the host, and
  * sigattn_plan_destroy releases the memory after it; d_lengths (d_mask) must stay valid
  * until the build has run on `stream`.  A larger worst case synchronises `stream` to read
  * the counts, sizes the arrays exactly and synchronises once more at the end.  On success *out owns device memory until sigattn_plan_destroy.
