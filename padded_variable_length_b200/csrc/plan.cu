@@ -440,7 +440,7 @@ struct LengthSrc {
 };
 
 // Transpose of a 32 x 32 bit matrix held one row per lane (bit c of lane r's word = entry
-// (r, c)): returns column `lane` (bit r = entry (r, lane)).  Five rounds of exchanging the
+// (r, c)): returns column `lane` (bit r = entry (r, lane)).  Five steps, each exchanging the
 // off-diagonal halves of ever smaller blocks between lanes lane and lane ^ j.
 __device__ __forceinline__ uint32_t transpose32(uint32_t x, int lane) {
   constexpr uint32_t kLow[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
