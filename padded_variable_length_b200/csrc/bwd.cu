@@ -1875,23 +1875,28 @@ __global__ void dq_zero_kernel(const int4* __restrict__ row_desc, const int64_t*
   for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) base[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 }
 
-// dQ = bf16(scale acc) on the rows of the listed q-tiles, 0 on the others: one block per
-// (q-tile, batch entry); each thread converts four 8-column pieces at a time, all loads
-// issued before the stores.
+// dQ = bf16(scale acc) on the rows of the listed q-tiles, 0 on the others.  Block
+// (qt * kConvParts + part, b) takes part `part` of the q-tile's 8-column pieces, so that the
+// listed q-tiles (which read the accumulator) spread over the whole GPU instead of a few of
+// them landing twice on one SM; each thread converts four pieces at a time, all loads issued
+// before the stores.
+constexpr int kConvParts = 8;
 __global__ void dq_convert_kernel(const int32_t* __restrict__ row_ptr, const float* __restrict__ dqacc,
                                   int QT, int Nq, int H, const int32_t* __restrict__ cu,
                                   float scale, __nv_bfloat16* __restrict__ dq, int64_t sb, int64_t sn,
                                   int64_t sh) {
-  const int qt = blockIdx.x, b = blockIdx.y;
+  const int qt = blockIdx.x / kConvParts, part = blockIdx.x % kConvParts, b = blockIdx.y;
   const SeqRows sq = seq_rows(cu, b, Nq);
   const int rows = min(kTile, sq.limit - qt * kTile);  // a packed sequence owns only its rows
   if (rows <= 0) return;
   const int r = b * QT + qt;
   const bool listed = row_ptr[r + 1] > row_ptr[r];
   const int per_row = H * 8;
-  const int n = rows * per_row;
+  const int n_all = rows * per_row;
+  const int per = (n_all + kConvParts - 1) / kConvParts;
+  const int i_begin = part * per, n = min(n_all, i_begin + per);
   constexpr int kU = 4;
-  for (int i0 = threadIdx.x; i0 < n; i0 += kU * blockDim.x) {
+  for (int i0 = i_begin + threadIdx.x; i0 < n; i0 += kU * blockDim.x) {
     float4 a[kU], e[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
@@ -2082,7 +2087,7 @@ int launch_bwd_fused_impl(const sigattn_plan* plan, int epilogue, int H, float s
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   {
-    dq_convert_kernel<<<dim3(plan->QT, plan->B), 256, 0, stream>>>(plan->row_ptr, dqacc, plan->QT,
+    dq_convert_kernel<<<dim3(plan->QT * kConvParts, plan->B), 256, 0, stream>>>(plan->row_ptr, dqacc, plan->QT,
                                                                      plan->Nq, H, plan->cu, scale,
                                                    static_cast<__nv_bfloat16*>(const_cast<void*>(dq.ptr)),
                                                    dq.sb, dq.sn, dq.sh);
