@@ -716,15 +716,19 @@ void plan_free_buffers(sigattn_plan* p) {
   p->ready = nullptr;
 }
 
-#define SIGATTN_TRY(x)            \
-  do {                            \
-    const int rc_ = (x);          \
-    if (rc_ != SIGATTN_OK) {      \
-      sc.release(stream);         \
-      plan_free_buffers(plan);    \
-      delete plan;                \
-      return rc_;                 \
-    }                             \
+// On failure: kernels of the build may already be queued on `stream` (which need not be
+// ordered with the legacy stream the plan's memory is freed on), so wait for it first.
+#define SIGATTN_TRY(x)                 \
+  do {                                 \
+    const int rc_ = (x);               \
+    if (rc_ != SIGATTN_OK) {           \
+      cudaStreamSynchronize(stream);   \
+      cudaGetLastError();              \
+      sc.release(stream);              \
+      plan_free_buffers(plan);         \
+      delete plan;                     \
+      return rc_;                      \
+    }                                  \
   } while (0)
 
 #define SIGATTN_TRY_CUDA(x) SIGATTN_TRY(cuda_status(x))
