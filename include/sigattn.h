@@ -31,7 +31,8 @@
  *   - Extents are the caller's promise, as with BLAS leading dimensions: the library
  *     sees pointers and strides only, so every tensor must hold the B x N x H x d (or
  *     T x H x d) elements its strides address, for the plan's B and N; a smaller buffer
- *     is read out of bounds, not reported.
+ *     is read out of bounds, not reported.  (The Python binding compares each tensor's
+ *     shape with the plan's B, Nq, Nk before it calls in, and raises on a short one.)
  *   - bias is fp32 [B, Nq] (per query row; row stride 1, batch stride given); NULL
  *     means 0.  For sigmoid attention the caller fills -log(n), e.g. with
  *     sigattn_bias_from_counts.

@@ -135,8 +135,9 @@ class Plan:
     plans are built asynchronously on the stream: the attention calls wait for the build,
     and sizes() / the exports wait for it on the host."""
 
-    def __init__(self, handle: int):
+    def __init__(self, handle: int, dims=None):
         self._h = ctypes.c_void_p(handle)
+        self._dims = dims  # (B, Nq, Nk, packed) when known on the host at construction
 
     @classmethod
     def from_lengths(cls, lengths: torch.Tensor, npad: int, stream=None) -> "Plan":
@@ -146,7 +147,7 @@ class Plan:
         _keep_until_run(lengths, stream)
         _check(_lib.sigattn_plan_from_lengths(lengths.data_ptr(), lengths.numel(), int(npad),
                                               _stream(stream), ctypes.byref(h)), "plan_from_lengths")
-        return cls(h.value)
+        return cls(h.value, (lengths.numel(), int(npad), int(npad), False))
 
     @classmethod
     def from_cu_seqlens(cls, cu: torch.Tensor, max_seqlen: int, stream=None) -> "Plan":
@@ -156,7 +157,7 @@ class Plan:
         h = ctypes.c_void_p()
         _check(_lib.sigattn_plan_from_cu_seqlens(cu.data_ptr(), cu.numel() - 1, int(max_seqlen),
                                                  _stream(stream), ctypes.byref(h)), "plan_from_cu_seqlens")
-        return cls(h.value)
+        return cls(h.value, (cu.numel() - 1, int(max_seqlen), int(max_seqlen), True))
 
     @classmethod
     def from_mask(cls, mask: torch.Tensor, stream=None) -> "Plan":
@@ -167,11 +168,21 @@ class Plan:
         B, Nq, Nk = mask.shape
         _check(_lib.sigattn_plan_from_mask(mask.data_ptr(), B, Nq, Nk, mask.stride(0), mask.stride(1),
                                            _stream(stream), ctypes.byref(h)), "plan_from_mask")
-        return cls(h.value)
+        return cls(h.value, (B, Nq, Nk, False))
 
     @property
     def handle(self):
         return self._h
+
+    def dims(self):
+        """(B, Nq, Nk, packed): the batch and row extents the plan addresses.  Known on the
+        host from the construction arguments, so this never waits for the build (a Plan
+        wrapped around a raw handle asks sigattn_plan_get_sizes, which may).  For a packed
+        plan Nq = Nk = the longest sequence."""
+        if self._dims is None:
+            z = self.sizes()
+            self._dims = (z["B"], z["Nq"], z["Nk"], False)
+        return self._dims
 
     def sizes(self) -> dict:
         s = PlanSizes()
@@ -248,8 +259,45 @@ def _shape(plan: "Plan", q: torch.Tensor):
     """(B, Nq, H, d): from a padded Q, or from the plan for a packed [T, H, d] Q."""
     if q.dim() == 4:
         return tuple(q.shape)
-    z = plan.sizes()
-    return z["B"], z["Nq"], q.shape[1], q.shape[2]
+    B, Nq, _, _ = plan.dims()
+    return B, Nq, q.shape[1], q.shape[2]
+
+
+def _check_extents(plan: "Plan", q_side, k_side, bias=None, lse=None, workspace=None):
+    """The library sees pointers and strides only: it addresses B x Nq (Q side) and B x Nk
+    (K side) rows of every tensor, B x Nq bias values and B x H x Nq fp32 row statistics,
+    with the plan's B and N.  Raise ValueError, before anything is launched, when a tensor
+    is smaller than that or disagrees with Q in H or d (a larger tensor is fine: rows past
+    the plan's extents are not touched).  Packed [T, H, d] tensors must all have Q's shape."""
+    B, Nq, Nk, packed = plan.dims()
+    q = q_side[0]
+    if packed:
+        if q.dim() != 3:
+            raise ValueError("a packed plan takes [T, H, d] tensors")
+        for t in list(q_side) + list(k_side):
+            if t.dim() != 3 or tuple(t.shape) != tuple(q.shape):
+                raise ValueError(f"packed tensors must all be {tuple(q.shape)}, got {tuple(t.shape)}")
+        H = q.shape[1]
+        if bias is not None and (bias.dim() != 1 or bias.shape[0] < q.shape[0]):
+            raise ValueError(f"bias of a packed plan must be [T] with T >= {q.shape[0]}")
+    else:
+        if q.dim() != 4:
+            raise ValueError("a padded plan takes [B, N, H, d] tensors")
+        H, d = q.shape[2], q.shape[3]
+        for side, n in ((q_side, Nq), (k_side, Nk)):
+            for t in side:
+                if (t.dim() != 4 or t.shape[0] < B or t.shape[1] < n or t.shape[2] != H
+                        or t.shape[3] != d):
+                    raise ValueError(f"tensor {tuple(t.shape)} does not cover the plan's "
+                                     f"[{B}, {n}, {H}, {d}]")
+        if bias is not None and (bias.dim() != 2 or bias.shape[0] < B or bias.shape[1] < Nq):
+            raise ValueError(f"bias {tuple(bias.shape)} does not cover the plan's [{B}, {Nq}]")
+    rows = B * H * Nq
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()
+                            or lse.numel() < rows):
+        raise ValueError(f"lse must be a contiguous fp32 [B, H, Nq] buffer of >= {rows} values")
+    if workspace is not None and workspace.numel() * workspace.element_size() < 4 * rows:
+        raise ValueError(f"workspace must hold >= {rows} fp32 values")
 
 
 def fwd(plan: Plan, q, k, v, bias=None, epilogue: int = SIGMOID, scale: Optional[float] = None,
@@ -262,6 +310,7 @@ def fwd(plan: Plan, q, k, v, bias=None, epilogue: int = SIGMOID, scale: Optional
         out = torch.empty_like(q)
     if epilogue != SIGMOID and lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check_extents(plan, (q, out), (k, v), bias, lse)
     bp, bs = _bias_args(bias)
     _check(_lib.sigattn_fwd(plan.handle, epilogue, H, d, float(scale),
                             q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
@@ -285,6 +334,8 @@ def bwd(plan: Plan, q, k, v, o, do, bias=None, epilogue: int = SIGMOID, lse=None
     dv = torch.empty_like(v) if dv is None else dv
     if epilogue != SIGMOID and workspace is None:
         workspace = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check_extents(plan, [x for x in (q, o, do, dq) if x is not None], (k, v, dk, dv), bias, lse,
+                   workspace)
     bp, bs = _bias_args(bias)
     o_ptr = o.data_ptr() if o is not None else None
     o_str = _strides(o) if o is not None else _I64x3(0, 0, 0)
@@ -320,6 +371,7 @@ def bwd_fused(plan: Plan, q, k, v, o, do, bias=None, epilogue: int = SIGMOID, ls
     if workspace is None:
         workspace = torch.empty((need + 3) // 4, dtype=torch.float32, device=q.device)
     nbytes = workspace.numel() * workspace.element_size()
+    _check_extents(plan, [x for x in (q, o, do, dq) if x is not None], (k, v, dk, dv), bias, lse)
     bp, bs = _bias_args(bias)
     o_ptr = o.data_ptr() if o is not None else None
     o_str = _strides(o) if o is not None else _I64x3(0, 0, 0)
