@@ -80,7 +80,8 @@ enum sigattn_status {
   SIGATTN_ERR_CUDA = -5,        /* a CUDA runtime / driver call failed */
   SIGATTN_ERR_TIMEOUT = -6,     /* a device-side bounded wait expired (see sigattn_get_status) */
   SIGATTN_ERR_NO_DEVICE = -7,   /* no sm_100 device is current */
-  SIGATTN_ERR_NOMEM = -8        /* device allocation failed */
+  SIGATTN_ERR_NOMEM = -8,       /* device allocation failed */
+  SIGATTN_ERR_PLAN = -9         /* a tile list failed a structural check (sigattn_plan_validate) */
 };
 
 /* Sizes of a plan.  QT = ceil(Nq / 128), KT = ceil(Nk / 128). */
@@ -189,6 +190,49 @@ SIGATTN_API int sigattn_plan_export_runs(const sigattn_plan* plan, int32_t* run_
  * the plan's own build.  Safe on NULL.  The caller must ensure that no attention kernel that
  * uses the plan is still running on a non-blocking stream. */
 SIGATTN_API void sigattn_plan_destroy(sigattn_plan* plan);
+
+/*
+ * Debug checks of a tile list (never called by the attention path; a plan the library built
+ * always passes).  The properties are those of the block list of "Binary Block Masking for
+ * FlashAttention", section "Comment ça marche ?" (each row's non-empty blocks, FULL or
+ * PARTIAL with a 128 x 128 block mask), in this library's layout (sigattn_plan_export):
+ *   1 row_ptr   CSR offsets non-decreasing, from 0 to `nonempty`
+ *   2 col_idx   k-tiles in [0, KT), strictly ascending within a row
+ *   3 kind      1 (FULL) or 2 (PARTIAL)
+ *   4 pidx      -1 for FULL; PARTIAL entries numbered 0, 1, ... in CSR order
+ *   5 colT_ptr  CSC offsets as row_ptr
+ *   6 rowT_idx  q-tiles in [0, QT), strictly ascending within a column
+ *   7 csc_map   each CSC entry names the CSR entry of the same (b, q-tile, k-tile)
+ *   8 bits      each PARTIAL bitmask has a set and a clear bit
+ *   9 runs      each row's runs cover its entries in maximal ranges of consecutive k-tiles
+ *               of one kind, {first k-tile, tiles, kind, first entry}
+ *  10 bitsT     (plan only) the transposed bitmasks match the bitmasks
+ *  11 work      (plan only) the longest-first work lists name rows / columns in range with
+ *               non-increasing lengths, and their 16-byte records match the offsets
+ * Both return SIGATTN_OK, or SIGATTN_ERR_PLAN with *first_bad (may be NULL; -1 when the list
+ * passes) = (check number << 40) | index of the failing row, column, entry, bitmask or slot,
+ * the smallest such value found.
+ *
+ * sigattn_plan_validate: checks 1-11 on the plan's device arrays with one kernel on `stream`
+ * and synchronises (it waits for the build first; PARTIAL numbering is checked within each
+ * row).  Allocates and frees 8 bytes of device memory.  Errors: INVALID, SHAPE (the plan
+ * belongs to another device), CUDA, TIMEOUT (the build gave up).
+ *
+ * sigattn_tile_list_check_host: checks 1-9 on HOST arrays sized as the caller says
+ * (nonempty entries, partial * 512 bitmask words, nruns runs of 4 int32; run_ptr NULL skips
+ * check 9), sequentially and with the PARTIAL numbering checked across the whole list.
+ * Needs no GPU.  Errors: INVALID (bad sizes or a needed array NULL).
+ */
+SIGATTN_API int sigattn_plan_validate(const sigattn_plan* plan, sigattn_stream stream,
+                                      int64_t* first_bad);
+SIGATTN_API int sigattn_tile_list_check_host(int B, int QT, int KT, int64_t nonempty,
+                                             int64_t partial, const int32_t* row_ptr,
+                                             const int32_t* col_idx, const uint8_t* kind,
+                                             const int32_t* pidx, const int32_t* colT_ptr,
+                                             const int32_t* rowT_idx, const int32_t* csc_map,
+                                             const uint32_t* bits, const int32_t* run_ptr,
+                                             const int32_t* runs, int64_t nruns,
+                                             int64_t* first_bad);
 
 /*
  * bias[i] = -log(counts[i]) for counts[i] > 0, else 0 (b = -log(n) of "Better Models,

@@ -19,8 +19,9 @@ LIB_PATH = os.path.join(_HERE, "libsigattn.so")
 
 SIGMOID, SOFTMAX, SOFTMAX1 = 0, 1, 2
 OK = 0
+ERR_PLAN = -9  # SIGATTN_ERR_PLAN: a tile list failed a structural check
 ERR = {-1: "INVALID", -2: "UNSUPPORTED", -3: "ALIGNMENT", -4: "SHAPE", -5: "CUDA",
-       -6: "TIMEOUT", -7: "NO_DEVICE", -8: "NOMEM"}
+       -6: "TIMEOUT", -7: "NO_DEVICE", -8: "NOMEM", -9: "PLAN"}
 
 
 class SigattnError(RuntimeError):
@@ -66,6 +67,9 @@ _sig("sigattn_plan_export", ctypes.c_int, _p, _p, _p, _p, _p, _p, _p, _p, _p)
 _sig("sigattn_plan_export_work", ctypes.c_int, _p, _p, _p)
 _sig("sigattn_plan_export_runs", ctypes.c_int, _p, _p, _p, ctypes.POINTER(_i64))
 _sig("sigattn_plan_destroy", None, _p)
+_sig("sigattn_plan_validate", ctypes.c_int, _p, _p, ctypes.POINTER(_i64))
+_sig("sigattn_tile_list_check_host", ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _i64, _i64,
+     _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i64, ctypes.POINTER(_i64))
 _sig("sigattn_bias_from_counts", ctypes.c_int, _p, _i64, _p, _p)
 _sig("sigattn_fwd", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
      _p, _I64x3, _p, _I64x3, _p, _I64x3, _p, _i64, _p, _I64x3, _p, _p)
@@ -224,6 +228,15 @@ class Plan:
                                              ctypes.byref(n)), "plan_export_runs")
         return run_ptr, runs
 
+    def validate(self, stream=None) -> int:
+        """Debug check of the plan's device arrays (sigattn_plan_validate): -1 when every
+        structural property holds, else (check number << 40) | index of the first failure."""
+        where = _i64()
+        rc = _lib.sigattn_plan_validate(self._h, _stream(stream), ctypes.byref(where))
+        if rc not in (OK, ERR_PLAN):
+            _check(rc, "plan_validate")
+        return where.value
+
     def close(self):
         if self._h is not None and self._h.value:
             _lib.sigattn_plan_destroy(self._h)
@@ -234,6 +247,27 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def tile_list_check_host(t: dict, run_ptr=None, runs=None) -> int:
+    """sigattn_tile_list_check_host on host arrays in the export layout (a dict with B, QT,
+    KT, row_ptr, col_idx, kind, pidx, colT_ptr, rowT_idx, csc_map, bits): -1 when the list
+    passes, else (check number << 40) | index of the first failure.  Needs no GPU."""
+    a = {k: np.ascontiguousarray(t[k], dtype=dt) for k, dt in (
+        ("row_ptr", np.int32), ("col_idx", np.int32), ("kind", np.uint8), ("pidx", np.int32),
+        ("colT_ptr", np.int32), ("rowT_idx", np.int32), ("csc_map", np.int32), ("bits", np.uint32))}
+    ptr = lambda x: x.ctypes.data if x is not None and x.size else None
+    rp = None if run_ptr is None else np.ascontiguousarray(run_ptr, dtype=np.int32)
+    ru = None if runs is None else np.ascontiguousarray(runs, dtype=np.int32).reshape(-1, 4)
+    where = _i64()
+    rc = _lib.sigattn_tile_list_check_host(
+        int(t["B"]), int(t["QT"]), int(t["KT"]), a["col_idx"].size, a["bits"].size // 512,
+        *(ptr(a[k]) for k in ("row_ptr", "col_idx", "kind", "pidx", "colT_ptr", "rowT_idx",
+                              "csc_map", "bits")),
+        ptr(rp), ptr(ru), 0 if ru is None else ru.shape[0], ctypes.byref(where))
+    if rc not in (OK, ERR_PLAN):
+        _check(rc, "tile_list_check_host")
+    return where.value
 
 
 def bias_from_counts(counts: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

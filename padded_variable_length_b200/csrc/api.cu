@@ -375,6 +375,7 @@ extern "C" const char* sigattn_error_string(int code) {
     case SIGATTN_ERR_TIMEOUT: return "a device-side bounded wait expired";
     case SIGATTN_ERR_NO_DEVICE: return "no CUDA device is current";
     case SIGATTN_ERR_NOMEM: return "device allocation failed";
+    case SIGATTN_ERR_PLAN: return "the tile list failed a structural check";
     default: return "unknown error code";
   }
 }

@@ -31,6 +31,7 @@ def _setup(lengths, H, d, seed):
     d_pad, plan_pad, bias_pad = Hn.device_setup(w, t)
     cu = torch.from_numpy(np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)).cuda()
     plan = Bd.Plan.from_cu_seqlens(cu, int(lengths.max()))
+    assert plan.validate() == -1  # the library's structural check of the tile list
     packed = {k: _pack(v, lengths) for k, v in d_pad.items()}
     bias = _pack(bias_pad, lengths)
     return w, t, d_pad, plan_pad, bias_pad, packed, plan, bias

@@ -13,6 +13,7 @@ KEYS = ("row_ptr", "col_idx", "kind", "pidx", "colT_ptr", "rowT_idx", "csc_map",
 
 
 def _compare(plan, ref):
+    from padded_variable_length_b200 import binding as Bd
     got = plan.export()
     for k in KEYS:
         assert got[k].shape == ref[k].shape, (k, got[k].shape, ref[k].shape)
@@ -25,6 +26,11 @@ def _compare(plan, ref):
     cols_cnt = np.diff(ref["colT_ptr"])
     assert z["rows_nonempty"] == int((rows_cnt > 0).sum())
     assert z["cols_nonempty"] == int((cols_cnt > 0).sum())
+    # the library's own structural check passes on the device arrays (bitmask transposes,
+    # work lists and runs included) and, on the exported copy, with its host twin
+    assert plan.validate() == -1
+    assert Bd.tile_list_check_host({**got, "B": z["B"], "QT": z["QT"], "KT": z["KT"]},
+                                   *plan.export_runs()) == -1
     rw, cw = plan.export_work()
     for work, cnt in ((rw, rows_cnt), (cw, cols_cnt)):
         assert sorted(work.tolist()) == list(range(len(cnt)))
@@ -201,3 +207,5 @@ def test_plan_large_grid_sizes_after_counting():
         words = np.packbits(dense.reshape(128, 4, 32)[:, :, ::-1], axis=-1, bitorder="big")
         want = words.view(">u4").reshape(128, 4).astype(np.uint32).ravel()
         assert np.array_equal(got["bits"][ref["pidx"][e]], want), f"bits of tile {e}"
+    # every bitmask, its transpose, the runs and the work lists, by the library's own check
+    assert plan.validate() == -1
