@@ -16,7 +16,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <vector>
 
 #include "internal.h"
 
